@@ -1,0 +1,283 @@
+/*
+ * HiLS attention forward pass -- fp64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously correct
+ * statement of what the CUDA path computes.  Only the test suite, the smoke
+ * check and the benchmark's CPU-baseline leg may load it.  It shares no code,
+ * header, table or constant with the CUDA library, and the library never
+ * calls it.
+ *
+ * Sources (the HiLS paper, "Hierarchical Sparse Attention Done Right: Toward
+ * Infinite Context Modeling", as summarised on these pages):
+ *   [HP-Abs]   hotpaper.ai page on the paper, abstract: each query attends
+ *              independently to each retrieved chunk, and the chunk outputs
+ *              are fused according to the chunk retrieval scores.
+ *   [AIT-Meth] aitrends.kr article, section "방법론" (Methodology): the
+ *              landmark query of a chunk attends over the chunk's keys; the
+ *              weighted key sum is the compressed key k'_c and the entropy
+ *              of that distribution is b'_c; the chunk score is
+ *              s^_{i,c} = q_i . k'_c / sqrt(d) + b'_c; the top-K chunks are
+ *              kept and an intra-chunk softmax gives token weights.  Worked
+ *              example: d = 64, q.k'/sqrt(64) = 2.0, b' = 0.7 -> 2.7,
+ *              exp(2.7) ~ 14.9.
+ *   [AIT-Tech] same article, section "기술 상세" (Technical details): the
+ *              first-order Taylor view log sum_j exp(s_j) ~ q.k'_c/sqrt(d)
+ *              + b'_c, with b'_c the entropy of the intra-chunk attention
+ *              distribution; chunk size 64.
+ *   [AIT-Gloss] same article, glossary entry "계층적 소프트맥스"
+ *              (hierarchical softmax): an inter-chunk softmax over the chunk
+ *              scores, then an intra-chunk softmax.
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes of the repository):
+ *   - the landmark softmax uses the same scale 1/sqrt(d) as the chunk score
+ *     (the only choice that makes the Taylor surrogate exact at q = lq);
+ *   - natural logarithm for the entropy;
+ *   - candidates of a query at position i are the chunks c < floor(i/C)
+ *     (fully past); the query's own chunk is always attended under the
+ *     causal mask and enters the fusion with its exact log-sum-exp as score;
+ *   - the fusion softmax runs over the selected chunks and the own chunk
+ *     only;
+ *   - query head hq reads kv head floor(hq / G);
+ *   - top-K ties: the lower chunk id wins; fewer than K candidates: keep
+ *     them all, pad the id list with -1; ids are reported in ascending order.
+ *
+ * Everything is computed in double precision from the exact stored input
+ * values (bf16 and fp32 values are exactly representable in double).
+ *
+ * Layouts (row-major, head_dim innermost):
+ *   K, V  [B, Hkv, N, d]    (N = token capacity)
+ *   LQ    [B, Hkv, N/C, d]  landmark queries
+ *   kp    [B, Hkv, N/C, d]  compressed keys (double)
+ *   bp    [B, Hkv, N/C]     entropy biases (double)
+ * Rows are given explicitly: for row r, its batch rb[r], query head rhq[r],
+ * position rpos[r] and its query vector qrows[r*d .. r*d+d).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct hils_oracle_dims {
+  int64_t B, Hq, Hkv, N, d, C, K;
+} hils_oracle_dims;
+
+static double dot_fd(const float* a, const float* b, int64_t d) {
+  double s = 0.0;
+  for (int64_t t = 0; t < d; ++t) s += (double)a[t] * (double)b[t];
+  return s;
+}
+
+static double dot_fdd(const float* a, const double* b, int64_t d) {
+  double s = 0.0;
+  for (int64_t t = 0; t < d; ++t) s += (double)a[t] * b[t];
+  return s;
+}
+
+/*
+ * Landmark summary of chunks [chunk_begin, chunk_end) of every (b, kv head)
+ * ([AIT-Meth], [AIT-Tech]):
+ *   z_j  = <lq_c, k_j> / sqrt(d)       for the C keys j of chunk c
+ *   p    = softmax(z)
+ *   k'_c = sum_j p_j k_j
+ *   b'_c = -sum_j p_j log p_j          (natural log)
+ * The entropy is evaluated as  log sum_j exp(z_j) - sum_j p_j z_j , which is
+ * the same quantity (log p_j = z_j - LSE(z)) and never takes log(0).
+ */
+void hils_oracle_summary(const hils_oracle_dims* D, const float* K, const float* LQ,
+                         int64_t chunk_begin, int64_t chunk_end, double* kp, double* bp) {
+  const int64_t d = D->d, C = D->C, nc = D->N / D->C;
+  const double tau = 1.0 / sqrt((double)d);
+  const int64_t nbh = D->B * D->Hkv;
+  const int64_t span = chunk_end - chunk_begin;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t u = 0; u < nbh * span; ++u) {
+    const int64_t bh = u / span, c = chunk_begin + u % span;
+    const float* lq = LQ + (bh * nc + c) * d;
+    const float* kc = K + (bh * D->N + c * C) * d;
+    double* z = (double*)malloc(sizeof(double) * (size_t)C);
+    double m = -INFINITY;
+    for (int64_t j = 0; j < C; ++j) {
+      z[j] = tau * dot_fd(lq, kc + j * d, d);
+      if (z[j] > m) m = z[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < C; ++j) Z += exp(z[j] - m);
+    const double lse = m + log(Z);
+    double* out = kp + (bh * nc + c) * d;
+    for (int64_t t = 0; t < d; ++t) out[t] = 0.0;
+    double pz = 0.0;
+    for (int64_t j = 0; j < C; ++j) {
+      const double p = exp(z[j] - m) / Z;
+      pz += p * z[j];
+      for (int64_t t = 0; t < d; ++t) out[t] += p * (double)kc[j * d + t];
+    }
+    bp[bh * nc + c] = lse - pz;
+    free(z);
+  }
+}
+
+/*
+ * Chunk scores of the given rows ([AIT-Meth]):
+ *   s^_{i,c} = <q_i, k'_c> / sqrt(d) + b'_c     for every candidate c < floor(i/C)
+ * out[r, c] = -inf for chunks that are not candidates of row r.
+ */
+void hils_oracle_scores(const hils_oracle_dims* D, const double* kp, const double* bp,
+                        int64_t n_rows, const int32_t* rb, const int32_t* rhq, const int64_t* rpos,
+                        const float* qrows, double* out) {
+  const int64_t d = D->d, nc = D->N / D->C, G = D->Hq / D->Hkv;
+  const double tau = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
+    const int64_t own = rpos[r] / D->C;
+    const float* q = qrows + r * d;
+    for (int64_t c = 0; c < nc; ++c) {
+      out[r * nc + c] = (c < own) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]
+                                  : -INFINITY;
+    }
+  }
+}
+
+typedef struct { double s; int64_t c; } scored_chunk;
+
+static int by_score_desc_id_asc(const void* x, const void* y) {
+  const scored_chunk* a = (const scored_chunk*)x;
+  const scored_chunk* b = (const scored_chunk*)y;
+  if (a->s > b->s) return -1;
+  if (a->s < b->s) return 1;
+  return (a->c < b->c) ? -1 : (a->c > b->c);
+}
+
+static int by_id_asc(const void* x, const void* y) {
+  const scored_chunk* a = (const scored_chunk*)x;
+  const scored_chunk* b = (const scored_chunk*)y;
+  return (a->c < b->c) ? -1 : (a->c > b->c);
+}
+
+/*
+ * Top-K chunk selection ([AIT-Meth]: keep the K chunks of largest score).
+ * Candidates are sorted by (score descending, chunk id ascending) and the
+ * first min(K, #candidates) are kept.  ids[r, :] lists them in ascending chunk
+ * id, padded with -1; sel[r, :] holds their scores (-inf for padding).
+ * gap[r] = (K-th best score) - ((K+1)-th best score), +inf when a row has at
+ * most K candidates.
+ */
+void hils_oracle_select(const hils_oracle_dims* D, const double* kp, const double* bp,
+                        int64_t n_rows, const int32_t* rb, const int32_t* rhq, const int64_t* rpos,
+                        const float* qrows, int32_t* ids, double* sel, double* gap) {
+  const int64_t d = D->d, nc = D->N / D->C, G = D->Hq / D->Hkv, K = D->K;
+  const double tau = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
+    const int64_t n_cand = rpos[r] / D->C;   /* candidates: the fully-past chunks 0 .. n_cand-1 */
+    const float* q = qrows + r * d;
+    scored_chunk* cand = (scored_chunk*)malloc(sizeof(scored_chunk) * (size_t)(n_cand + 1));
+    for (int64_t c = 0; c < n_cand; ++c) {
+      cand[c].s = tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c];
+      cand[c].c = c;
+    }
+    qsort(cand, (size_t)n_cand, sizeof(scored_chunk), by_score_desc_id_asc);
+    const int64_t keep = n_cand < K ? n_cand : K;
+    if (gap) gap[r] = (n_cand > K) ? cand[K - 1].s - cand[K].s : INFINITY;
+    qsort(cand, (size_t)keep, sizeof(scored_chunk), by_id_asc);
+    for (int64_t t = 0; t < K; ++t) {
+      ids[r * K + t] = (t < keep) ? (int32_t)cand[t].c : -1;
+      if (sel) sel[r * K + t] = (t < keep) ? cand[t].s : -INFINITY;
+    }
+    free(cand);
+  }
+}
+
+/*
+ * Softmax attention of query q over keys [j0, j1) of one (b, kv head):
+ * s_j = <q, k_j>/sqrt(d); returns LSE(s) and writes o = sum_j softmax(s)_j v_j.
+ */
+static double attend_keys(const float* q, const float* Kbh, const float* Vbh, int64_t j0, int64_t j1,
+                          int64_t d, double tau, double* s, double* o) {
+  double m = -INFINITY;
+  for (int64_t j = j0; j < j1; ++j) {
+    s[j - j0] = tau * dot_fd(q, Kbh + j * d, d);
+    if (s[j - j0] > m) m = s[j - j0];
+  }
+  double l = 0.0;
+  for (int64_t t = 0; t < d; ++t) o[t] = 0.0;
+  for (int64_t j = j0; j < j1; ++j) {
+    const double e = exp(s[j - j0] - m);
+    l += e;
+    for (int64_t t = 0; t < d; ++t) o[t] += e * (double)Vbh[j * d + t];
+  }
+  for (int64_t t = 0; t < d; ++t) o[t] /= l;
+  return m + log(l);
+}
+
+/*
+ * Hierarchical attention of the given rows ([HP-Abs], [AIT-Meth], [AIT-Gloss]):
+ *   for each selected chunk c (ids[r, :], -1 entries skipped):
+ *       o_c = softmax_j(<q, k_j>/sqrt(d)) V   over the chunk's C keys
+ *       u_c = s^_{i,c}                      (score_mode 0: the surrogate)
+ *           = log sum_j exp(<q,k_j>/sqrt(d))  (score_mode 1: the exact chunk
+ *                                              log-sum-exp; used by the
+ *                                              dense-equivalence pin)
+ *   own chunk o = floor(i/C): keys j in [o*C, i] (causal),
+ *       o_own = softmax V, u_own = exact log-sum-exp of those logits
+ *   w = softmax(u over selected chunks and the own chunk)
+ *   O = sum w_c o_c + w_own o_own
+ * lse_own (nullable) receives u_own.
+ */
+void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* V,
+                        const double* kp, const double* bp,
+                        int64_t n_rows, const int32_t* rb, const int32_t* rhq, const int64_t* rpos,
+                        const float* qrows, const int32_t* ids, int64_t ids_stride, int score_mode,
+                        double* O, double* lse_own) {
+  const int64_t d = D->d, C = D->C, nc = D->N / D->C, G = D->Hq / D->Hkv;
+  const double tau = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 8)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
+    const int64_t i = rpos[r], own = i / C;
+    const float* q = qrows + r * d;
+    const float* Kbh = K + bh * D->N * d;
+    const float* Vbh = V + bh * D->N * d;
+    const int64_t nsel = ids_stride;
+    double* u = (double*)malloc(sizeof(double) * (size_t)(nsel + 1));
+    double* oc = (double*)malloc(sizeof(double) * (size_t)((nsel + 1) * d));
+    double* s = (double*)malloc(sizeof(double) * (size_t)C);
+    int64_t m_used = 0;
+    for (int64_t t = 0; t < nsel; ++t) {
+      const int64_t c = ids[r * ids_stride + t];
+      if (c < 0) continue;
+      const double lse = attend_keys(q, Kbh, Vbh, c * C, (c + 1) * C, d, tau, s, oc + m_used * d);
+      u[m_used] = (score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]
+                                    : lse;
+      ++m_used;
+    }
+    const double lo = attend_keys(q, Kbh, Vbh, own * C, i + 1, d, tau, s, oc + m_used * d);
+    u[m_used] = lo;
+    if (lse_own) lse_own[r] = lo;
+    ++m_used;
+    double M = -INFINITY;
+    for (int64_t t = 0; t < m_used; ++t) if (u[t] > M) M = u[t];
+    double Z = 0.0;
+    for (int64_t t = 0; t < m_used; ++t) Z += exp(u[t] - M);
+    double* out = O + r * d;
+    for (int64_t x = 0; x < d; ++x) out[x] = 0.0;
+    for (int64_t t = 0; t < m_used; ++t) {
+      const double w = exp(u[t] - M) / Z;
+      for (int64_t x = 0; x < d; ++x) out[x] += w * oc[t * d + x];
+    }
+    free(u);
+    free(oc);
+    free(s);
+  }
+}
+
+int hils_oracle_max_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,50 @@
+"""Plant plausible mistakes in copies of the oracle and check that its pins
+(tests/test_oracle.py) reject every one of them.  Runs on the CPU only."""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "hils_oracle.c")
+
+MUTANTS = {
+    "summary_without_scale": ("z[j] = tau * dot_fd(lq, kc + j * d, d);", "z[j] = dot_fd(lq, kc + j * d, d);"),
+    "entropy_sign_flipped": ("bp[bh * nc + c] = lse - pz;", "bp[bh * nc + c] = pz - lse;"),
+    "score_without_bias": ("(c < own) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]",
+                           "(c < own) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d)"),
+    "select_without_bias": ("cand[c].s = tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c];",
+                            "cand[c].s = tau * dot_fdd(q, kp + (bh * nc + c) * d, d);"),
+    "fusion_without_bias": ("(score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]",
+                            "(score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d)"),
+    "fusion_surrogate_unscaled": ("(score_mode == 0) ? tau * dot_fdd(", "(score_mode == 0) ? dot_fdd("),
+    "compressed_key_wrong_index": ("out[t] += p * (double)kc[j * d + t];", "out[t] += p * (double)kc[t * d + j % d];"),
+    "causal_mask_off_by_one": ("own * C, i + 1, d, tau", "own * C, i, d, tau"),
+    "kv_head_mapping_modulo": ("const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;\n    const int64_t i = rpos[r]",
+                               "const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] % D->Hkv;\n    const int64_t i = rpos[r]"),
+    "select_ascending": ("if (a->s > b->s) return -1;\n  if (a->s < b->s) return 1;",
+                         "if (a->s < b->s) return -1;\n  if (a->s > b->s) return 1;"),
+    "own_chunk_is_candidate": ("const int64_t n_cand = rpos[r] / D->C;", "const int64_t n_cand = rpos[r] / D->C + 1;"),
+    "fusion_uniform_weights": ("const double w = exp(u[t] - M) / Z;", "const double w = 1.0 / (double)m_used;"),
+    "fusion_drops_own_chunk": ("u[m_used] = lo;", "u[m_used] = -INFINITY;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site of {name} not unique"
+    with tempfile.TemporaryDirectory() as tmp:
+        cfile = os.path.join(tmp, "mutant.c")
+        lib = os.path.join(tmp, "libmutant.so")
+        open(cfile, "w").write(src.replace(old, new))
+        subprocess.check_call(["gcc", "-O1", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared", "-std=c11",
+                               cfile, "-o", lib, "-lm"])
+        env = dict(os.environ, HILS_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+        r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle.py")],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
