@@ -1,0 +1,356 @@
+"""Benchmark of the HiLS attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of synthetic input
+already resident in HBM: landmark summary (a) -> chunk scoring + top-K (b) ->
+sparse prefill attention with fusion (c) -> one decode step at full length
+(d).  Prints ONE JSON line (rank 0).  For N > 1 (torchrun) every rank runs
+the same independent workload (weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+method: there is no other implementation to run) on a bounded sample of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunk_wise_sparse_b200.inputs import WORKLOADS, generate, sample_rows  # noqa: E402
+
+DEFAULT_WORKLOAD = "prefill-512k-h16-d64"
+METRIC = "HiLS prefill tokens/s (landmark summary + top-K selection + sparse attention, with one decode step)"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained", j["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def useful_work(w):
+    """Algorithmic work of one step (counts documented in the design doc)."""
+    B, Hq, Hkv, N, d, C, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.C, w.K
+    nc = N // C
+    i = np.arange(N, dtype=np.int64)
+    own = i // C
+    keys = np.minimum(K, own) * C + (i % C) + 1
+    flops_score = 2 * d * Hq * B * C * nc * (nc - 1) // 2
+    flops_attn = 4 * d * Hq * B * int(keys.sum())
+    bytes_summary = B * Hkv * nc * (C * d * 2 + d * 2 + 4 * d + 4 + 2 * (d + 16))
+    return dict(flops_score=flops_score, flops_attn=flops_attn, bytes_summary=bytes_summary)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index, self.proc, self.out = index, None, None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for _, _, r in rows for k, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_sample(w, inp, budget_s=15.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
+    the summaries of a head subset plus sampled prefill rows.  Returns
+    (tokens/s, description, threads)."""
+    from oracle.oracle import Oracle, Rows, max_threads
+    o = Oracle.for_workload(w)
+    # summaries: all chunks of one (b, kv head)
+    one = Oracle(1, w.G, 1, w.N, w.d, w.C, w.K)
+    t0 = time.perf_counter()
+    kp1, bp1 = one.summary(inp.k_f32[:1, :1], inp.lq_f32[:1, :1])
+    t_sum_head = time.perf_counter() - t0
+    t_summary = t_sum_head * w.B * w.Hkv
+    kp = np.zeros((w.B, w.Hkv, w.nc, w.d))
+    bp = np.zeros((w.B, w.Hkv, w.nc))
+    kp[0, 0], bp[0, 0] = kp1[0, 0], bp1[0, 0]
+    # rows of head 0 spread over the sequence
+    n = 64
+    elapsed, done = 0.0, 0
+    rng = np.random.default_rng(w.seed + 2000)
+    while elapsed < budget_s and done < w.N:
+        pos = np.sort(rng.choice(w.N, size=n, replace=False))
+        rows = Rows(np.zeros(n), np.zeros(n), pos, inp.q_f32[0, 0, pos] if w.kind != "decode" else
+                    np.repeat(inp.q_f32[:1, 0], n, axis=0))
+        t0 = time.perf_counter()
+        ids, _, _ = o.select(kp, bp, rows)
+        o.attend(inp.k_f32, inp.v_f32, kp, bp, rows, ids)
+        elapsed += time.perf_counter() - t0
+        done += n
+        n = min(2 * n, 4096)
+    t_per_row = elapsed / done
+    t_token = t_summary / w.N + t_per_row * w.Hq * w.B
+    desc = (f"fp64 oracle: summaries of 1 of {w.B * w.Hkv} (b, kv head) slabs ({t_sum_head:.2f} s, scaled), "
+            f"select+attend of {done} sampled rows of head 0 ({elapsed:.1f} s); tokens/s = 1 / (summary "
+            f"time per token + row time x {w.B * w.Hq} rows per token)")
+    return 1.0 / t_token, desc, max_threads()
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    inp = generate(w)
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, inp, budget_s=2.0)
+    for _ in range(args.steps):
+        v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget)
+        vals.append(v)
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.B * w.N / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "C": w.C, "K": w.K,
+            "needles": w.needles, "seed": w.seed, "parallelism": f"dp{n_gpus} (independent replicas)",
+            "l2": "inputs larger than L2 (Q, K, V are each larger than 126 MB); no flush"}
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from chunk_wise_sparse_b200 import hils
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hils.lib()
+    inp = generate(w)
+
+    def to_dev(name):
+        bits = getattr(inp, name + "_bits")
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(getattr(inp, name + "_f32")).to(dev)
+
+    q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
+    B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
+    dims = hils.dims_for(q, k, K)
+    summ = hils.Summary(dims, dev)
+    ids = torch.empty((B, Hq, N, K), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, Hq, N, K), dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    qd = q[:, :, -1, :].contiguous()
+    seq = torch.full((B,), N, dtype=torch.int32, device=dev)
+    ddims = hils.make_dims(B, Hq, Hkv, d, N, K, q.dtype)
+    ws = torch.empty((hils.hils_decode_workspace_bytes(ddims),), dtype=torch.uint8, device=dev)
+    od = torch.empty_like(qd)
+    ids_d = torch.empty((B, Hq, K), dtype=torch.int32, device=dev)
+    sc_d = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        hils.hils_landmark_summary(dims, k, lq, 0, N // 64, summ.kprime, summ.bprime, summ.kprime_mma, stream)
+        if ev: ev[1].record(stream)
+        hils.hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
+        if ev: ev[2].record(stream)
+        hils.hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, stream)
+        if ev: ev[3].record(stream)
+        hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
+                              ws, stream=stream)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hils.hils_get_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = hils.hils_kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = hils.hils_kernel_launches() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # ms per kernel
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = world * B * N / (ms_step / 1e3)
+
+    # end to end through the public API: pinned host inputs -> device -> path -> host result
+    e2e = None
+    if not args.no_e2e:
+        host = {n: getattr(inp, n + "_bits") if getattr(inp, n + "_bits") is not None else getattr(inp, n + "_f32")
+                for n in ("q", "k", "v", "lq")}
+        pinned = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
+                  for n, a in host.items()}
+        dev_t = {"q": q, "k": k, "v": v, "lq": lq}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        od_host = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = o_host.numel() * o_host.element_size() + od_host.numel() * od_host.element_size()
+
+        def e2e_step():
+            for n, t in pinned.items():
+                dev_t[n].view(torch.int16 if dev_t[n].dtype == torch.bfloat16 else dev_t[n].dtype).copy_(
+                    t, non_blocking=True)
+            step()
+            o_host.copy_(o, non_blocking=True)
+            od_host.copy_(od, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(2, min(args.steps, 5))
+        if world > 1:
+            dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a0.elapsed_time(a1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * B * N / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    if rank != 0:
+        return
+
+    work = useful_work(w)
+    peaks = load_peaks()
+    names = ["summary", "select", "prefill", "decode"]
+    avg = per.mean(axis=0)
+    kernels_ms = {n: float(a) for n, a in zip(names, avg)}
+    dom = names[int(np.argmax(avg))]
+    if dom in ("select", "prefill"):
+        fl = work["flops_score"] if dom == "select" else work["flops_attn"]
+        ach = fl / (kernels_ms[dom] / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"] + " bf16 dense burst"}
+    else:
+        by = work["bytes_summary"]
+        ach = by / (kernels_ms[dom] / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"] + " copy"}
+    bc_flops = work["flops_score"] + work["flops_attn"]
+    bc_ms = kernels_ms["select"] + kernels_ms["prefill"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": f"synthetic: i.i.d. N(0,1) Q/K/V/landmark queries, {w.needles} planted needle chunks, seed {w.seed}",
+        "config": workload_config(w, world),
+        "kernels_ms": kernels_ms,
+        "decode_us_per_step": 1e3 * kernels_ms["decode"],
+        "prefill_bc_tflops_useful": bc_flops / (bc_ms / 1e3) / 1e12,
+        "prefill_bc_frac_of_bf16_peak": bc_flops / (bc_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    if w.kind == "decode":
+        raise SystemExit("bench.py times prefill workloads; decode-only workloads are covered by the tests")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

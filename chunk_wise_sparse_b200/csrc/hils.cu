@@ -1,0 +1,236 @@
+// C ABI of the HiLS attention forward library: argument validation, dispatch
+// on (dtype, head_dim) and kernel launches.  See include/hils.h for the
+// contract of every entry point.
+#include <atomic>
+#include <type_traits>
+
+#include "hils.h"
+#include "common.cuh"
+#include "summary.cuh"
+#include "select_simt.cuh"
+#include "attend_simt.cuh"
+#include "decode.cuh"
+
+using namespace hils;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+
+int check_dims(const hils_dims* d) {
+  if (d == nullptr) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->batch < 1 || d->heads_q < 1 || d->heads_kv < 1 || d->heads_q % d->heads_kv != 0)
+    return HILS_ERR_INVALID_ARGUMENT;
+  if (d->seqlen < 1 || d->chunk < 1 || d->reserved != 0) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->dtype != HILS_BF16 && d->dtype != HILS_FP32) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->chunk != kChunk) return HILS_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return HILS_ERR_UNSUPPORTED;
+  if (d->topk < 1 || d->topk > kMaxTopK) return HILS_ERR_UNSUPPORTED;
+  if (d->seqlen % d->chunk != 0) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->seqlen > (int64_t(1) << 31)) return HILS_ERR_UNSUPPORTED;
+  return HILS_OK;
+}
+
+inline int launched(int n) {
+  g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+// cudaFuncSetAttribute for dynamic shared memory, once per (kernel, device).
+template <auto FN>
+cudaError_t set_smem(size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::atomic<uint32_t> done_mask{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint32_t bit = 1u << (dev & 31);
+  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(FN, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <typename T, int D>
+int launch_summary(const hils_dims* d, const void* k, const void* lq, int64_t c0, int64_t c1, float* kp,
+                   float* bp, void* kmma, cudaStream_t st) {
+  const int64_t nc = d->seqlen / kChunk, span = c1 - c0;
+  const int64_t units = int64_t(d->batch) * d->heads_kv * span;
+  const int64_t blocks = (units * 32 + 255) / 256;
+  summary_kernel<T, D><<<dim3(unsigned(blocks)), 256, 0, st>>>(
+      static_cast<const T*>(k), static_cast<const T*>(lq), d->seqlen, nc, c0, span, units, kp, bp,
+      static_cast<__nv_bfloat16*>(kmma), 1.f / sqrtf(float(D)));
+  return launched(1);
+}
+
+template <typename T, int D, bool MMA>
+int launch_select_simt(const hils_dims* d, const void* q, const float* kp, const float* bp, const void* kmma,
+                       int32_t* ids, float* scores, cudaStream_t st) {
+  const size_t smem = select_simt_smem<D>(d->topk);
+  constexpr auto fn = select_simt_kernel<T, D, MMA>;
+  if (set_smem<fn>(smem) != cudaSuccess) return HILS_ERR_CUDA;
+  dim3 grid(unsigned((d->seqlen + kSelRows - 1) / kSelRows), unsigned(d->batch * d->heads_q));
+  fn<<<grid, kSelRows, smem, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma),
+                                  d->seqlen, d->seqlen / kChunk, d->heads_q, d->heads_q / d->heads_kv,
+                                  d->heads_kv, d->topk, 1.f / sqrtf(float(D)), ids, scores);
+  return launched(1);
+}
+
+template <typename T, int D>
+int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
+                        const float* scores, void* o, float* lse, cudaStream_t st) {
+  const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
+  const int64_t blocks = (rows + 3) / 4;
+  prefill_simt_kernel<T, D><<<dim3(unsigned(blocks)), 128, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ids, scores,
+      static_cast<T*>(o), lse, d->seqlen, d->heads_q, d->heads_q / d->heads_kv, d->heads_kv, d->topk,
+      1.f / sqrtf(float(D)), rows);
+  return launched(1);
+}
+
+template <typename T, int D>
+int launch_decode(const hils_dims* d, const void* q, const void* kc, const void* vc, const float* kp,
+                  const float* bp, const void* kmma, const int32_t* seqlens, void* o, int32_t* ids_out,
+                  float* scores_out, void* ws_ptr, cudaStream_t st) {
+  constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
+  const int64_t nc = d->seqlen / kChunk, rows = int64_t(d->batch) * d->heads_q;
+  const int G = d->heads_q / d->heads_kv, K = d->topk;
+  const float tau = 1.f / sqrtf(float(D));
+  DecodeWs ws;
+  decode_ws_layout(rows, nc, K, D, static_cast<char*>(ws_ptr), &ws);
+  const size_t smem1 = sizeof(float) * size_t(G) * D;
+  constexpr auto k1 = decode_scores_kernel<T, D, BF>;
+  if (set_smem<k1>(smem1) != cudaSuccess) return HILS_ERR_CUDA;
+  dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
+  k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
+                            d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores);
+  decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
+                                                      ws.sel_scores);
+  const int64_t units = rows * (K + 1);
+  decode_partial_kernel<T, D><<<unsigned((units + 3) / 4), 128, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
+      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, units);
+  decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(
+      ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
+      ids_out, scores_out, rows);
+  return launched(4);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hils_landmark_summary(const hils_dims* d, const void* k, const void* lq, int64_t chunk_begin,
+                          int64_t chunk_end, float* kprime, float* bprime, void* kprime_mma,
+                          hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  const int64_t nc = d->seqlen / kChunk;
+  if (!ptr_ok(k) || !ptr_ok(lq) || !ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
+  if (kprime_mma != nullptr && (d->dtype != HILS_BF16 || !aligned16(kprime_mma))) return HILS_ERR_INVALID_ARGUMENT;
+  if (chunk_begin < 0 || chunk_end < chunk_begin || chunk_end > nc) return HILS_ERR_INVALID_ARGUMENT;
+  if (chunk_end == chunk_begin) return HILS_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16) {
+    if (d->head_dim == 64) return launch_summary<__nv_bfloat16, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st);
+    return launch_summary<__nv_bfloat16, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st);
+  }
+  if (d->head_dim == 64) return launch_summary<float, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st);
+  return launch_summary<float, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st);
+}
+
+size_t hils_kprime_mma_bytes(const hils_dims* d) {
+  if (check_dims(d) != HILS_OK) return 0;
+  return size_t(d->batch) * d->heads_kv * size_t(d->seqlen / kChunk) * size_t(d->head_dim + kExt) * 2;
+}
+
+int hils_select(const hils_dims* d, const void* q, const float* kprime, const float* bprime, const void* kprime_mma,
+                int32_t* ids, float* scores, hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if (!ptr_ok(q) || !ptr_ok(ids) || (scores != nullptr && !aligned16(scores))) return HILS_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16) {
+    if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
+    if (d->head_dim == 64)
+      return launch_select_simt<__nv_bfloat16, 64, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
+    return launch_select_simt<__nv_bfloat16, 128, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
+  }
+  if (!ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->head_dim == 64) return launch_select_simt<float, 64, false>(d, q, kprime, bprime, nullptr, ids, scores, st);
+  return launch_select_simt<float, 128, false>(d, q, kprime, bprime, nullptr, ids, scores, st);
+}
+
+int hils_attn_prefill(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
+                      const float* scores, void* o, float* lse_own, hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(ids) || !ptr_ok(scores) || !ptr_ok(o))
+    return HILS_ERR_INVALID_ARGUMENT;
+  if (lse_own != nullptr && !aligned16(lse_own)) return HILS_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16) {
+    if (d->head_dim == 64) return launch_prefill_simt<__nv_bfloat16, 64>(d, q, k, v, ids, scores, o, lse_own, st);
+    return launch_prefill_simt<__nv_bfloat16, 128>(d, q, k, v, ids, scores, o, lse_own, st);
+  }
+  if (d->head_dim == 64) return launch_prefill_simt<float, 64>(d, q, k, v, ids, scores, o, lse_own, st);
+  return launch_prefill_simt<float, 128>(d, q, k, v, ids, scores, o, lse_own, st);
+}
+
+size_t hils_decode_workspace_bytes(const hils_dims* d) {
+  if (check_dims(d) != HILS_OK) return 0;
+  return decode_ws_layout(int64_t(d->batch) * d->heads_q, d->seqlen / kChunk, d->topk, d->head_dim, nullptr, nullptr);
+}
+
+int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
+                     const float* kprime, const float* bprime, const void* kprime_mma, const int32_t* seqlens,
+                     void* o, int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                     hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if (!ptr_ok(q) || !ptr_ok(k_cache) || !ptr_ok(v_cache) || !ptr_ok(seqlens) || !ptr_ok(o) || !ptr_ok(workspace))
+    return HILS_ERR_INVALID_ARGUMENT;
+  if ((ids_out != nullptr && !aligned16(ids_out)) || (scores_out != nullptr && !aligned16(scores_out)))
+    return HILS_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < hils_decode_workspace_bytes(d)) return HILS_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16) {
+    if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
+    if (d->head_dim == 64)
+      return launch_decode<__nv_bfloat16, 64>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st);
+    return launch_decode<__nv_bfloat16, 128>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st);
+  }
+  if (!ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->head_dim == 64)
+    return launch_decode<float, 64>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st);
+  return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st);
+}
+
+int hils_get_status(int32_t* host_status, hils_stream_t stream) {
+  if (host_status == nullptr) return HILS_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HILS_ERR_CUDA;
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return HILS_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return HILS_ERR_CUDA;
+  *host_status = v;
+  return HILS_OK;
+}
+
+const char* hils_strerror(int s) {
+  switch (s) {
+    case HILS_OK: return "ok";
+    case HILS_ERR_INVALID_ARGUMENT: return "invalid argument (null or misaligned pointer, or bad size)";
+    case HILS_ERR_UNSUPPORTED: return "unsupported sizes (chunk must be 64, head_dim 64 or 128, topk 1..64)";
+    case HILS_ERR_CUDA: return "CUDA error";
+    case HILS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case HILS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case HILS_ERR_DEVICE_BOUNDS: return "a device-side index (chunk id or seqlen) was out of range and skipped";
+    default: return "unknown status";
+  }
+}
+
+uint64_t hils_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,212 @@
+"""Python binding of ``libhils.so`` (the C ABI declared in include/hils.h).
+
+Argument marshalling only: every step of the HiLS forward pass runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhils.so")
+
+BF16, FP32 = 0, 1
+CHUNK = 64
+STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUPPORTED", 3: "HILS_ERR_CUDA",
+                4: "HILS_ERR_WORKSPACE_TOO_SMALL", 5: "HILS_ERR_DEVICE_TIMEOUT", 6: "HILS_ERR_DEVICE_BOUNDS"}
+EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_attn_prefill",
+           "hils_decode_workspace_bytes", "hils_attn_decode", "hils_get_status", "hils_strerror",
+           "hils_kernel_launches")
+
+
+class HilsError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {STATUS_NAMES.get(status, status)} ({strerror(status)})")
+        self.status = status
+
+
+class hils_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("chunk", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("seqlen", ctypes.c_int64), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libhils.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m chunk_wise_sparse_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        D = ctypes.POINTER(hils_dims)
+        L.hils_landmark_summary.argtypes = [D, P, P, I64, I64, P, P, P, P]
+        L.hils_kprime_mma_bytes.argtypes = [D]
+        L.hils_kprime_mma_bytes.restype = SZ
+        L.hils_select.argtypes = [D, P, P, P, P, P, P, P]
+        L.hils_attn_prefill.argtypes = [D, P, P, P, P, P, P, P, P]
+        L.hils_decode_workspace_bytes.argtypes = [D]
+        L.hils_decode_workspace_bytes.restype = SZ
+        L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
+        L.hils_strerror.argtypes = [ctypes.c_int]
+        L.hils_strerror.restype = ctypes.c_char_p
+        L.hils_kernel_launches.restype = ctypes.c_uint64
+        for name in EXPORTS:
+            getattr(L, name).restype = getattr(L, name).restype or ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().hils_strerror(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(call, rc):
+    if rc != 0:
+        raise HilsError(call, rc)
+
+
+def make_dims(batch, heads_q, heads_kv, head_dim, seqlen, topk, dtype, chunk=CHUNK) -> hils_dims:
+    if isinstance(dtype, torch.dtype):
+        dtype = BF16 if dtype == torch.bfloat16 else FP32 if dtype == torch.float32 else -1
+    return hils_dims(batch, heads_q, heads_kv, head_dim, chunk, topk, seqlen, dtype, 0)
+
+
+def dims_for(q, k, topk) -> hils_dims:
+    """Dims of a prefill from q [B,Hq,N,d] and k [B,Hkv,N,d]."""
+    B, Hq, N, d = q.shape
+    return make_dims(B, Hq, k.shape[1], d, N, topk, q.dtype)
+
+
+# ---------------------------------------------------------------------------
+# The C entry points, one Python function each (same names).
+
+def hils_landmark_summary(dims, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma=None, stream=None):
+    _check("hils_landmark_summary",
+           lib().hils_landmark_summary(ctypes.byref(dims), _ptr(k), _ptr(lq), int(chunk_begin), int(chunk_end),
+                                       _ptr(kprime), _ptr(bprime), _ptr(kprime_mma), _stream(stream)))
+
+
+def hils_kprime_mma_bytes(dims) -> int:
+    return int(lib().hils_kprime_mma_bytes(ctypes.byref(dims)))
+
+
+def hils_select(dims, q, kprime, bprime, kprime_mma, ids, scores=None, stream=None):
+    _check("hils_select", lib().hils_select(ctypes.byref(dims), _ptr(q), _ptr(kprime), _ptr(bprime),
+                                            _ptr(kprime_mma), _ptr(ids), _ptr(scores), _stream(stream)))
+
+
+def hils_attn_prefill(dims, q, k, v, ids, scores, o, lse_own=None, stream=None):
+    _check("hils_attn_prefill", lib().hils_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(ids),
+                                                        _ptr(scores), _ptr(o), _ptr(lse_own), _stream(stream)))
+
+
+def hils_decode_workspace_bytes(dims) -> int:
+    return int(lib().hils_decode_workspace_bytes(ctypes.byref(dims)))
+
+
+def hils_attn_decode(dims, q, k_cache, v_cache, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out,
+                     workspace, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("hils_attn_decode",
+           lib().hils_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kprime),
+                                  _ptr(bprime), _ptr(kprime_mma), _ptr(seqlens), _ptr(o), _ptr(ids_out),
+                                  _ptr(scores_out), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def hils_get_status(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("hils_get_status", lib().hils_get_status(ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def hils_kernel_launches() -> int:
+    return int(lib().hils_kernel_launches())
+
+
+# ---------------------------------------------------------------------------
+# Convenience layer: allocate outputs with torch and chain the calls.
+
+class Summary:
+    """Landmark summaries of one KV sequence set: fp32 k', b' and the bf16
+    scoring operand (bf16 only)."""
+
+    def __init__(self, dims, device):
+        B, H, nc, d = dims.batch, dims.heads_kv, dims.seqlen // CHUNK, dims.head_dim
+        self.kprime = torch.empty((B, H, nc, d), dtype=torch.float32, device=device)
+        self.bprime = torch.empty((B, H, nc), dtype=torch.float32, device=device)
+        self.kprime_mma = None
+        if dims.dtype == BF16:
+            n = hils_kprime_mma_bytes(dims)
+            self.kprime_mma = torch.empty((n // 2,), dtype=torch.bfloat16, device=device)
+
+
+def landmark_summary(k, lq, topk=1, chunk_begin=0, chunk_end=None, out: Summary | None = None, stream=None):
+    B, H, N, d = k.shape
+    dims = make_dims(B, H, H, d, N, topk, k.dtype)
+    out = out or Summary(dims, k.device)
+    chunk_end = N // CHUNK if chunk_end is None else chunk_end
+    hils_landmark_summary(dims, k, lq, chunk_begin, chunk_end, out.kprime, out.bprime, out.kprime_mma, stream)
+    return out
+
+
+def select(q, summ: Summary, heads_kv, topk, stream=None):
+    B, Hq, N, d = q.shape
+    dims = make_dims(B, Hq, heads_kv, d, N, topk, q.dtype)
+    ids = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device)
+    scores = torch.empty((B, Hq, N, topk), dtype=torch.float32, device=q.device)
+    hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
+    return ids, scores
+
+
+def prefill(q, k, v, lq, topk, stream=None, return_all=False):
+    """Full HiLS prefill: summary -> select -> sparse attention.  Returns O
+    (and, with return_all, the summary, ids, scores and lse_own)."""
+    dims = dims_for(q, k, topk)
+    summ = landmark_summary(k, lq, topk, stream=stream)
+    ids, scores = select(q, summ, k.shape[1], topk, stream)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, stream)
+    if return_all:
+        return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse)
+    return o
+
+
+def decode_step(q, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None):
+    """One decode step for q [B,Hq,d] against caches [B,Hkv,cap,d]."""
+    B, Hq, d = q.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    dims = make_dims(B, Hq, Hkv, d, cap, topk, q.dtype)
+    if workspace is None:
+        workspace = torch.empty((hils_decode_workspace_bytes(dims),), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    ids = torch.empty((B, Hq, topk), dtype=torch.int32, device=q.device)
+    scores = torch.empty((B, Hq, topk), dtype=torch.float32, device=q.device)
+    hils_attn_decode(dims, q, k_cache, v_cache, summ.kprime, summ.bprime, summ.kprime_mma, seqlens, o, ids, scores,
+                     workspace, stream=stream)
+    return o, ids, scores

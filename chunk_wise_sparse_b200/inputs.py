@@ -12,11 +12,13 @@ article, sections "기술 상세" (chunk size 64, top-K) and "주요 결과" (34
 models, 512K context)).  Values are i.i.d. N(0, 1); no dataset is involved.
 
 Recipe (fixed, deterministic):
-  * ``numpy.random.default_rng(seed)`` (PCG64); float32 ``standard_normal``
-    draws in the order Q, K, V, LQ, each in its row-major layout
-    (Q [B,Hq,N,d] -- or [B,Hq,d] for a decode-only workload --, K and V
-    [B,Hkv,N,d], LQ [B,Hkv,N/C,d]); then the needle picks from the same
-    generator.
+  * float32 ``standard_normal`` draws (numpy PCG64) for Q, K, V, LQ, each in
+    its row-major layout (Q [B,Hq,N,d] -- or [B,Hq,d] for a decode-only
+    workload --, K and V [B,Hkv,N,d], LQ [B,Hkv,N/C,d]).  Tensor t (0 Q, 1 K,
+    2 V, 3 LQ) is filled in blocks of 2^22 consecutive elements; block j is
+    drawn from ``default_rng(SeedSequence([seed, t, j]))`` (so blocks can be
+    drawn in parallel).  The needle picks use
+    ``default_rng(SeedSequence([seed, 4]))``.
   * Needles: a needle chunk has all of its keys shifted by
     ``+1.5 * unit(mean query of a later 256-query block)``.  The direction is
     computed per (batch, kv head) from the fp32 draws of the queries of the
@@ -35,10 +37,14 @@ Recipe (fixed, deterministic):
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 QUERY_BLOCK = 256
 NEEDLE_SHIFT = 1.5
+DRAW_BLOCK = 1 << 22
 
 
 @dataclasses.dataclass(frozen=True)
@@ -93,10 +99,13 @@ def custom(name="custom", *, B=1, Hq=1, Hkv=1, d=64, N=1024, C=64, K=3, seed=0,
 
 def round_bf16_bits(x: np.ndarray) -> np.ndarray:
     """fp32 -> bf16 bit patterns (uint16), round to nearest, ties to even."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
-    return r.astype(np.uint16)
+    u = np.array(x, dtype=np.float32, copy=True).view(np.uint32)
+    lsb = u >> np.uint32(16)
+    lsb &= np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u >>= np.uint32(16)
+    return u.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -167,16 +176,35 @@ def _pick_needles(w: Workload, rng: np.random.Generator):
     return chunks, blocks
 
 
+def _normal(shape, seed: int, tensor: int) -> np.ndarray:
+    out = np.empty(int(np.prod(shape)), np.float32)
+
+    def fill(j):
+        rng = np.random.default_rng(np.random.SeedSequence([seed, tensor, j]))
+        rng.standard_normal(out=out[j * DRAW_BLOCK:(j + 1) * DRAW_BLOCK], dtype=np.float32)
+
+    nblk = (out.size + DRAW_BLOCK - 1) // DRAW_BLOCK
+    with ThreadPoolExecutor(min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(nblk)))
+    return out.reshape(shape)
+
+
+def _to_bf16(x: np.ndarray):
+    """(bf16 bits, exact fp32 values) with round-to-nearest-even."""
+    import torch
+    t = torch.from_numpy(x).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16), t.float().numpy()
+
+
 def generate(w: Workload) -> Inputs:
-    rng = np.random.default_rng(w.seed)
     if w.kind == "decode":
-        q = rng.standard_normal((w.B, w.Hq, w.d), dtype=np.float32)
+        q = _normal((w.B, w.Hq, w.d), w.seed, 0)
     else:
-        q = rng.standard_normal((w.B, w.Hq, w.N, w.d), dtype=np.float32)
-    k = rng.standard_normal((w.B, w.Hkv, w.N, w.d), dtype=np.float32)
-    v = rng.standard_normal((w.B, w.Hkv, w.N, w.d), dtype=np.float32)
-    lq = rng.standard_normal((w.B, w.Hkv, w.nc, w.d), dtype=np.float32)
-    chunks, blocks = _pick_needles(w, rng)
+        q = _normal((w.B, w.Hq, w.N, w.d), w.seed, 0)
+    k = _normal((w.B, w.Hkv, w.N, w.d), w.seed, 1)
+    v = _normal((w.B, w.Hkv, w.N, w.d), w.seed, 2)
+    lq = _normal((w.B, w.Hkv, w.nc, w.d), w.seed, 3)
+    chunks, blocks = _pick_needles(w, np.random.default_rng(np.random.SeedSequence([w.seed, 4])))
     for c, blk in zip(chunks, blocks):
         s, e = blk * QUERY_BLOCK, (blk + 1) * QUERY_BLOCK
         for b in range(w.B):
@@ -188,9 +216,9 @@ def generate(w: Workload) -> Inputs:
     inp = Inputs(w, q, k, v, lq, chunks, blocks)
     if w.dtype == "bf16":
         for name in ("q", "k", "v", "lq"):
-            bits = round_bf16_bits(getattr(inp, name + "_f32"))
+            bits, vals = _to_bf16(getattr(inp, name + "_f32"))
             setattr(inp, name + "_bits", bits)
-            setattr(inp, name + "_f32", bf16_bits_to_f32(bits))
+            setattr(inp, name + "_f32", vals)
     elif w.dtype != "fp32":
         raise ValueError(w.dtype)
     return inp

@@ -1,0 +1,187 @@
+/*
+ * hils.h -- C ABI of the B200 (sm_100a) HiLS attention forward library.
+ *
+ * HiLS = Hierarchical Landmark Sparse attention ("Hierarchical Sparse
+ * Attention Done Right: Toward Infinite Context Modeling").  Citations below
+ * name the page and its section:
+ *   [HP-Abs]    hotpaper.ai page on the paper, abstract
+ *   [AIT-Meth]  aitrends.kr article, section "방법론" (Methodology)
+ *   [AIT-Tech]  aitrends.kr article, section "기술 상세" (Technical details)
+ *   [AIT-Gloss] aitrends.kr article, glossary "계층적 소프트맥스"
+ *   [AIP-Perf]  ai-papers.net article, section "実験結果と性能"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers, 16-byte aligned, row-major with
+ *   head_dim innermost.  The caller allocates and frees every buffer; the
+ *   library never allocates, frees or synchronises (hils_get_status is the
+ *   one call that synchronises its stream).
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and returns an int status:
+ *     HILS_OK (0)                    launched (or nothing to do)
+ *     HILS_ERR_INVALID_ARGUMENT (1)  null / misaligned pointer, bad size;
+ *                                    nothing was launched
+ *     HILS_ERR_UNSUPPORTED (2)       sizes outside the compiled set
+ *                                    (chunk != 64, head_dim not 64/128,
+ *                                    topk outside 1..64, fp32 on a
+ *                                    bf16-only call); nothing was launched
+ *     HILS_ERR_CUDA (3)              a CUDA launch error
+ *     HILS_ERR_WORKSPACE_TOO_SMALL (4)
+ *   Device-side faults are never raised by trapping.  A kernel that meets a
+ *   bad value (a chunk id or seqlen out of range) or a bounded wait that ran
+ *   out records a code in a device status word and skips the access:
+ *     HILS_ERR_DEVICE_TIMEOUT (5), HILS_ERR_DEVICE_BOUNDS (6)
+ *   Read (and clear) that word with hils_get_status.
+ * - No C++ exception crosses this boundary.  Calls are re-entrant across
+ *   streams (they keep no host state besides a launch counter).
+ * - Row = (b, hq, i).  Its kv head is h = hq / G with G = heads_q/heads_kv
+ *   (contiguous query-head groups share a kv head).  Its own chunk is
+ *   floor(i/chunk); its candidate chunks are the fully-past ones,
+ *   c < floor(i/chunk).  tau = 1/sqrt(head_dim).
+ */
+#ifndef HILS_H_
+#define HILS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hils_stream_t; /* identical to cudaStream_t */
+
+enum hils_dtype { HILS_BF16 = 0, HILS_FP32 = 1 };
+
+enum hils_status {
+  HILS_OK = 0,
+  HILS_ERR_INVALID_ARGUMENT = 1,
+  HILS_ERR_UNSUPPORTED = 2,
+  HILS_ERR_CUDA = 3,
+  HILS_ERR_WORKSPACE_TOO_SMALL = 4,
+  HILS_ERR_DEVICE_TIMEOUT = 5,
+  HILS_ERR_DEVICE_BOUNDS = 6
+};
+
+typedef struct hils_dims {
+  int32_t batch;     /* B */
+  int32_t heads_q;   /* Hq */
+  int32_t heads_kv;  /* Hkv; heads_q % heads_kv == 0 */
+  int32_t head_dim;  /* d in {64, 128} */
+  int32_t chunk;     /* C; must be 64 ([AIT-Tech]: chunk size 64) */
+  int32_t topk;      /* K in 1..64 */
+  int64_t seqlen;    /* prefill: N tokens; decode: KV-cache capacity in tokens.
+                        Must be a positive multiple of chunk. */
+  int32_t dtype;     /* HILS_BF16 (bf16 storage, fp32 accumulation) or HILS_FP32 */
+  int32_t reserved;  /* must be 0 */
+} hils_dims;
+
+/*
+ * Landmark summary of chunks [chunk_begin, chunk_end) -- [AIT-Meth], [AIT-Tech]:
+ * for each (b, h, c) the landmark query lq_c attends over the chunk's C keys,
+ *     z_j = tau * <lq_c, k_j>,  p = softmax(z),
+ *     k'_c = sum_j p_j k_j          (compressed key)
+ *     b'_c = -sum_j p_j log p_j     (entropy bias, natural log)
+ * so that tau*<q, k'_c> + b'_c is the first-order Taylor surrogate of the
+ * chunk's log-sum-exp log sum_j exp(tau*<q,k_j>).
+ *   k           [B, Hkv, seqlen, d]   dtype
+ *   lq          [B, Hkv, seqlen/C, d] dtype (one landmark query per chunk)
+ *   kprime      [B, Hkv, seqlen/C, d] fp32, written for the chunk range
+ *   bprime      [B, Hkv, seqlen/C]    fp32, written for the chunk range
+ *   kprime_mma  bf16 only (NULL for fp32; optional for bf16): the scoring
+ *               operand, hils_kprime_mma_bytes() bytes, written for the
+ *               range.  Layout [B, Hkv, seqlen/C, d+16] bf16: k'_c rounded to
+ *               bf16, then x_hi, x_lo with x_hi + x_lo ~ b'_c / tau, then 14
+ *               zeros.  hils_select and hils_attn_decode read it for bf16.
+ * 0 <= chunk_begin <= chunk_end <= seqlen/C.  Decode appends one chunk at a
+ * time by passing [c, c+1) once chunk c is full.
+ */
+int hils_landmark_summary(const hils_dims* dims, const void* k, const void* lq,
+                          int64_t chunk_begin, int64_t chunk_end,
+                          float* kprime, float* bprime, void* kprime_mma,
+                          hils_stream_t stream);
+
+/* Bytes of the bf16 scoring operand written by hils_landmark_summary. */
+size_t hils_kprime_mma_bytes(const hils_dims* dims);
+
+/*
+ * Chunk scoring and top-K selection for every query row of a prefill --
+ * [AIT-Meth]: s^_{i,c} = tau*<q_i, k'_c> + b'_c over the candidates
+ * c < floor(i/C); keep the K largest.  Ties go to the lower chunk id.
+ *   q          [B, Hq, seqlen, d] dtype
+ *   kprime     fp32 [B,Hkv,nc,d]  (fp32 path; may be NULL for bf16)
+ *   bprime     fp32 [B,Hkv,nc]    (fp32 path; may be NULL for bf16)
+ *   kprime_mma bf16 scoring operand (required for bf16, ignored for fp32);
+ *              the bf16 path scores on tensor cores with bf16 k'.
+ *   ids        [B, Hq, seqlen, K] int32 out: the kept chunk ids in ascending
+ *              order; rows with fewer than K candidates are padded with -1.
+ *   scores     [B, Hq, seqlen, K] fp32 out (nullable): s^ of each id, -inf
+ *              for padding.  hils_attn_prefill consumes it.
+ */
+int hils_select(const hils_dims* dims, const void* q, const float* kprime, const float* bprime,
+                const void* kprime_mma, int32_t* ids, float* scores, hils_stream_t stream);
+
+/*
+ * Prefill sparse attention with hierarchical fusion -- [HP-Abs], [AIT-Meth],
+ * [AIT-Gloss]: for each row and each kept chunk c, an intra-chunk softmax
+ * over the chunk's C keys gives o_c and its log-sum-exp; the row's own chunk
+ * is attended under the causal mask (keys floor(i/C)*C .. i) and enters the
+ * fusion with its exact log-sum-exp lse_own as score; the fusion weights are
+ * a softmax over {s^_c : c kept} U {lse_own}:
+ *     O_i = sum_c w_c o_c + w_own o_own.
+ *   q, k, v   [B,Hq,N,d] / [B,Hkv,N,d] / [B,Hkv,N,d] dtype
+ *   ids       [B,Hq,N,K] int32 from hils_select (-1 entries are skipped; an id
+ *             outside [0, floor(i/C)) is recorded as HILS_ERR_DEVICE_BOUNDS
+ *             and skipped)
+ *   scores    [B,Hq,N,K] fp32 from hils_select (required)
+ *   o         [B,Hq,N,d] dtype out
+ *   lse_own   [B,Hq,N] fp32 out (nullable)
+ */
+int hils_attn_prefill(const hils_dims* dims, const void* q, const void* k, const void* v,
+                      const int32_t* ids, const float* scores, void* o, float* lse_own,
+                      hils_stream_t stream);
+
+/* Device workspace bytes hils_attn_decode needs for these dims. */
+size_t hils_decode_workspace_bytes(const hils_dims* dims);
+
+/*
+ * One decode step -- [AIT-Meth] scoring and selection plus the fused sparse
+ * attention of hils_attn_prefill, for one new query per (b, hq) at position
+ * t_b = seqlens[b] - 1 whose key/value are already in the cache ([AIP-Perf]:
+ * per-token decode with sparse KV access).  Chunks 0 .. floor(t_b/C)-1 must
+ * have summaries.
+ *   dims.seqlen  KV-cache capacity in tokens
+ *   q            [B, Hq, d] dtype
+ *   k_cache, v_cache [B, Hkv, seqlen, d] dtype
+ *   kprime, bprime   fp32 summaries (fp32 path)
+ *   kprime_mma   bf16 scoring operand (bf16 path)
+ *   seqlens      device int32 [B], 1 <= seqlens[b] <= seqlen (violations are
+ *                recorded as HILS_ERR_DEVICE_BOUNDS and the row is zeroed)
+ *   o            [B, Hq, d] dtype out
+ *   ids_out      [B, Hq, K] int32 out (nullable)
+ *   scores_out   [B, Hq, K] fp32 out (nullable)
+ *   workspace    device scratch of at least hils_decode_workspace_bytes(dims)
+ */
+int hils_attn_decode(const hils_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                     const float* kprime, const float* bprime, const void* kprime_mma,
+                     const int32_t* seqlens, void* o, int32_t* ids_out, float* scores_out,
+                     void* workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * Synchronises `stream`, copies the device status word of the current device
+ * into *host_status (HILS_OK or a HILS_ERR_DEVICE_* code recorded by a kernel
+ * since the last call) and clears it.  Returns HILS_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+int hils_get_status(int32_t* host_status, hils_stream_t stream);
+
+/* Static English description of a status code. */
+const char* hils_strerror(int status);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t hils_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HILS_H_ */

@@ -1,0 +1,77 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/hils.h, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunk_wise_sparse_b200 import hils
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hils.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hils_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from chunk_wise_sparse_b200 import build
+    build.build()
+    return hils.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(hils.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def dims(**kw):
+    base = dict(batch=1, heads_q=2, heads_kv=1, head_dim=64, seqlen=1024, topk=4, dtype=hils.BF16)
+    base.update(kw)
+    return hils.make_dims(base["batch"], base["heads_q"], base["heads_kv"], base["head_dim"], base["seqlen"],
+                          base["topk"], base["dtype"], base.get("chunk", 64))
+
+
+def test_sizes(lib):
+    d = dims(batch=2, heads_q=8, heads_kv=2, head_dim=128, seqlen=4096, topk=8)
+    assert hils.hils_kprime_mma_bytes(d) == 2 * 2 * 64 * (128 + 16) * 2
+    assert hils.hils_decode_workspace_bytes(d) > 2 * 8 * 64 * 4
+    assert hils.hils_kprime_mma_bytes(dims(chunk=32)) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(chunk=32), 2), (dict(head_dim=96), 2), (dict(topk=0), 2), (dict(topk=65), 2),
+    (dict(seqlen=1000), 1), (dict(heads_q=3, heads_kv=2), 1), (dict(dtype=7), 1), (dict(batch=0), 1),
+])
+def test_bad_dims_rejected_before_launch(lib, kw, code):
+    d = dims(**kw)
+    p = ctypes.c_void_p(256)     # never dereferenced: validation fails first
+    rc = lib.hils_select(ctypes.byref(d), p, p, p, p, p, None, None)
+    assert rc == code
+    rc = lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, None)
+    assert rc == code
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    d = dims()
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(258)
+    assert lib.hils_select(ctypes.byref(d), None, p, p, p, p, None, None) == 1
+    assert lib.hils_select(ctypes.byref(d), bad, p, p, p, p, None, None) == 1
+    assert lib.hils_select(ctypes.byref(d), p, p, p, None, p, None, None) == 1   # bf16 needs the MMA operand
+    assert lib.hils_landmark_summary(ctypes.byref(d), p, p, 0, 17, p, p, None, None) == 1   # range past nc
+    assert lib.hils_landmark_summary(ctypes.byref(d), p, p, 3, 3, p, p, None, None) == 0    # empty range
+    small = hils.hils_decode_workspace_bytes(d) - 1
+    assert lib.hils_attn_decode(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, p, small, None) == 4
+    assert lib.hils_get_status(None, None) == 1
+
+
+def test_strerror(lib):
+    for code in range(7):
+        assert len(hils.strerror(code)) >= 2
+    assert hils.strerror(99) == "unknown status"

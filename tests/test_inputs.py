@@ -17,6 +17,14 @@ def test_bf16_rounding_matches_torch_rne():
     assert np.array_equal(bf16_bits_to_f32(ours), torch.from_numpy(x).to(torch.bfloat16).float().numpy())
 
 
+def test_generator_rounding_matches_numpy_rne():
+    """The generator's bf16 conversion equals an independent numpy RNE."""
+    w = custom(B=1, Hq=1, Hkv=1, d=64, N=4096, K=4, seed=9, dtype="bf16")
+    inp = generate(w)
+    from chunk_wise_sparse_b200.inputs import _normal
+    assert np.array_equal(inp.v_bits, round_bf16_bits(_normal((1, 1, 4096, 64), 9, 2)))
+
+
 def test_generation_is_deterministic():
     w = custom(B=1, Hq=2, Hkv=1, d=32, N=2048, K=4, seed=7, dtype="bf16", needles=3, needle_mode="random")
     a, b = generate(w), generate(w)
@@ -32,9 +40,8 @@ def test_needles_lie_before_their_block_and_shift_keys():
     for c, blk in zip(inp.needle_chunks, inp.needle_blocks):
         assert (c + 1) * w.C <= blk * QUERY_BLOCK
     # the needle chunk keys carry a 1.5 * unit-vector shift: their mean moves
-    rng = np.random.default_rng(w.seed)
-    rng.standard_normal((w.B, w.Hq, w.N, w.d), dtype=np.float32)
-    k0 = rng.standard_normal((w.B, w.Hkv, w.N, w.d), dtype=np.float32)
+    from chunk_wise_sparse_b200.inputs import _normal
+    k0 = _normal((w.B, w.Hkv, w.N, w.d), w.seed, 1)
     for c in inp.needle_chunks:
         delta = (inp.k_f32 - k0)[:, :, c * w.C:(c + 1) * w.C]
         assert np.allclose(np.linalg.norm(delta.mean(axis=2), axis=-1), 1.5, atol=1e-5)
