@@ -4,12 +4,16 @@
 #include <atomic>
 #include <type_traits>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "hils.h"
 #include "common.cuh"
 #include "summary.cuh"
 #include "select_simt.cuh"
 #include "attend_simt.cuh"
 #include "decode.cuh"
+#include "select_tc.cuh"
 
 using namespace hils;
 
@@ -39,18 +43,89 @@ inline int launched(int n) {
   return cudaGetLastError() == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
 }
 
-// cudaFuncSetAttribute for dynamic shared memory, once per (kernel, device).
+constexpr int kMaxSmem = 227 * 1024;
+
+// cudaFuncSetAttribute to the largest dynamic shared memory, once per (kernel, device).
 template <auto FN>
-cudaError_t set_smem(size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
+cudaError_t set_smem_max() {
   static std::atomic<uint32_t> done_mask{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const uint32_t bit = 1u << (dev & 31);
   if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(FN, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  cudaError_t e = cudaFuncSetAttribute(FN, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
   return e;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> fn{nullptr};
+  void* f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn.store(f, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// 2D bf16 tensor map: `rows` rows of `inner` elements, `row_bytes` apart.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core selection handles bf16 with G a power of two up to 16.
+bool select_tc_supported(const hils_dims* d) {
+  const int G = d->heads_q / d->heads_kv;
+  const int64_t rows_q = int64_t(d->batch) * d->heads_q * d->seqlen;
+  return d->dtype == HILS_BF16 && G <= 16 && (G & (G - 1)) == 0 && rows_q < (int64_t(1) << 31);
+}
+
+template <int D>
+int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_t* ids, float* scores,
+                     cudaStream_t st) {
+  using C = SelTc<D>;
+  const int G = d->heads_q / d->heads_kv, P = C::M / G;
+  const int64_t N = d->seqlen, nc = N / kChunk;
+  const uint64_t rows_q = uint64_t(d->batch) * d->heads_q * N, rows_k = uint64_t(d->batch) * d->heads_kv * nc;
+  CUtensorMap tq, tkb, tke;
+  if (!make_map_2d(&tq, q, D, rows_q, D * 2, 64, P, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tkb, kmma, D + kExt, rows_k, (D + kExt) * 2, 64, C::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tke, kmma, D + kExt, rows_k, (D + kExt) * 2, kExt, C::NT, CU_TENSOR_MAP_SWIZZLE_32B))
+    return HILS_ERR_CUDA;
+  int stages = 4;
+  while (stages > 2 && C::layout(d->topk, stages).total > uint32_t(kMaxSmem)) --stages;
+  const uint32_t smem = C::layout(d->topk, stages).total;
+  if (smem > uint32_t(kMaxSmem)) return HILS_ERR_UNSUPPORTED;
+  constexpr auto fn = select_tc_kernel<D>;
+  if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
+  SelTcParams p;
+  p.n_tok = N;
+  p.nc = nc;
+  p.Hq = d->heads_q;
+  p.Hkv = d->heads_kv;
+  p.G = G;
+  p.K = d->topk;
+  p.P = P;
+  p.n_row_tiles = int((N + P - 1) / P);
+  p.stages = stages;
+  p.tau = 1.f / sqrtf(float(D));
+  p.ids = ids;
+  p.scores = scores;
+  dim3 grid(unsigned(p.n_row_tiles), unsigned(d->batch * d->heads_kv));
+  fn<<<grid, C::THREADS, smem, st>>>(tq, tkb, tke, p);
+  return launched(1);
 }
 
 template <typename T, int D>
@@ -70,7 +145,7 @@ int launch_select_simt(const hils_dims* d, const void* q, const float* kp, const
                        int32_t* ids, float* scores, cudaStream_t st) {
   const size_t smem = select_simt_smem<D>(d->topk);
   constexpr auto fn = select_simt_kernel<T, D, MMA>;
-  if (set_smem<fn>(smem) != cudaSuccess) return HILS_ERR_CUDA;
+  if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 grid(unsigned((d->seqlen + kSelRows - 1) / kSelRows), unsigned(d->batch * d->heads_q));
   fn<<<grid, kSelRows, smem, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma),
                                   d->seqlen, d->seqlen / kChunk, d->heads_q, d->heads_q / d->heads_kv,
@@ -102,7 +177,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   decode_ws_layout(rows, nc, K, D, static_cast<char*>(ws_ptr), &ws);
   const size_t smem1 = sizeof(float) * size_t(G) * D;
   constexpr auto k1 = decode_scores_kernel<T, D, BF>;
-  if (set_smem<k1>(smem1) != cudaSuccess) return HILS_ERR_CUDA;
+  if (smem1 > 48 * 1024 && set_smem_max<k1>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
   k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores);
@@ -154,6 +229,10 @@ int hils_select(const hils_dims* d, const void* q, const float* kprime, const fl
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d->dtype == HILS_BF16) {
     if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
+    if (select_tc_supported(d)) {
+      if (d->head_dim == 64) return launch_select_tc<64>(d, q, kprime_mma, ids, scores, st);
+      return launch_select_tc<128>(d, q, kprime_mma, ids, scores, st);
+    }
     if (d->head_dim == 64)
       return launch_select_simt<__nv_bfloat16, 64, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
     return launch_select_simt<__nv_bfloat16, 128, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);

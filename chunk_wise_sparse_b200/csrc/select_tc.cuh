@@ -1,0 +1,301 @@
+// Kernel (b), tensor-core variant (bf16): chunk scoring on tcgen05 + fused
+// per-row top-K.
+//
+// HiLS paper, aitrends.kr article, section "방법론" (Methodology):
+//   s^_{i,c} = <q_i, k'_c>/sqrt(d) + b'_c over the fully-past chunks; keep the
+//   K largest.
+//
+// One CTA scores a tile of 128 query rows -- P = 128/G consecutive positions
+// of the G query heads that share a kv head, so the compressed keys are read
+// once for all G heads -- against the causal prefix of compressed keys, in
+// tiles of 128 chunks:
+//   warp 0 (one lane)  TMA producer: the Q tile once, then k' tiles into a
+//                      STAGES-deep shared-memory ring (128B swizzle).
+//   warp 1 (one lane)  MMA issuer: S = Q . K'^T with tcgen05.mma (M=128,
+//                      N=128, bf16 in, fp32 accumulators in TMEM, two TMEM
+//                      buffers so the epilogue of tile j overlaps the MMA of
+//                      tile j+1).  The entropy bias enters the MMA: the
+//                      scoring operand carries x = b'/tau as a bf16 hi/lo
+//                      pair in 16 extra K columns, and a constant A slice
+//                      [1, 1, 0, ...] multiplies it, so TMEM holds
+//                      <q,k'> + b'/tau and s^ = tau * acc.
+//   warps 2-5          epilogue, one thread per row (= TMEM lane): 32 scores
+//                      per tcgen05.ld; each is tested against the row's
+//                      current K-th best with one FFMA and its sign bit is
+//                      funnel-shifted into a 32-bit mask; only rows with set
+//                      bits stage their scores and insert them into a sorted
+//                      top-K list in shared memory.  Ties keep the lower
+//                      chunk id (chunks are visited in ascending order).
+// Every wait is bounded in time; a time-out records HILS_ERR_DEVICE_TIMEOUT,
+// drains in-flight copies and MMAs, frees TMEM and returns.
+#pragma once
+#include "sm100.cuh"
+
+namespace hils {
+
+template <int D>
+struct SelTc {
+  static constexpr int M = 128;           // rows per tile (TMEM lanes)
+  static constexpr int NT = 128;          // chunks per k' tile (MMA N)
+  static constexpr int KATOMS = D / 64;   // 128-byte swizzle atoms along K
+  static constexpr uint32_t A_ATOM = M * 128;
+  static constexpr uint32_t A_BYTES = KATOMS * A_ATOM;
+  static constexpr uint32_t AEXT_BYTES = M * 32;
+  static constexpr uint32_t B_ATOM = NT * 128;
+  static constexpr uint32_t B_MAIN = KATOMS * B_ATOM;
+  static constexpr uint32_t B_EXT = NT * 32;
+  static constexpr uint32_t B_STAGE = B_MAIN + B_EXT;
+  static constexpr int STG_STRIDE = 36;   // floats per thread in the staging area (conflict-free float4)
+  static constexpr uint32_t STG_BYTES = M * STG_STRIDE * 4;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 2 * NT;
+  static constexpr uint32_t IDESC = sm100::idesc_bf16(M, NT);
+
+  struct Layout {
+    uint32_t a, aext, b, stg, topv, topi, bars, misc, total;
+    int stages;
+  };
+  // Shared-memory layout (offsets from a 1024-byte aligned base).
+  __host__ __device__ static Layout layout(int K, int stages) {
+    Layout L;
+    L.stages = stages;
+    L.a = 0;
+    L.aext = A_BYTES;
+    L.b = (L.aext + AEXT_BYTES + 1023u) & ~1023u;
+    L.stg = L.b + uint32_t(stages) * B_STAGE;
+    L.topv = L.stg + STG_BYTES;
+    L.topi = L.topv + uint32_t(K) * M * 4;
+    L.bars = L.topi + uint32_t(K) * M * 4;
+    L.misc = L.bars + uint32_t(2 * stages + 6) * 8;
+    L.total = L.misc + 16 + 1024;  // + slack for aligning the dynamic base
+    return L;
+  }
+};
+
+struct SelTcParams {
+  int64_t n_tok, nc;
+  int Hq, Hkv, G, K, P;  // P = 128 / G positions per tile
+  int n_row_tiles, stages;
+  float tau;
+  int32_t* ids;
+  float* scores;
+};
+
+template <int D>
+__global__ void __launch_bounds__(SelTc<D>::THREADS, 1)
+select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kb,
+                 const __grid_constant__ CUtensorMap tm_ke, const SelTcParams p) {
+  using C = SelTc<D>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+  const typename C::Layout L = C::layout(p.K, p.stages);
+  uint8_t* sA = smem + L.a;
+  uint8_t* sAext = smem + L.aext;
+  uint8_t* sB = smem + L.b;
+  float* stg = reinterpret_cast<float*>(smem + L.stg);
+  float* topv = reinterpret_cast<float*>(smem + L.topv);
+  int32_t* topi = reinterpret_cast<int32_t*>(smem + L.topi);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + L.stages;
+  uint64_t* tfull = bars + 2 * L.stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* qfull = tempty + 2;
+  uint64_t* done = qfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
+  int* issued_slot = reinterpret_cast<int*>(smem + L.misc + 8);
+  int* consumed_slot = reinterpret_cast<int*>(smem + L.misc + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = p.n_row_tiles - 1 - int(blockIdx.x);  // longest causal prefixes first
+  const int bh = blockIdx.y;
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int64_t pos0 = int64_t(tile) * p.P;
+  const int64_t pos_end = (pos0 + p.P < p.n_tok) ? pos0 + p.P : p.n_tok;
+  const int64_t c_hi = (pos_end - 1) / kChunk;          // candidates of the tile's last row
+  const int n_tiles = int((c_hi + C::NT - 1) / C::NT);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&tfull[t], 1);
+      mbar_init(&tempty[t], 4);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    *issued_slot = 0;
+    *consumed_slot = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // constant A slice [1, 1, 0, ...] in the 32-byte swizzled K-major layout:
+    // the two 16-byte halves of row r swap when bit 2 of r is set.
+    const int r = int(threadIdx.x) - 64;
+    uint4* row = reinterpret_cast<uint4*>(sAext + r * 32);
+    const int sw = (r >> 2) & 1;
+    row[sw] = make_uint4(0x3F803F80u, 0u, 0u, 0u);
+    row[sw ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0 && n_tiles > 0) {
+    // ------------------------------------------------------------ producer
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kb);
+    prefetch_tmap(&tm_ke);
+    mbar_arrive_expect_tx(qfull, C::A_BYTES);
+    for (int g = 0; g < p.G; ++g) {
+      const int y = int((int64_t(b) * p.Hq + int64_t(h) * p.G + g) * p.n_tok + pos0);
+      for (int a = 0; a < C::KATOMS; ++a) tma_load_2d(sA + a * C::A_ATOM + g * p.P * 128, &tm_q, qfull, a * 64, y);
+    }
+    int j = 0;
+    for (; j < n_tiles; ++j) {
+      const int s = j % L.stages, u = j / L.stages;
+      if (!mbar_wait(&empty[s], (u & 1) ^ 1, abort_flag)) break;
+      mbar_arrive_expect_tx(&full[s], C::B_STAGE);
+      uint8_t* bs = sB + s * C::B_STAGE;
+      const int y = int(int64_t(bh) * p.nc + int64_t(j) * C::NT);
+      for (int a = 0; a < C::KATOMS; ++a) tma_load_2d(bs + a * C::B_ATOM, &tm_kb, &full[s], a * 64, y);
+      tma_load_2d(bs + C::B_MAIN, &tm_ke, &full[s], D, y);
+    }
+    *issued_slot = j;
+  } else if (warp == 1 && lane == 0 && n_tiles > 0) {
+    // ------------------------------------------------------------ MMA issuer
+    int j = 0;
+    if (mbar_wait(qfull, 0, abort_flag)) {
+      const uint32_t a0 = smem_u32(sA), ae = smem_u32(sAext);
+      for (; j < n_tiles; ++j) {
+        const int s = j % L.stages, u = j / L.stages, buf = j & 1, ub = j >> 1;
+        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
+        if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(buf * C::NT);
+        const uint32_t b0 = smem_u32(sB + s * C::B_STAGE);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = uint32_t((k >> 2) * C::A_ATOM + (k & 3) * 32);
+          const uint32_t offb = uint32_t((k >> 2) * C::B_ATOM + (k & 3) * 32);
+          mma_bf16(d, desc_sw128(a0 + off), desc_sw128(b0 + offb), C::IDESC, k > 0 ? 1u : 0u);
+        }
+        mma_bf16(d, desc_sw32(ae), desc_sw32(b0 + C::B_MAIN), C::IDESC, 1u);
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[buf]);
+      }
+    }
+    *consumed_slot = j;
+    mma_commit(done);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int g = r / p.P;
+    const int64_t pos = pos0 + r % p.P;
+    const bool valid = pos < p.n_tok;
+    const int64_t n_cand = valid ? pos / kChunk : 0;
+    const int K = p.K;
+    const float tau = p.tau;
+    float* tv = topv + r;
+    int32_t* ti = topi + r;
+    float* my_stg = stg + r * C::STG_STRIDE;
+    float thr = -INFINITY;
+    int count = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int buf = j & 1, ub = j >> 1;
+      if (!mbar_wait(&tfull[buf], ub & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(buf * C::NT);
+#pragma unroll 1
+      for (int gi = 0; gi < C::NT / 32; ++gi) {
+        float v[32];
+        tmem_ld32(tb + gi * 32, v);
+        const int64_t cbase = int64_t(j) * C::NT + gi * 32;
+        const int64_t lim = n_cand - cbase;
+        uint32_t bits = 0;
+        if (lim > 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) bits = __funnelshift_l(__float_as_uint(fmaf(-tau, v[e], thr)), bits, 1);
+          if (lim < 32) bits &= ~(0xFFFFFFFFu >> int(lim));
+        }
+        if (__any_sync(0xffffffffu, bits != 0)) {
+          if (bits) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          }
+          while (bits) {
+            const int e = __clz(bits);
+            bits &= ~(0x80000000u >> e);
+            const float s = tau * my_stg[e];
+            if (count == K && !(s > thr)) continue;
+            int q = count < K ? count : K - 1;
+            while (q > 0 && tv[(q - 1) * C::M] < s) {
+              tv[q * C::M] = tv[(q - 1) * C::M];
+              ti[q * C::M] = ti[(q - 1) * C::M];
+              --q;
+            }
+            tv[q * C::M] = s;
+            ti[q * C::M] = int32_t(cbase + e);
+            if (count < K) ++count;
+            if (count == K) thr = tv[(K - 1) * C::M];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+    if (valid) {
+      // ascending chunk id, then write out
+      for (int a = 1; a < count; ++a) {
+        const int32_t ci = ti[a * C::M];
+        const float cv = tv[a * C::M];
+        int q = a;
+        while (q > 0 && ti[(q - 1) * C::M] > ci) {
+          ti[q * C::M] = ti[(q - 1) * C::M];
+          tv[q * C::M] = tv[(q - 1) * C::M];
+          --q;
+        }
+        ti[q * C::M] = ci;
+        tv[q * C::M] = cv;
+      }
+      const int64_t row = (int64_t(b) * p.Hq + int64_t(h) * p.G + g) * p.n_tok + pos;
+      int32_t* out_i = p.ids + row * K;
+      float* out_s = p.scores ? p.scores + row * K : nullptr;
+      for (int t = 0; t < K; ++t) {
+        out_i[t] = t < count ? ti[t * C::M] : -1;
+        if (out_s) out_s[t] = t < count ? tv[t * C::M] : -INFINITY;
+      }
+    }
+  }
+  // ------------------------------------------------------------ teardown
+  __syncthreads();
+  if (threadIdx.x == 0 && n_tiles > 0) {
+    // copies still in flight (only after an abort): wait for them to land
+    mbar_wait_drain(qfull, 0);
+    for (int j = *consumed_slot; j < *issued_slot; ++j)
+      mbar_wait_drain(&full[j % L.stages], (j / L.stages) & 1);
+  }
+  if (warp == 1) {
+    if (lane == 0 && n_tiles > 0) mbar_wait_drain(done, 0);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace hils

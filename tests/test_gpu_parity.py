@@ -87,6 +87,9 @@ SMALL = [
     custom("bf16-k64-short", B=1, Hq=2, Hkv=1, d=64, N=2048, K=64, seed=35, dtype="bf16"),
     custom("bf16-k1", B=1, Hq=2, Hkv=2, d=128, N=1536, K=1, seed=36, dtype="bf16", needles=2,
            needle_mode="random"),
+    custom("bf16-gqa3-cuda-core-select", B=1, Hq=6, Hkv=2, d=64, N=1600, K=7, seed=37, dtype="bf16", needles=2,
+           needle_mode="random"),
+    custom("bf16-gqa16-d128", B=1, Hq=16, Hkv=1, d=128, N=1024, K=12, seed=38, dtype="bf16"),
 ]
 
 
