@@ -287,6 +287,46 @@ int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, con
   return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of hils_attn_decode_fixed_scratch: one array per device, shared by
+// every call, kept until the process exits.
+__device__ __align__(256) unsigned char g_decode_scratch[HILS_DECODE_FIXED_SCRATCH_BYTES];
+
+// Device address of g_decode_scratch on the current device (looked up once per
+// device; host code cannot use the symbol itself as a device pointer).
+void* decode_scratch_address() {
+  static std::atomic<void*> addr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  void* p = addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hils_attn_decode_fixed_scratch(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
+                                   const float* kprime, const float* bprime, const void* kprime_mma,
+                                   const int32_t* seqlens, void* o, int32_t* ids_out, float* scores_out,
+                                   hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  const size_t need = hils_decode_workspace_bytes(d);
+  if (need > size_t(HILS_DECODE_FIXED_SCRATCH_BYTES)) return HILS_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = decode_scratch_address();
+  if (scratch == nullptr) return HILS_ERR_CUDA;
+  return hils_attn_decode(d, q, k_cache, v_cache, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out,
+                          scratch, size_t(HILS_DECODE_FIXED_SCRATCH_BYTES), stream);
+}
+
 int hils_get_status(int32_t* host_status, hils_stream_t stream) {
   if (host_status == nullptr) return HILS_ERR_INVALID_ARGUMENT;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HILS_ERR_CUDA;

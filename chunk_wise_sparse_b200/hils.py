@@ -20,8 +20,9 @@ CHUNK = 64
 STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUPPORTED", 3: "HILS_ERR_CUDA",
                 4: "HILS_ERR_WORKSPACE_TOO_SMALL", 5: "HILS_ERR_DEVICE_TIMEOUT", 6: "HILS_ERR_DEVICE_BOUNDS"}
 EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_attn_prefill",
-           "hils_decode_workspace_bytes", "hils_attn_decode", "hils_get_status", "hils_strerror",
-           "hils_kernel_launches")
+           "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
+           "hils_get_status", "hils_strerror", "hils_kernel_launches")
+DECODE_FIXED_SCRATCH_BYTES = 16 << 20
 
 
 class HilsError(RuntimeError):
@@ -56,6 +57,7 @@ def lib():
         L.hils_decode_workspace_bytes.argtypes = [D]
         L.hils_decode_workspace_bytes.restype = SZ
         L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_attn_decode_fixed_scratch.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P]
         L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
         L.hils_strerror.argtypes = [ctypes.c_int]
         L.hils_strerror.restype = ctypes.c_char_p
@@ -136,6 +138,18 @@ def hils_attn_decode(dims, q, k_cache, v_cache, kprime, bprime, kprime_mma, seql
            lib().hils_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kprime),
                                   _ptr(bprime), _ptr(kprime_mma), _ptr(seqlens), _ptr(o), _ptr(ids_out),
                                   _ptr(scores_out), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def hils_attn_decode_fixed_scratch(dims, q, k_cache, v_cache, kprime, bprime, kprime_mma, seqlens, o, ids_out,
+                                   scores_out, stream=None):
+    """hils_attn_decode without a workspace, for callers that cannot allocate
+    device memory (a host engine that owns all device memory, or a decode loop
+    that must not pay cudaMalloc's implicit synchronisation).  Scratch is the
+    library's fixed 16 MiB device array; overlapping calls race on it."""
+    _check("hils_attn_decode_fixed_scratch",
+           lib().hils_attn_decode_fixed_scratch(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                                _ptr(kprime), _ptr(bprime), _ptr(kprime_mma), _ptr(seqlens),
+                                                _ptr(o), _ptr(ids_out), _ptr(scores_out), _stream(stream)))
 
 
 def hils_get_status(stream=None) -> int:

@@ -168,6 +168,35 @@ int hils_attn_decode(const hils_dims* dims, const void* q, const void* k_cache, 
                      void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
 /*
+ * Decode step that allocates nothing.  This entry point has no counterpart in
+ * the paper; it exists for callers that cannot call cudaMalloc -- for example
+ * a plugin inside a host inference engine that owns all device memory and
+ * hands its plugins no workspace, or a latency-critical decode loop where the
+ * device-wide synchronisation implied by cudaMalloc would stall other work.
+ *
+ * Same arguments and results as hils_attn_decode, minus the workspace: the
+ * scratch lives in a file-scope device array of
+ * HILS_DECODE_FIXED_SCRATCH_BYTES (16 MiB) inside the library, which every
+ * GPU that loads the library keeps until the process exits.
+ * - Sizes whose hils_decode_workspace_bytes() exceeds that maximum are
+ *   rejected with HILS_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every call uses the same array and it keeps the previous call's
+ *   contents.  Each byte a call reads is written earlier in that same call,
+ *   so nothing has to start at zero.  Calls whose executions overlap on the
+ *   GPU (other streams, other host threads) race on the array: serialise
+ *   them.
+ * - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define HILS_DECODE_FIXED_SCRATCH_BYTES (16u << 20)
+int hils_attn_decode_fixed_scratch(const hils_dims* dims, const void* q, const void* k_cache,
+                                   const void* v_cache, const float* kprime, const float* bprime,
+                                   const void* kprime_mma, const int32_t* seqlens, void* o,
+                                   int32_t* ids_out, float* scores_out, hils_stream_t stream);
+
+/*
  * Synchronises `stream`, copies the device status word of the current device
  * into *host_status (HILS_OK or a HILS_ERR_DEVICE_* code recorded by a kernel
  * since the last call) and clears it.  Returns HILS_ERR_CUDA if the
