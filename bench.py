@@ -186,6 +186,7 @@ def run_ours(args, w, rank, world, local_rank):
     seq = torch.full((B,), N, dtype=torch.int32, device=dev)
     ddims = hils.make_dims(B, Hq, Hkv, d, N, K, q.dtype)
     ws = torch.empty((hils.hils_decode_workspace_bytes(ddims),), dtype=torch.uint8, device=dev)
+    pws = hils.prefill_workspace(dims, dev)
     od = torch.empty_like(qd)
     ids_d = torch.empty((B, Hq, K), dtype=torch.int32, device=dev)
     sc_d = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
@@ -197,7 +198,7 @@ def run_ours(args, w, rank, world, local_rank):
         if ev: ev[1].record(stream)
         hils.hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
         if ev: ev[2].record(stream)
-        hils.hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, stream)
+        hils.hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, pws, stream=stream)
         if ev: ev[3].record(stream)
         hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
                               ws, stream=stream)
@@ -225,6 +226,9 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     launches = hils.hils_kernel_launches() - launches0
     clk = clocks.stop()
+    status = hils.hils_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({hils.strerror(status)}) during the timed steps")
     if world > 1:
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
@@ -304,6 +308,7 @@ def run_ours(args, w, rank, world, local_rank):
         "data": f"synthetic: i.i.d. N(0,1) Q/K/V/landmark queries, {w.needles} planted needle chunks, seed {w.seed}",
         "config": workload_config(w, world),
         "kernels_ms": kernels_ms,
+        "kernels_ms_per_step": per.round(4).tolist(),
         "decode_us_per_step": 1e3 * kernels_ms["decode"],
         "prefill_bc_tflops_useful": bc_flops / (bc_ms / 1e3) / 1e12,
         "prefill_bc_frac_of_bf16_peak": bc_flops / (bc_ms / 1e3) / 1e12 / peaks["bf16_tflops"],

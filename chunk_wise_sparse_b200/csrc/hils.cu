@@ -14,6 +14,7 @@
 #include "attend_simt.cuh"
 #include "decode.cuh"
 #include "select_tc.cuh"
+#include "prefill_cc.cuh"
 
 using namespace hils;
 
@@ -92,10 +93,10 @@ bool select_tc_supported(const hils_dims* d) {
   return d->dtype == HILS_BF16 && G <= 16 && (G & (G - 1)) == 0 && rows_q < (int64_t(1) << 31);
 }
 
-template <int D>
+template <int D, int KCAP>
 int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_t* ids, float* scores,
                      cudaStream_t st) {
-  using C = SelTc<D>;
+  using C = SelTc<D, KCAP>;
   const int G = d->heads_q / d->heads_kv, P = C::M / G;
   const int64_t N = d->seqlen, nc = N / kChunk;
   const uint64_t rows_q = uint64_t(d->batch) * d->heads_q * N, rows_k = uint64_t(d->batch) * d->heads_kv * nc;
@@ -104,11 +105,12 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
       !make_map_2d(&tkb, kmma, D + kExt, rows_k, (D + kExt) * 2, 64, C::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tke, kmma, D + kExt, rows_k, (D + kExt) * 2, kExt, C::NT, CU_TENSOR_MAP_SWIZZLE_32B))
     return HILS_ERR_CUDA;
-  int stages = 4;
+  // d=64 fits two CTAs per SM with 3 stages; d=128 runs one CTA with up to 4.
+  int stages = D == 64 ? 3 : 4;
   while (stages > 2 && C::layout(d->topk, stages).total > uint32_t(kMaxSmem)) --stages;
   const uint32_t smem = C::layout(d->topk, stages).total;
   if (smem > uint32_t(kMaxSmem)) return HILS_ERR_UNSUPPORTED;
-  constexpr auto fn = select_tc_kernel<D>;
+  constexpr auto fn = select_tc_kernel<D, KCAP>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   SelTcParams p;
   p.n_tok = N;
@@ -126,6 +128,104 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
   dim3 grid(unsigned(p.n_row_tiles), unsigned(d->batch * d->heads_kv));
   fn<<<grid, C::THREADS, smem, st>>>(tq, tkb, tke, p);
   return launched(1);
+}
+
+// ---------------------------------------------------------------- chunk-centric prefill (bf16)
+struct CcPlan {
+  CcDims c;
+  int64_t rows, n_slots;
+  size_t off_oacc, off_rowstat, off_counts, off_cursor, off_offsets, off_tiles, off_entries, total;
+};
+
+bool cc_supported(const hils_dims* d) {
+  const int64_t G = d->heads_q / d->heads_kv;
+  return d->dtype == HILS_BF16 && G * d->seqlen <= (int64_t(1) << 25) &&
+         int64_t(d->batch) * d->heads_q * d->seqlen < (int64_t(1) << 31);
+}
+
+CcPlan cc_plan(const hils_dims* d) {
+  CcPlan P;
+  const int64_t N = d->seqlen, D = d->head_dim, G = d->heads_q / d->heads_kv;
+  P.c.n_tok = N;
+  P.c.nc = N / kChunk;
+  P.c.Hq = d->heads_q;
+  P.c.Hkv = d->heads_kv;
+  P.c.G = int(G);
+  P.c.K = d->topk;
+  P.c.tau = 1.f / sqrtf(float(D));
+  // window: the fp32 accumulators and bf16 queries of one window of one kv head
+  // (G x W positions) stay within 64 MiB of L2
+  int shift = 6;
+  while ((int64_t(1) << (shift + 1)) <= N && G * (int64_t(1) << (shift + 1)) * D * 6 <= (int64_t(64) << 20)) ++shift;
+  P.c.win_shift = shift;
+  P.c.n_win = int((N + (int64_t(1) << shift) - 1) >> shift);
+  P.c.n_keys = int64_t(d->batch) * d->heads_kv * P.c.n_win * P.c.nc;
+  P.rows = int64_t(d->batch) * d->heads_q * N;
+  P.n_slots = P.rows * d->topk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
+  P.off_oacc = take(sizeof(float) * P.rows * D);
+  P.off_rowstat = take(sizeof(float) * P.rows);
+  P.off_counts = take(sizeof(int32_t) * P.c.n_keys);
+  P.off_cursor = take(sizeof(int32_t) * P.c.n_keys);
+  P.off_offsets = take(sizeof(int64_t) * (P.c.n_keys + 1));
+  P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
+  P.off_entries = take(sizeof(int32_t) * P.n_slots);
+  P.total = off;
+  return P;
+}
+
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int v = cached[dev & 63].load(std::memory_order_relaxed);
+  if (v == 0) {
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev & 63].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+template <int D>
+int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
+                      const float* scores, void* o, float* lse, void* ws, cudaStream_t st) {
+  using C = CcTc<D>;
+  const CcPlan P = cc_plan(d);
+  char* base = static_cast<char*>(ws);
+  float* oacc = reinterpret_cast<float*>(base + P.off_oacc);
+  float* rowstat = reinterpret_cast<float*>(base + P.off_rowstat);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + P.off_counts);
+  int32_t* cursor = reinterpret_cast<int32_t*>(base + P.off_cursor);
+  int64_t* offsets = reinterpret_cast<int64_t*>(base + P.off_offsets);
+  int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
+  int32_t* entries = reinterpret_cast<int32_t*>(base + P.off_entries);
+  const uint64_t kv_rows = uint64_t(d->batch) * d->heads_kv * d->seqlen;
+  CUtensorMap tk, tv;
+  if (!make_map_2d(&tk, k, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tv, v, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+    return HILS_ERR_CUDA;
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess) return HILS_ERR_CUDA;
+  cc_own_kernel<__nv_bfloat16, D><<<unsigned((P.rows + 3) / 4), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), ids, scores, oacc, rowstat, lse, counts, P.c, P.rows);
+  cc_scan_kernel<<<1, 1024, 0, st>>>(counts, P.c.n_keys, offsets, tiles, cursor);
+  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, offsets, cursor, entries, P.c, P.n_slots);
+  constexpr auto fn = cc_attend_kernel<D>;
+  if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
+  CcTcParams prm;
+  prm.c = P.c;
+  prm.offsets = offsets;
+  prm.tile_start = tiles;
+  prm.entries = entries;
+  prm.scores = scores;
+  prm.rowstat = rowstat;
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.oacc = oacc;
+  fn<<<unsigned(sm_count() * C::MAX_CTAS), 128, C::SMEM, st>>>(tk, tv, prm);
+  const int64_t n8 = P.rows * D / 8;
+  cc_final_kernel<D><<<unsigned((n8 + 255) / 256), 256, 0, st>>>(oacc, static_cast<__nv_bfloat16*>(o), n8);
+  return launched(5);
 }
 
 template <typename T, int D>
@@ -230,8 +330,15 @@ int hils_select(const hils_dims* d, const void* q, const float* kprime, const fl
   if (d->dtype == HILS_BF16) {
     if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
     if (select_tc_supported(d)) {
-      if (d->head_dim == 64) return launch_select_tc<64>(d, q, kprime_mma, ids, scores, st);
-      return launch_select_tc<128>(d, q, kprime_mma, ids, scores, st);
+      const int K = d->topk;
+      if (d->head_dim == 64) {
+        if (K <= 16) return launch_select_tc<64, 16>(d, q, kprime_mma, ids, scores, st);
+        if (K <= 32) return launch_select_tc<64, 32>(d, q, kprime_mma, ids, scores, st);
+        return launch_select_tc<64, 0>(d, q, kprime_mma, ids, scores, st);
+      }
+      if (K <= 16) return launch_select_tc<128, 16>(d, q, kprime_mma, ids, scores, st);
+      if (K <= 32) return launch_select_tc<128, 32>(d, q, kprime_mma, ids, scores, st);
+      return launch_select_tc<128, 0>(d, q, kprime_mma, ids, scores, st);
     }
     if (d->head_dim == 64)
       return launch_select_simt<__nv_bfloat16, 64, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
@@ -242,14 +349,28 @@ int hils_select(const hils_dims* d, const void* q, const float* kprime, const fl
   return launch_select_simt<float, 128, false>(d, q, kprime, bprime, nullptr, ids, scores, st);
 }
 
+size_t hils_prefill_workspace_bytes(const hils_dims* d) {
+  if (check_dims(d) != HILS_OK) return 0;
+  if (!cc_supported(d)) return 0;
+  return cc_plan(d).total;
+}
+
 int hils_attn_prefill(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
-                      const float* scores, void* o, float* lse_own, hils_stream_t stream) {
+                      const float* scores, void* o, float* lse_own, void* workspace, size_t workspace_bytes,
+                      hils_stream_t stream) {
   int rc = check_dims(d);
   if (rc) return rc;
   if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(ids) || !ptr_ok(scores) || !ptr_ok(o))
     return HILS_ERR_INVALID_ARGUMENT;
   if (lse_own != nullptr && !aligned16(lse_own)) return HILS_ERR_INVALID_ARGUMENT;
+  const size_t need = hils_prefill_workspace_bytes(d);
+  if (workspace_bytes < need) return HILS_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && !ptr_ok(workspace)) return HILS_ERR_INVALID_ARGUMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16 && need > 0) {
+    if (d->head_dim == 64) return launch_prefill_cc<64>(d, q, k, v, ids, scores, o, lse_own, workspace, st);
+    return launch_prefill_cc<128>(d, q, k, v, ids, scores, o, lse_own, workspace, st);
+  }
   if (d->dtype == HILS_BF16) {
     if (d->head_dim == 64) return launch_prefill_simt<__nv_bfloat16, 64>(d, q, k, v, ids, scores, o, lse_own, st);
     return launch_prefill_simt<__nv_bfloat16, 128>(d, q, k, v, ids, scores, o, lse_own, st);

@@ -33,7 +33,7 @@
 
 namespace hils {
 
-template <int D>
+template <int D, int KCAP>
 struct SelTc {
   static constexpr int M = 128;           // rows per tile (TMEM lanes)
   static constexpr int NT = 128;          // chunks per k' tile (MMA N)
@@ -46,6 +46,7 @@ struct SelTc {
   static constexpr uint32_t B_EXT = NT * 32;
   static constexpr uint32_t B_STAGE = B_MAIN + B_EXT;
   static constexpr int STG_STRIDE = 36;   // floats per thread in the staging area (conflict-free float4)
+  // KCAP > 0: the per-row top-K lives in registers (K <= KCAP); 0: in shared memory.
   static constexpr uint32_t STG_BYTES = M * STG_STRIDE * 4;
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 2 * NT;
@@ -63,9 +64,10 @@ struct SelTc {
     L.aext = A_BYTES;
     L.b = (L.aext + AEXT_BYTES + 1023u) & ~1023u;
     L.stg = L.b + uint32_t(stages) * B_STAGE;
+    const uint32_t list_bytes = KCAP > 0 ? 0u : uint32_t(K) * M * 4;
     L.topv = L.stg + STG_BYTES;
-    L.topi = L.topv + uint32_t(K) * M * 4;
-    L.bars = L.topi + uint32_t(K) * M * 4;
+    L.topi = L.topv + list_bytes;
+    L.bars = L.topi + list_bytes;
     L.misc = L.bars + uint32_t(2 * stages + 6) * 8;
     L.total = L.misc + 16 + 1024;  // + slack for aligning the dynamic base
     return L;
@@ -81,11 +83,11 @@ struct SelTcParams {
   float* scores;
 };
 
-template <int D>
-__global__ void __launch_bounds__(SelTc<D>::THREADS, 1)
+template <int D, int KCAP>
+__global__ void __launch_bounds__(SelTc<D, KCAP>::THREADS, 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kb,
                  const __grid_constant__ CUtensorMap tm_ke, const SelTcParams p) {
-  using C = SelTc<D>;
+  using C = SelTc<D, KCAP>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -209,11 +211,23 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int64_t n_cand = valid ? pos / kChunk : 0;
     const int K = p.K;
     const float tau = p.tau;
+    float* my_stg = stg + r * C::STG_STRIDE;
+    // Register list (KCAP > 0): sorted descending; slots [0, KCAP-K) hold +inf
+    // so that the K-th best is always the last slot.  Shared-memory list
+    // (KCAP == 0): sorted descending, K slots, `count` filled.
+    constexpr int KR = KCAP > 0 ? KCAP : 1;
+    float rv[KR];
+    int32_t ri[KR];
+#pragma unroll
+    for (int t = 0; t < KR; ++t) {
+      const bool pad = t < KR - K;
+      rv[t] = pad ? INFINITY : -INFINITY;
+      ri[t] = pad ? -2 : -1;
+    }
     float* tv = topv + r;
     int32_t* ti = topi + r;
-    float* my_stg = stg + r * C::STG_STRIDE;
-    float thr = -INFINITY;
     int count = 0;
+    float thr = -INFINITY;
     for (int j = 0; j < n_tiles; ++j) {
       const int buf = j & 1, ub = j >> 1;
       if (!mbar_wait(&tfull[buf], ub & 1, abort_flag)) break;
@@ -227,6 +241,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int64_t lim = n_cand - cbase;
         uint32_t bits = 0;
         if (lim > 0) {
+          // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr)
 #pragma unroll
           for (int e = 0; e < 32; ++e) bits = __funnelshift_l(__float_as_uint(fmaf(-tau, v[e], thr)), bits, 1);
           if (lim < 32) bits &= ~(0xFFFFFFFFu >> int(lim));
@@ -240,18 +255,35 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           while (bits) {
             const int e = __clz(bits);
             bits &= ~(0x80000000u >> e);
-            const float s = tau * my_stg[e];
-            if (count == K && !(s > thr)) continue;
-            int q = count < K ? count : K - 1;
-            while (q > 0 && tv[(q - 1) * C::M] < s) {
-              tv[q * C::M] = tv[(q - 1) * C::M];
-              ti[q * C::M] = ti[(q - 1) * C::M];
-              --q;
+            const float sc = tau * my_stg[e];
+            const int32_t cid = int32_t(cbase + e);
+            if constexpr (KCAP > 0) {
+              if (!(sc > rv[KR - 1])) continue;
+              // insert keeping descending order; equal scores stay ahead (lower ids)
+              bool ge[KR];
+#pragma unroll
+              for (int t = 0; t < KR; ++t) ge[t] = rv[t] >= sc;
+#pragma unroll
+              for (int t = KR - 1; t >= 1; --t) {
+                rv[t] = ge[t] ? rv[t] : (ge[t - 1] ? sc : rv[t - 1]);
+                ri[t] = ge[t] ? ri[t] : (ge[t - 1] ? cid : ri[t - 1]);
+              }
+              rv[0] = ge[0] ? rv[0] : sc;
+              ri[0] = ge[0] ? ri[0] : cid;
+              thr = rv[KR - 1];
+            } else {
+              if (count == K && !(sc > thr)) continue;
+              int q = count < K ? count : K - 1;
+              while (q > 0 && tv[(q - 1) * C::M] < sc) {
+                tv[q * C::M] = tv[(q - 1) * C::M];
+                ti[q * C::M] = ti[(q - 1) * C::M];
+                --q;
+              }
+              tv[q * C::M] = sc;
+              ti[q * C::M] = cid;
+              if (count < K) ++count;
+              if (count == K) thr = tv[(K - 1) * C::M];
             }
-            tv[q * C::M] = s;
-            ti[q * C::M] = int32_t(cbase + e);
-            if (count < K) ++count;
-            if (count == K) thr = tv[(K - 1) * C::M];
           }
         }
       }
@@ -260,25 +292,44 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (lane == 0) mbar_arrive(&tempty[buf]);
     }
     if (valid) {
-      // ascending chunk id, then write out
-      for (int a = 1; a < count; ++a) {
-        const int32_t ci = ti[a * C::M];
-        const float cv = tv[a * C::M];
-        int q = a;
-        while (q > 0 && ti[(q - 1) * C::M] > ci) {
-          ti[q * C::M] = ti[(q - 1) * C::M];
-          tv[q * C::M] = tv[(q - 1) * C::M];
-          --q;
-        }
-        ti[q * C::M] = ci;
-        tv[q * C::M] = cv;
-      }
       const int64_t row = (int64_t(b) * p.Hq + int64_t(h) * p.G + g) * p.n_tok + pos;
       int32_t* out_i = p.ids + row * K;
       float* out_s = p.scores ? p.scores + row * K : nullptr;
-      for (int t = 0; t < K; ++t) {
-        out_i[t] = t < count ? ti[t * C::M] : -1;
-        if (out_s) out_s[t] = t < count ? tv[t * C::M] : -INFINITY;
+      if constexpr (KCAP > 0) {
+        // ascending chunk id: each kept entry goes to its rank among the kept ids
+        int n_kept = 0;
+#pragma unroll
+        for (int t = 0; t < KR; ++t) n_kept += ri[t] >= 0;
+#pragma unroll
+        for (int t = 0; t < KR; ++t) {
+          if (ri[t] < 0) continue;
+          int rank = 0;
+#pragma unroll
+          for (int u = 0; u < KR; ++u) rank += (ri[u] >= 0) & (ri[u] < ri[t]);
+          out_i[rank] = ri[t];
+          if (out_s) out_s[rank] = rv[t];
+        }
+        for (int t = n_kept; t < K; ++t) {
+          out_i[t] = -1;
+          if (out_s) out_s[t] = -INFINITY;
+        }
+      } else {
+        for (int a = 1; a < count; ++a) {
+          const int32_t ci = ti[a * C::M];
+          const float cv = tv[a * C::M];
+          int q = a;
+          while (q > 0 && ti[(q - 1) * C::M] > ci) {
+            ti[q * C::M] = ti[(q - 1) * C::M];
+            tv[q * C::M] = tv[(q - 1) * C::M];
+            --q;
+          }
+          ti[q * C::M] = ci;
+          tv[q * C::M] = cv;
+        }
+        for (int t = 0; t < K; ++t) {
+          out_i[t] = t < count ? ti[t * C::M] : -1;
+          if (out_s) out_s[t] = t < count ? tv[t * C::M] : -INFINITY;
+        }
       }
     }
   }

@@ -19,7 +19,8 @@ BF16, FP32 = 0, 1
 CHUNK = 64
 STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUPPORTED", 3: "HILS_ERR_CUDA",
                 4: "HILS_ERR_WORKSPACE_TOO_SMALL", 5: "HILS_ERR_DEVICE_TIMEOUT", 6: "HILS_ERR_DEVICE_BOUNDS"}
-EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_attn_prefill",
+EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_prefill_workspace_bytes",
+           "hils_attn_prefill",
            "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
            "hils_get_status", "hils_strerror", "hils_kernel_launches")
 DECODE_FIXED_SCRATCH_BYTES = 16 << 20
@@ -53,7 +54,9 @@ def lib():
         L.hils_kprime_mma_bytes.argtypes = [D]
         L.hils_kprime_mma_bytes.restype = SZ
         L.hils_select.argtypes = [D, P, P, P, P, P, P, P]
-        L.hils_attn_prefill.argtypes = [D, P, P, P, P, P, P, P, P]
+        L.hils_prefill_workspace_bytes.argtypes = [D]
+        L.hils_prefill_workspace_bytes.restype = SZ
+        L.hils_attn_prefill.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_workspace_bytes.argtypes = [D]
         L.hils_decode_workspace_bytes.restype = SZ
         L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -121,9 +124,23 @@ def hils_select(dims, q, kprime, bprime, kprime_mma, ids, scores=None, stream=No
                                             _ptr(kprime_mma), _ptr(ids), _ptr(scores), _stream(stream)))
 
 
-def hils_attn_prefill(dims, q, k, v, ids, scores, o, lse_own=None, stream=None):
+def hils_prefill_workspace_bytes(dims) -> int:
+    return int(lib().hils_prefill_workspace_bytes(ctypes.byref(dims)))
+
+
+def hils_attn_prefill(dims, q, k, v, ids, scores, o, lse_own=None, workspace=None, workspace_bytes=None,
+                      stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("hils_attn_prefill", lib().hils_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(ids),
-                                                        _ptr(scores), _ptr(o), _ptr(lse_own), _stream(stream)))
+                                                        _ptr(scores), _ptr(o), _ptr(lse_own), _ptr(workspace),
+                                                        int(workspace_bytes), _stream(stream)))
+
+
+def prefill_workspace(dims, device):
+    """A device workspace for hils_attn_prefill (None when none is needed)."""
+    n = hils_prefill_workspace_bytes(dims)
+    return torch.empty((n,), dtype=torch.uint8, device=device) if n else None
 
 
 def hils_decode_workspace_bytes(dims) -> int:
@@ -205,7 +222,7 @@ def prefill(q, k, v, lq, topk, stream=None, return_all=False):
     ids, scores = select(q, summ, k.shape[1], topk, stream)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, stream)
+    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, prefill_workspace(dims, q.device), stream=stream)
     if return_all:
         return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse)
     return o

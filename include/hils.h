@@ -122,6 +122,15 @@ int hils_select(const hils_dims* dims, const void* q, const float* kprime, const
                 const void* kprime_mma, int32_t* ids, float* scores, hils_stream_t stream);
 
 /*
+ * Device workspace bytes hils_attn_prefill needs for these dims (0 when the
+ * call needs none: the fp32 path).  For bf16 it holds an fp32 output
+ * accumulator (rows x d), the fusion normaliser of every row, and the
+ * inverted index of (row, slot) pairs per (kv head, window, chunk): about
+ * rows x (4d + 4 + 4K) bytes.
+ */
+size_t hils_prefill_workspace_bytes(const hils_dims* dims);
+
+/*
  * Prefill sparse attention with hierarchical fusion -- [HP-Abs], [AIT-Meth],
  * [AIT-Gloss]: for each row and each kept chunk c, an intra-chunk softmax
  * over the chunk's C keys gives o_c and its log-sum-exp; the row's own chunk
@@ -136,10 +145,13 @@ int hils_select(const hils_dims* dims, const void* q, const float* kprime, const
  *   scores    [B,Hq,N,K] fp32 from hils_select (required)
  *   o         [B,Hq,N,d] dtype out
  *   lse_own   [B,Hq,N] fp32 out (nullable)
+ *   workspace device scratch of at least hils_prefill_workspace_bytes(dims)
+ *             (may be NULL when that is 0); HILS_ERR_WORKSPACE_TOO_SMALL
+ *             otherwise
  */
 int hils_attn_prefill(const hils_dims* dims, const void* q, const void* k, const void* v,
                       const int32_t* ids, const float* scores, void* o, float* lse_own,
-                      hils_stream_t stream);
+                      void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
 /* Device workspace bytes hils_attn_decode needs for these dims. */
 size_t hils_decode_workspace_bytes(const hils_dims* dims);

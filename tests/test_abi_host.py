@@ -54,7 +54,7 @@ def test_bad_dims_rejected_before_launch(lib, kw, code):
     p = ctypes.c_void_p(256)     # never dereferenced: validation fails first
     rc = lib.hils_select(ctypes.byref(d), p, p, p, p, p, None, None)
     assert rc == code
-    rc = lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, None)
+    rc = lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, None, 0, None)
     assert rc == code
 
 
@@ -69,6 +69,11 @@ def test_null_and_misaligned_pointers_rejected(lib):
     small = hils.hils_decode_workspace_bytes(d) - 1
     assert lib.hils_attn_decode(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, p, small, None) == 4
     assert lib.hils_get_status(None, None) == 1
+    # bf16 prefill needs its workspace
+    need = hils.hils_prefill_workspace_bytes(d)
+    assert need > 0
+    assert lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, p, need - 1, None) == 4
+    assert hils.hils_prefill_workspace_bytes(dims(dtype=hils.FP32)) == 0
 
 
 def test_strerror(lib):
