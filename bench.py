@@ -152,6 +152,22 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own tokens_per_rank per step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def workload_config(w, n_gpus):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "C": w.C, "K": w.K,
             "needles": w.needles, "seed": w.seed, "parallelism": f"dp{n_gpus} (independent replicas)",
@@ -231,14 +247,10 @@ def run_ours(args, w, rank, world, local_rank):
         raise RuntimeError(f"device status {status} ({hils.strerror(status)}) during the timed steps")
     if world > 1:
         dist.barrier()
-    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # ms per kernel
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     ms_step = total_ms / args.steps
-    value = world * B * N / (ms_step / 1e3)
+    value = job_throughput(world, B * N, ms_step)
 
     # end to end through the public API: pinned host inputs -> device -> path -> host result
     e2e = None
@@ -272,12 +284,8 @@ def run_ours(args, w, rank, world, local_rank):
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-        e_ms = a0.elapsed_time(a1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * B * N / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e_ms = max_over_ranks(a0.elapsed_time(a1) / n_e2e, world, dev)
+        e2e = {"value": job_throughput(world, B * N, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
     if rank != 0:
         return

@@ -133,14 +133,17 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
 // ---------------------------------------------------------------- chunk-centric prefill (bf16)
 struct CcPlan {
   CcDims c;
-  int64_t rows, n_slots;
-  size_t off_oacc, off_rowstat, off_counts, off_cursor, off_offsets, off_tiles, off_entries, total;
+  int64_t rows, n_slots, max_items, n_scan_blocks;
+  int P, own_tiles;
+  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_erow, off_efac,
+      total;
 };
 
 bool cc_supported(const hils_dims* d) {
   const int64_t G = d->heads_q / d->heads_kv;
-  return d->dtype == HILS_BF16 && G * d->seqlen <= (int64_t(1) << 25) &&
-         int64_t(d->batch) * d->heads_q * d->seqlen < (int64_t(1) << 31);
+  const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
+  return d->dtype == HILS_BF16 && G <= 16 && (G & (G - 1)) == 0 && G * d->seqlen <= (int64_t(1) << 25) &&
+         rows * d->topk < (int64_t(1) << 31);
 }
 
 CcPlan cc_plan(const hils_dims* d) {
@@ -162,15 +165,22 @@ CcPlan cc_plan(const hils_dims* d) {
   P.c.n_keys = int64_t(d->batch) * d->heads_kv * P.c.n_win * P.c.nc;
   P.rows = int64_t(d->batch) * d->heads_q * N;
   P.n_slots = P.rows * d->topk;
+  P.P = int(128 / G);
+  P.own_tiles = int((N + P.P - 1) / P.P);
+  P.n_scan_blocks = (P.c.n_keys + kScanBlock - 1) / kScanBlock;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
   P.off_oacc = take(sizeof(float) * P.rows * D);
   P.off_rowstat = take(sizeof(float) * P.rows);
   P.off_counts = take(sizeof(int32_t) * P.c.n_keys);
-  P.off_cursor = take(sizeof(int32_t) * P.c.n_keys);
+  P.off_ranks = take(sizeof(int32_t) * P.n_slots);
   P.off_offsets = take(sizeof(int64_t) * (P.c.n_keys + 1));
   P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
-  P.off_entries = take(sizeof(int32_t) * P.n_slots);
+  P.max_items = P.n_slots / kCcTileRows + P.c.n_keys + 1;
+  P.off_items = take(sizeof(int4) * P.max_items);
+  P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
+  P.off_erow = take(sizeof(int32_t) * P.n_slots);
+  P.off_efac = take(sizeof(float) * P.n_slots);
   P.total = off;
   return P;
 }
@@ -191,41 +201,64 @@ template <int D>
 int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
                       const float* scores, void* o, float* lse, void* ws, cudaStream_t st) {
   using C = CcTc<D>;
+  using CO = CcOwn<D>;
   const CcPlan P = cc_plan(d);
   char* base = static_cast<char*>(ws);
   float* oacc = reinterpret_cast<float*>(base + P.off_oacc);
   float* rowstat = reinterpret_cast<float*>(base + P.off_rowstat);
   int32_t* counts = reinterpret_cast<int32_t*>(base + P.off_counts);
-  int32_t* cursor = reinterpret_cast<int32_t*>(base + P.off_cursor);
+  int32_t* ranks = reinterpret_cast<int32_t*>(base + P.off_ranks);
   int64_t* offsets = reinterpret_cast<int64_t*>(base + P.off_offsets);
   int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
-  int32_t* entries = reinterpret_cast<int32_t*>(base + P.off_entries);
+  int4* items = reinterpret_cast<int4*>(base + P.off_items);
+  int64_t* sums = reinterpret_cast<int64_t*>(base + P.off_sums);
+  int32_t* e_row = reinterpret_cast<int32_t*>(base + P.off_erow);
+  float* e_fac = reinterpret_cast<float*>(base + P.off_efac);
   const uint64_t kv_rows = uint64_t(d->batch) * d->heads_kv * d->seqlen;
-  CUtensorMap tk, tv;
-  if (!make_map_2d(&tk, k, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tv, v, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+  const uint32_t nk_own = P.P >= kChunk ? uint32_t(P.P) : uint32_t(kChunk);
+  CUtensorMap tq_tile, tq_row, tk, tv, tk_own, tv_own;
+  if (!make_map_2d(&tq_tile, q, D, uint64_t(P.rows), D * 2, 64, uint32_t(P.P), CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tq_row, q, D, uint64_t(P.rows), D * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tk, k, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tv, v, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tk_own, k, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tv_own, v, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B))
     return HILS_ERR_CUDA;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess) return HILS_ERR_CUDA;
-  cc_own_kernel<__nv_bfloat16, D><<<unsigned((P.rows + 3) / 4), 128, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), ids, scores, oacc, rowstat, lse, counts, P.c, P.rows);
-  cc_scan_kernel<<<1, 1024, 0, st>>>(counts, P.c.n_keys, offsets, tiles, cursor);
-  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, offsets, cursor, entries, P.c, P.n_slots);
+  constexpr auto own_fn = cc_own_tc_kernel<D>;
+  if (set_smem_max<own_fn>() != cudaSuccess) return HILS_ERR_CUDA;
+  CcOwnParams op;
+  op.c = P.c;
+  op.ids = ids;
+  op.scores = scores;
+  op.oacc = oacc;
+  op.rowstat = rowstat;
+  op.lse_own = lse;
+  op.counts = counts;
+  op.ranks = ranks;
+  op.P = P.P;
+  op.n_tiles = P.own_tiles;
+  own_fn<<<dim3(unsigned(P.own_tiles), unsigned(d->batch * d->heads_kv)), 128, CO::SMEM, st>>>(tq_tile, tk_own,
+                                                                                            tv_own, op);
+  const unsigned nsb = unsigned(P.n_scan_blocks);
+  cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
+  cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
+  cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
+  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_row, e_fac,
+                                                                     P.c, P.n_slots);
   constexpr auto fn = cc_attend_kernel<D>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   CcTcParams prm;
   prm.c = P.c;
-  prm.offsets = offsets;
   prm.tile_start = tiles;
-  prm.entries = entries;
-  prm.scores = scores;
-  prm.rowstat = rowstat;
-  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.items = items;
+  prm.e_row = e_row;
+  prm.e_fac = e_fac;
   prm.oacc = oacc;
-  fn<<<unsigned(sm_count() * C::MAX_CTAS), 128, C::SMEM, st>>>(tk, tv, prm);
+  fn<<<unsigned(sm_count() * C::MAX_CTAS), C::THREADS, C::SMEM, st>>>(tq_row, tk, tv, prm);
   const int64_t n8 = P.rows * D / 8;
   cc_final_kernel<D><<<unsigned((n8 + 255) / 256), 256, 0, st>>>(oacc, static_cast<__nv_bfloat16*>(o), n8);
-  return launched(5);
+  return launched(8);
 }
 
 template <typename T, int D>
@@ -456,6 +489,13 @@ int hils_get_status(int32_t* host_status, hils_stream_t stream) {
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return HILS_ERR_CUDA;
   *host_status = v;
   return HILS_OK;
+}
+
+int hils_selftest_bounded_wait(int32_t limit_ms, hils_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return HILS_ERR_INVALID_ARGUMENT;
+  sm100::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      uint64_t(limit_ms) * 1000000ull);
+  return launched(1);
 }
 
 const char* hils_strerror(int s) {

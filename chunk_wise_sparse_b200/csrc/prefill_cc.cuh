@@ -47,129 +47,433 @@ __device__ __forceinline__ int64_t cc_key(const CcDims& c, int64_t bh, int64_t p
   return (bh * c.n_win + (pos >> c.win_shift)) * c.nc + chunk;
 }
 
-// ---------------------------------------------------------------- own chunk + counts
-template <typename T, int D>
+// MN-major, 128B-swizzled operand: 64-element rows along N, 8-row groups
+// (along K) 1024 bytes apart, 64-wide N blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// Four rows y0..y3 of a tensor map whose box is one row of 64 elements.
+__device__ __forceinline__ void tma_gather4(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
+                                            int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(sm100::smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------- own chunk + counts (tcgen05)
+// One CTA per tile of 128 rows: P = 128/G consecutive positions of the G query
+// heads of one kv head.  The tile's keys are the NK = max(64, P) keys of the
+// chunks that hold those positions; S = Q K^T and O = P V run on tcgen05 and
+// one thread per row applies the causal own-chunk mask.  Per row it also forms
+// the fusion normaliser M' = log(sum_kept exp(s^) + exp(lse_own)), writes the
+// own chunk's weighted output exp(lse_own - M') softmax(s) V (= exp(s - M') V)
+// to the fp32 accumulator, and counts each kept (row, slot) pair under its key,
+// keeping the pair's rank within the key for the fill pass.
+template <int D>
+struct CcOwn {
+  static constexpr int M = 128;
+  static constexpr int KATOMS = D / 64;
+  static constexpr uint32_t ATOM = 128 * 128;   // 128 rows x 128 bytes
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = KATOMS * ATOM;
+  static constexpr uint32_t OFF_V = OFF_K + KATOMS * ATOM;
+  // P (up to 128 keys = two atoms) overwrites Q and K once S = Q K^T is done
+  static constexpr uint32_t OFF_P = OFF_Q;
+  static constexpr uint32_t OFF_BAR = OFF_V + KATOMS * ATOM;
+  static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+  // S (NK <= 128 columns) is read out before P V overwrites its first D columns
+  static constexpr uint32_t TMEM_COLS = 128;
+};
+
+struct CcOwnParams {
+  CcDims c;
+  const int32_t* ids;
+  const float* scores;
+  float* oacc;
+  float* rowstat;
+  float* lse_own;
+  int32_t* counts;
+  int32_t* ranks;
+  int P;            // positions per tile
+  int n_tiles;      // tiles per kv head
+};
+
+template <int D>
 __global__ void __launch_bounds__(128)
-cc_own_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-              const int32_t* __restrict__ ids, const float* __restrict__ scores, float* __restrict__ oacc,
-              float* __restrict__ rowstat, float* __restrict__ lse_own, int32_t* __restrict__ counts,
-              const CcDims c, int64_t n_rows) {
-  using L = RowLayout<T, D>;
-  constexpr int E = L::E, LPK = L::LPK;
-  const int lane = threadIdx.x & 31, sub = lane % LPK;
-  const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= n_rows) return;
-  const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
-  const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
-  const int64_t bh = b * c.Hkv + hq / c.G;
-  const T* kbh = k + bh * c.n_tok * D;
-  const T* vbh = v + bh * c.n_tok * D;
-  float qv[E];
-  Vec16<T>::load(q + row * D + sub * E, qv);
-  const int64_t own = i / kChunk;
-  float oc[E];
-  const float lo = attend_range<T, D>(qv, kbh, vbh, own * kChunk, i + 1, c.tau, oc);
-  // fusion normaliser over the valid selected chunks and the own chunk
-  float M = lo;
-  for (int t = lane; t < c.K; t += 32) {
-    const int32_t ci = __ldg(ids + row * c.K + t);
-    if (ci >= 0 && ci < own) M = fmaxf(M, __ldg(scores + row * c.K + t));
+cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const CcOwnParams p) {
+  using C = CcOwn<D>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+  uint64_t* ld_bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* mma_bar = ld_bar + 1;
+  uint64_t* done_bar = ld_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 28);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const CcDims& c = p.c;
+  const int P = p.P, G = c.G;
+  const int NK = P >= kChunk ? P : kChunk;
+  const int tile = int(blockIdx.x);
+  const int64_t bh = blockIdx.y, b = bh / c.Hkv, h = bh % c.Hkv;
+  const int64_t p0 = int64_t(tile) * P;
+  const int64_t kbase = (p0 / kChunk) * kChunk;
+
+  if (tid == 0) {
+    mbar_init(ld_bar, 1);
+    mbar_init(mma_bar, 1);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    const uint32_t kv_bytes = uint32_t(NK) * 128;
+    mbar_arrive_expect_tx(ld_bar, C::KATOMS * (C::ATOM + 2 * kv_bytes));
+    for (int g = 0; g < G; ++g) {
+      const int y = int((b * c.Hq + h * G + g) * c.n_tok + p0);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float Z = 0.f;
-  for (int t = lane; t < c.K; t += 32) {
-    const int32_t ci = __ldg(ids + row * c.K + t);
-    if (ci < 0) continue;
-    if (ci >= own) {
-      record_error(HILS_ERR_DEVICE_BOUNDS);
-      continue;
+      for (int a = 0; a < C::KATOMS; ++a) tma_load_2d(smem + C::OFF_Q + a * C::ATOM + g * P * 128, &tm_q, ld_bar, a * 64, y);
     }
-    Z += expf(__ldg(scores + row * c.K + t) - M);
-    atomicAdd(counts + cc_key(c, bh, i, ci), 1);
-  }
+    const int yk = int(bh * c.n_tok + kbase);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
-  Z += expf(lo - M);
-  const float Mp = M + logf(Z);
-  const float w_own = expf(lo - Mp);
-  if (lane < LPK) {
-    float* dst = oacc + row * D + sub * E;
-#pragma unroll
-    for (int e = 0; e < E; e += 4)
-      *reinterpret_cast<float4*>(dst + e) = make_float4(w_own * oc[e], w_own * oc[e + 1], w_own * oc[e + 2], w_own * oc[e + 3]);
+    for (int a = 0; a < C::KATOMS; ++a) {
+      tma_load_2d(smem + C::OFF_K + a * C::ATOM, &tm_k, ld_bar, a * 64, yk);
+      tma_load_2d(smem + C::OFF_V + a * C::ATOM, &tm_v, ld_bar, a * 64, yk);
+    }
   }
-  if (lane == 0) {
-    rowstat[row] = Mp;
-    if (lse_own) lse_own[row] = lo;
+  // this thread's row and its kept slots (loads overlap the copies and the MMA)
+  const int r = tid;                         // TMEM lane == row of the tile
+  const int g = r / P;
+  const int64_t pos = p0 + r % P;
+  const bool live = pos < c.n_tok;
+  const int64_t row = (b * c.Hq + h * G + g) * c.n_tok + pos;
+  const int64_t own = pos / kChunk;
+  float smax = -INFINITY;
+  if (live) {
+    if ((c.K & 3) == 0) {
+      const int4* i4 = reinterpret_cast<const int4*>(p.ids + row * c.K);
+      const float4* s4 = reinterpret_cast<const float4*>(p.scores + row * c.K);
+      for (int t = 0; t < c.K / 4; ++t) {
+        const int4 ci = __ldg(i4 + t);
+        const float4 sc = __ldg(s4 + t);
+        if (ci.x >= 0 && ci.x < own) smax = fmaxf(smax, sc.x);
+        if (ci.y >= 0 && ci.y < own) smax = fmaxf(smax, sc.y);
+        if (ci.z >= 0 && ci.z < own) smax = fmaxf(smax, sc.z);
+        if (ci.w >= 0 && ci.w < own) smax = fmaxf(smax, sc.w);
+      }
+    } else {
+      for (int t = 0; t < c.K; ++t) {
+        const int32_t ci = __ldg(p.ids + row * c.K + t);
+        if (ci >= 0 && ci < own) smax = fmaxf(smax, __ldg(p.scores + row * c.K + t));
+      }
+    }
+  }
+  bool ok = true;
+  if (tid == 0) {
+    ok = mbar_wait(ld_bar, 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t sq = smem_u32(smem + C::OFF_Q), sk = smem_u32(smem + C::OFF_K);
+      const uint32_t idesc = idesc_bf16(C::M, NK);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = uint32_t((kk >> 2) * C::ATOM + (kk & 3) * 32);
+        mma_bf16(tmem, desc_sw128(sq + off), desc_sw128(sk + off), idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(mma_bar);
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) ok = mbar_wait(mma_bar, 0, abort_flag);
+  tc_fence_after();
+  // causal softmax statistics over the own chunk's keys: tile key j is key
+  // kbase + j, valid for j in [jlo, jhi] (same chunk as the row, not after it)
+  const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
+  const int jlo = int(own * kChunk - kbase), jhi = int(pos - kbase);
+  const float k2 = c.tau * 1.4426950408889634f;
+  float m = -INFINITY;
+#pragma unroll 1
+  for (int q4 = 0; q4 < NK / 32; ++q4) {
+    float tmp[32];
+    tmem_ld32(t_row + uint32_t(q4 * 32), tmp);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const int j = q4 * 32 + t;
+      if (j >= jlo && j <= jhi) m = fmaxf(m, tmp[t]);
+    }
+  }
+  float l = 0.f;
+#pragma unroll 1
+  for (int q4 = 0; q4 < NK / 32; ++q4) {
+    float tmp[32];
+    tmem_ld32(t_row + uint32_t(q4 * 32), tmp);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const int j = q4 * 32 + t;
+      if (j >= jlo && j <= jhi) l += ex2_approx(fmaf(tmp[t], k2, -m * k2));
+    }
+  }
+  const float lse = m * c.tau + logf(l);   // log sum_j exp(tau s_j)
+  // fusion normaliser and pair counts
+  float Mp = lse;
+  if (live) {
+    const float Mx = fmaxf(smax, lse);
+    float Z = expf(lse - Mx);
+    const int64_t bhk = bh;
+    // eight slots at a time so that the counting atomics are in flight together
+    for (int t0 = 0; t0 < c.K; t0 += 8) {
+      int32_t rk[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u;
+        rk[u] = -1;
+        if (t >= c.K) continue;
+        const int32_t ci = __ldg(p.ids + row * c.K + t);
+        if (ci < 0) continue;
+        if (ci >= own) {
+          record_error(HILS_ERR_DEVICE_BOUNDS);
+          continue;
+        }
+        Z += expf(__ldg(p.scores + row * c.K + t) - Mx);
+        rk[u] = atomicAdd(p.counts + cc_key(c, bhk, pos, ci), 1);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (rk[u] >= 0) p.ranks[row * c.K + t0 + u] = rk[u];
+    }
+    Mp = Mx + logf(Z);
+    p.rowstat[row] = Mp;
+    if (p.lse_own) p.lse_own[row] = lse;
+  }
+  // P = exp(tau s - M') on the causal own-chunk keys, bf16, 128B-swizzled K-major
+  const float mb = Mp * 1.4426950408889634f;
+#pragma unroll 1
+  for (int q4 = 0; q4 < NK / 32; ++q4) {
+    float tmp[32];
+    tmem_ld32(t_row + uint32_t(q4 * 32), tmp);
+    uint8_t* prow = smem + C::OFF_P + (q4 >> 1) * C::ATOM + r * 128;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {           // four 16-byte pieces of 8 keys
+      uint32_t wd[4];
+#pragma unroll
+      for (int v2 = 0; v2 < 4; ++v2) {
+        float e2[2];
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+          const int tt = 8 * t + 2 * v2 + z;
+          const int j = q4 * 32 + tt;
+          e2[z] = (live && j >= jlo && j <= jhi) ? ex2_approx(fmaf(tmp[tt], k2, -mb)) : 0.f;
+        }
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(e2[0], e2[1]);
+        wd[v2] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      const int piece = (q4 & 1) * 4 + t;   // 16-byte piece within the 128-byte row
+      *reinterpret_cast<uint4*>(prow + ((piece ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    const uint32_t sp = smem_u32(smem + C::OFF_P), svv = smem_u32(smem + C::OFF_V);
+    const uint32_t idesc = idesc_bf16(C::M, D) | (1u << 16);
+    for (int kk = 0; kk < NK / 16; ++kk)
+      mma_bf16(tmem, desc_sw128(sp + (kk >> 2) * C::ATOM + (kk & 3) * 32),
+               desc_sw128_mn(svv + kk * 2048, C::ATOM), idesc, kk > 0 ? 1u : 0u);
+    mma_commit(mma_bar);
+  }
+  if (ok) ok = mbar_wait(mma_bar, 1, abort_flag);
+  tc_fence_after();
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    float o[32];
+    tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(cc * 32), o);
+    if (live && ok) {
+      float* dst = p.oacc + row * D + cc * 32;
+#pragma unroll
+      for (int t = 0; t < 32; t += 4) *reinterpret_cast<float4*>(dst + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && !ok) {
+    // after a time-out: let the copies land and any issued MMA finish before TMEM is freed
+    mbar_wait_drain(ld_bar, 0);
+    mma_commit(done_bar);
+    mbar_wait_drain(done_bar, 0);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-// ---------------------------------------------------------------- scan (one CTA)
+// ---------------------------------------------------------------- scan (three passes)
 constexpr int kCcTileRows = 128;
+constexpr int kScanBlock = 4096;   // keys per CTA (256 threads x 16)
 
-// Each of the 1024 threads owns a contiguous segment of keys: local sums,
-// one block-wide exclusive scan, then the segment's offsets.
-__global__ void __launch_bounds__(1024)
-cc_scan_kernel(const int32_t* __restrict__ counts, int64_t n_keys, int64_t* __restrict__ offsets,
-               int32_t* __restrict__ tile_start, int32_t* __restrict__ cursor) {
-  __shared__ int64_t s_a[32], s_t[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t seg = (n_keys + 1023) / 1024;
-  const int64_t k0 = tid * seg, k1 = (k0 + seg < n_keys) ? k0 + seg : n_keys;
-  int64_t sa = 0, st = 0;
-  for (int64_t kk = k0; kk < k1; ++kk) {
-    const int64_t cnt = counts[kk];
-    sa += cnt;
-    st += (cnt + kCcTileRows - 1) / kCcTileRows;
+__device__ __forceinline__ int64_t cc_tiles(int64_t cnt) { return (cnt + kCcTileRows - 1) / kCcTileRows; }
+
+// pass 1: per-CTA totals of pairs and tiles
+__global__ void __launch_bounds__(256)
+cc_scan_sums_kernel(const int32_t* __restrict__ counts, int64_t n_keys, int64_t* __restrict__ sums) {
+  __shared__ int64_t sa[8], st[8];
+  const int64_t k0 = int64_t(blockIdx.x) * kScanBlock + threadIdx.x * 16;
+  int64_t a = 0, t = 0;
+#pragma unroll 4
+  for (int e = 0; e < 16; ++e) {
+    const int64_t kk = k0 + e;
+    const int64_t c = kk < n_keys ? counts[kk] : 0;
+    a += c;
+    t += cc_tiles(c);
   }
-  int64_t a = sa, t = st;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    t += __shfl_xor_sync(0xffffffffu, t, o);
+  }
+  if ((threadIdx.x & 31) == 0) { sa[threadIdx.x >> 5] = a; st[threadIdx.x >> 5] = t; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t A = 0, T = 0;
+    for (int w = 0; w < 8; ++w) { A += sa[w]; T += st[w]; }
+    sums[2 * blockIdx.x] = A;
+    sums[2 * blockIdx.x + 1] = T;
+  }
+}
+
+// pass 2 (one CTA): exclusive prefix of the per-CTA totals, in place; also the grand totals
+__global__ void __launch_bounds__(1024)
+cc_scan_blocks_kernel(int64_t* __restrict__ sums, int64_t n_blocks, int64_t n_keys, int64_t* __restrict__ offsets,
+                      int32_t* __restrict__ tile_start) {
+  __shared__ int64_t wa[32], wt[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t per = (n_blocks + 1023) / 1024;
+  const int64_t b0 = tid * per, b1 = (b0 + per < n_blocks) ? b0 + per : n_blocks;
+  int64_t a = 0, t = 0;
+  for (int64_t b = b0; b < b1; ++b) { a += sums[2 * b]; t += sums[2 * b + 1]; }
+  int64_t ia = a, it = t;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int64_t ya = __shfl_up_sync(0xffffffffu, a, o), yt = __shfl_up_sync(0xffffffffu, t, o);
-    if (lane >= o) { a += ya; t += yt; }
+    const int64_t ya = __shfl_up_sync(0xffffffffu, ia, o), yt = __shfl_up_sync(0xffffffffu, it, o);
+    if (lane >= o) { ia += ya; it += yt; }
   }
-  if (lane == 31) { s_a[warp] = a; s_t[warp] = t; }
+  if (lane == 31) { wa[warp] = ia; wt[warp] = it; }
   __syncthreads();
-  int64_t pa = 0, pt = 0, ta = 0, tt = 0;
+  int64_t pa = 0, pt = 0, TA = 0, TT = 0;
   for (int w = 0; w < 32; ++w) {
-    if (w < warp) { pa += s_a[w]; pt += s_t[w]; }
-    ta += s_a[w];
-    tt += s_t[w];
+    if (w < warp) { pa += wa[w]; pt += wt[w]; }
+    TA += wa[w];
+    TT += wt[w];
   }
-  int64_t ra = pa + a - sa, rt = pt + t - st;   // exclusive prefix of this segment
-  for (int64_t kk = k0; kk < k1; ++kk) {
-    const int64_t cnt = counts[kk];
-    offsets[kk] = ra;
-    tile_start[kk] = int32_t(rt);
-    cursor[kk] = 0;
-    ra += cnt;
-    rt += (cnt + kCcTileRows - 1) / kCcTileRows;
+  int64_t ra = pa + ia - a, rt = pt + it - t;
+  for (int64_t b = b0; b < b1; ++b) {
+    const int64_t xa = sums[2 * b], xt = sums[2 * b + 1];
+    sums[2 * b] = ra;
+    sums[2 * b + 1] = rt;
+    ra += xa;
+    rt += xt;
   }
   if (tid == 0) {
-    offsets[n_keys] = ta;
-    tile_start[n_keys] = int32_t(tt);
+    offsets[n_keys] = TA;
+    tile_start[n_keys] = int32_t(TT);
+  }
+}
+
+// pass 3: per-key offsets, tile starts and the tile -> key table
+__global__ void __launch_bounds__(256)
+cc_scan_apply_kernel(const int32_t* __restrict__ counts, const CcDims c, const int64_t* __restrict__ sums,
+                     int64_t* __restrict__ offsets, int32_t* __restrict__ tile_start, int4* __restrict__ items) {
+  const int64_t n_keys = c.n_keys;
+  __shared__ int64_t sa[8], st[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t k0 = int64_t(blockIdx.x) * kScanBlock + threadIdx.x * 16;
+  int64_t cnt[16];
+  int64_t a = 0, t = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int64_t kk = k0 + e;
+    cnt[e] = kk < n_keys ? counts[kk] : 0;
+    a += cnt[e];
+    t += cc_tiles(cnt[e]);
+  }
+  int64_t ia = a, it = t;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t ya = __shfl_up_sync(0xffffffffu, ia, o), yt = __shfl_up_sync(0xffffffffu, it, o);
+    if (lane >= o) { ia += ya; it += yt; }
+  }
+  if (lane == 31) { sa[warp] = ia; st[warp] = it; }
+  __syncthreads();
+  int64_t pa = sums[2 * blockIdx.x], pt = sums[2 * blockIdx.x + 1];
+  for (int w = 0; w < warp; ++w) { pa += sa[w]; pt += st[w]; }
+  int64_t ra = pa + ia - a, rt = pt + it - t;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int64_t kk = k0 + e;
+    if (kk >= n_keys) break;
+    offsets[kk] = ra;
+    tile_start[kk] = int32_t(rt);
+    const int64_t tl = cc_tiles(cnt[e]);
+    const int64_t bh = kk / (int64_t(c.n_win) * c.nc), chunk = kk % c.nc;
+    const int32_t kvrow = int32_t(bh * c.n_tok + chunk * kChunk);
+    for (int64_t u = 0; u < tl; ++u) {
+      const int64_t left = cnt[e] - u * kCcTileRows;
+      items[rt + u] = make_int4(int32_t(ra + u * kCcTileRows), kvrow, int32_t(left < kCcTileRows ? left : kCcTileRows), 0);
+    }
+    ra += cnt[e];
+    rt += tl;
   }
 }
 
 // ---------------------------------------------------------------- fill the inverted index
+// ranks[slot] is the slot's position within its key's list, taken when the
+// pair was counted, so filling is a plain scatter of the pair's global row id
+// and its fusion factor s^ - M'.
 __global__ void __launch_bounds__(256)
-cc_fill_kernel(const int32_t* __restrict__ ids, const int64_t* __restrict__ offsets, int32_t* __restrict__ cursor,
-               int32_t* __restrict__ entries, const CcDims c, int64_t n_slots) {
+cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const float* __restrict__ scores,
+               const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int32_t* __restrict__ e_row,
+               float* __restrict__ e_fac, const CcDims c, int64_t n_slots) {
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n_slots) return;
   const int32_t ci = __ldg(ids + idx);
   if (ci < 0) return;
   const int64_t row = idx / c.K;
-  const int slot = int(idx % c.K);
   const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
+  if (ci >= i / kChunk) return;   // out of range: recorded when counting
   const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
-  if (ci >= i / kChunk) return;   // recorded by cc_own_kernel
   const int64_t bh = b * c.Hkv + hq / c.G;
-  const int64_t key = cc_key(c, bh, i, ci);
-  const int32_t at = atomicAdd(cursor + key, 1);
-  const int64_t row_in_bh = (hq % c.G) * c.n_tok + i;   // (g, position) within the kv head
-  entries[offsets[key] + at] = int32_t((row_in_bh << 6) | slot);
+  const int64_t at = offsets[cc_key(c, bh, i, ci)] + __ldg(ranks + idx);
+  e_row[at] = int32_t(row);
+  e_fac[at] = __ldg(scores + idx) - __ldg(rowstat + row);
 }
 
 // ---------------------------------------------------------------- accumulator -> output
@@ -185,86 +489,100 @@ cc_final_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ o, i
 }
 
 // ---------------------------------------------------------------- chunk tiles on tcgen05
+// Warp-specialised, two-stage pipeline per CTA over its tiles (item = blockIdx.x
+// + j * gridDim.x):
+//   warp 0       producer: the tile's entries -> row ids (shared memory), then
+//                one lane issues TMA loads of the chunk's K and V and 32*d/64
+//                gather4 loads of the rows' queries (128B swizzle);
+//   warp 1       one lane issues S = Q K^T into TMEM buffer b, and once the
+//                softmax warps have written P, O = P V into TMEM buffer b;
+//   warps 2-5    one thread per row: the fusion factor s^ - M' (two loads),
+//                softmax of its 64 scores into P (bf16, shared memory), then
+//                its row of O added to the accumulator (16-byte reductions).
+// Stage / TMEM buffer b = j & 1, so loading tile j+1 and the MMAs of tile j+1
+// overlap the softmax and reductions of tile j.
 template <int D>
 struct CcTc {
   static constexpr int M = kCcTileRows;
   static constexpr int KATOMS = D / 64;
+  static constexpr int NS = 3;                      // shared-memory stages
   static constexpr uint32_t Q_ATOM = M * 128;       // 16 KB
   static constexpr uint32_t KV_ATOM = kChunk * 128; // 8 KB
   static constexpr uint32_t Q_BYTES = KATOMS * Q_ATOM;
   static constexpr uint32_t K_BYTES = KATOMS * KV_ATOM;
   static constexpr uint32_t P_BYTES = M * 128;      // 128 rows x 64 keys bf16
-  static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES, OFF_P = OFF_V + K_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
-  static constexpr uint32_t TMEM_COLS = D == 64 ? 128 : 256;   // S: 64 columns, O: D columns
-  static constexpr uint32_t SMEM_MIN = OFF_BAR + 64 + 1024;
-  // at most 512 / TMEM_COLS CTAs may share an SM, or a tcgen05.alloc could wait
-  // for columns that a co-resident persistent CTA never frees: request enough
-  // shared memory that no more CTAs fit.
+  // P overwrites the stage's Q tile once S = Q K^T is done
+  static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES;
+  static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES, OFF_P = 0;
+  static constexpr uint32_t OFF_META = NS * STAGE;                // per stage: rows[128] i32, fac[128] f32, n
+  static constexpr uint32_t META = M * 4 + M * 4 + 16;
+  static constexpr uint32_t OFF_BAR = OFF_META + NS * META;
+  static constexpr uint32_t SMEM_MIN = OFF_BAR + 16 * 8 + 32 + 1024;
+  static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;    // S[2] x 64 + O[2] x D
   static constexpr uint32_t MAX_CTAS = 512 / TMEM_COLS;
+  // at most MAX_CTAS CTAs may share an SM, or a tcgen05.alloc could wait for
+  // columns that a co-resident persistent CTA never frees
   static constexpr uint32_t SMEM_FLOOR = 233472u / (MAX_CTAS + 1) + 1024u;
   static constexpr uint32_t SMEM = SMEM_MIN > SMEM_FLOOR ? SMEM_MIN : SMEM_FLOOR;
+  static constexpr uint32_t TX_BYTES = M * D * 2 + 2 * K_BYTES;
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16(M, kChunk);
   // P (K-major) x V (MN-major: d contiguous in each key row)
   static constexpr uint32_t IDESC_O = sm100::idesc_bf16(M, D) | (1u << 16);
+  static constexpr int THREADS = 192;
+  static_assert(P_BYTES <= Q_BYTES, "P reuses the Q tile");
 };
-
-// MN-major, 128B-swizzled operand: 64-element rows along N, 8-row groups
-// (along K) 1024 bytes apart, 64-wide N blocks `lbo` bytes apart.
-__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
-  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) | (uint64_t(1024 >> 4) << 32) |
-         (uint64_t(1) << 46) | (uint64_t(2) << 61);
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 struct CcTcParams {
   CcDims c;
-  const int64_t* offsets;
-  const int32_t* tile_start;
-  const int32_t* entries;
-  const float* scores;
-  const float* rowstat;
-  const __nv_bfloat16* q;
+  const int32_t* tile_start;   // [n_keys + 1]; the last entry is the number of tiles
+  const int4* items;           // per tile: first entry, K/V row, pair count
+  const int32_t* e_row;        // per entry: global row id
+  const float* e_fac;          // per entry: s^ - M'
   float* oacc;
 };
 
 template <int D>
-__global__ void __launch_bounds__(128)
-cc_attend_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const CcTcParams p) {
+__global__ void __launch_bounds__(CcTc<D>::THREADS, 1)
+cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const CcTcParams p) {
   using C = CcTc<D>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
-  uint64_t* kv_bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* mma_bar = kv_bar + 1;
-  uint64_t* done_bar = kv_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 24);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 28);
-  int64_t* s_item = reinterpret_cast<int64_t*>(smem + C::OFF_BAR + 32);   // key, first entry, count
-  const uint32_t sQ = smem_u32(smem + C::OFF_Q), sK = smem_u32(smem + C::OFF_K);
-  const uint32_t sV = smem_u32(smem + C::OFF_V), sP = smem_u32(smem + C::OFF_P);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* load_full = bars;        // [NS] producer -> MMA, softmax
+  uint64_t* load_empty = bars + 3;   // [NS] MMA (after PV) -> producer
+  uint64_t* p_full = bars + 6;       // [NS] softmax -> MMA
+  uint64_t* s_full = bars + 9;       // [2] MMA -> softmax
+  uint64_t* o_full = bars + 11;      // [2] MMA -> epilogue
+  uint64_t* t_empty = bars + 13;     // [2] epilogue -> MMA
+  uint64_t* done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 16 * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 16 * 8 + 4);
+  int* issued_slot = reinterpret_cast<int*>(smem + C::OFF_BAR + 16 * 8 + 8);
+  int* consumed_slot = reinterpret_cast<int*>(smem + C::OFF_BAR + 16 * 8 + 12);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const CcDims& c = p.c;
 
   if (tid == 0) {
-    mbar_init(kv_bar, 1);
-    mbar_init(mma_bar, 1);
-    mbar_init(done_bar, 1);
+    for (int t = 0; t < C::NS; ++t) {
+      mbar_init(&load_full[t], 1);
+      mbar_init(&load_empty[t], 1);
+      mbar_init(&p_full[t], 4);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&o_full[t], 1);
+      mbar_init(&t_empty[t], 4);
+    }
+    mbar_init(done, 1);
     *abort_flag = 0;
+    *issued_slot = 0;
+    *consumed_slot = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -272,159 +590,186 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_lane = uint32_t(warp * 32) << 16;
   const int32_t n_items = p.tile_start[c.n_keys];
-  uint32_t kv_phase = 0, mma_phase = 0;
-  bool ok = true, issued_mma = false;
+  const int n_my = n_items > int32_t(blockIdx.x) ? (n_items - 1 - int32_t(blockIdx.x)) / int32_t(gridDim.x) + 1 : 0;
 
-  for (int32_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-    if (tid == 0) {
-      // key = last index with tile_start[key] <= item
-      int64_t lo = 0, hi = c.n_keys - 1;
-      while (lo < hi) {
-        const int64_t mid = (lo + hi + 1) >> 1;
-        if (p.tile_start[mid] <= item) lo = mid; else hi = mid - 1;
-      }
-      const int64_t key = lo;
-      const int64_t t = item - p.tile_start[key];
-      const int64_t first = p.offsets[key] + t * C::M;
-      const int64_t cnt = p.offsets[key + 1] - first;
-      s_item[0] = key;
-      s_item[1] = first;
-      s_item[2] = cnt < C::M ? cnt : C::M;
-      // chunk K and V tiles
-      const int64_t chunk = key % c.nc;
-      const int64_t bh = key / (c.nc * c.n_win);
-      const int y = int(bh * c.n_tok + chunk * kChunk);
-      mbar_arrive_expect_tx(kv_bar, 2 * C::K_BYTES);
-#pragma unroll
-      for (int a = 0; a < C::KATOMS; ++a) {
-        tma_load_2d(smem + C::OFF_K + a * C::KV_ATOM, &tm_k, kv_bar, a * 64, y);
-        tma_load_2d(smem + C::OFF_V + a * C::KV_ATOM, &tm_v, kv_bar, a * 64, y);
-      }
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
     }
-    __syncthreads();
-    const int64_t key = s_item[0], first = s_item[1];
-    const int n = int(s_item[2]);
-    const int64_t bh = key / (c.nc * c.n_win);
-    const int64_t b = bh / c.Hkv, h = bh % c.Hkv;
-    // row of this thread and its fusion factor s^ - M'
-    int64_t grow = -1;
-    float fac = 0.f;
-    if (tid < n) {
-      const int32_t e = p.entries[first + tid];
-      const int64_t row_in_bh = e >> 6;
-      const int slot = e & 63;
-      const int64_t g = row_in_bh / c.n_tok, pos = row_in_bh % c.n_tok;
-      grow = (b * c.Hq + h * c.G + g) * c.n_tok + pos;
-      fac = p.scores[grow * c.K + slot] - p.rowstat[grow];
-      const __nv_bfloat16* src = p.q + grow * D;
+    // metadata of tile j is loaded into registers while tile j-1 is issued
+    int4 rec = make_int4(0, 0, 1, 0);
+    int32_t nrow[C::M / 32];
+    float nfac[C::M / 32];
+    auto fetch = [&](int jj) {
+      const int32_t item = int32_t(blockIdx.x) + jj * int32_t(gridDim.x);
+      rec = __ldg(p.items + item);
 #pragma unroll
-      for (int a = 0; a < C::KATOMS; ++a)
+      for (int q4 = 0; q4 < C::M / 32; ++q4) {
+        const int r = q4 * 32 + lane;
+        const int at = rec.x + (r < rec.z ? r : rec.z - 1);
+        nrow[q4] = __ldg(p.e_row + at);
+        nfac[q4] = __ldg(p.e_fac + at);
+      }
+    };
+    if (n_my > 0) fetch(0);
+    int j = 0;
+    for (; j < n_my; ++j) {
+      const int s = j % C::NS, u = j / C::NS;
+      const int4 cur = rec;
+      int32_t crow[C::M / 32];
+      float cfac[C::M / 32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          cp_async16(sQ + a * C::Q_ATOM + tid * 128 + ((j ^ (tid & 7)) << 4), src + a * 64 + j * 8);
+      for (int q4 = 0; q4 < C::M / 32; ++q4) { crow[q4] = nrow[q4]; cfac[q4] = nfac[q4]; }
+      if (j + 1 < n_my) fetch(j + 1);
+      if (!mbar_wait(&load_empty[s], (u & 1) ^ 1, abort_flag)) break;
+      uint8_t* meta = smem + C::OFF_META + s * C::META;
+      int32_t* rows = reinterpret_cast<int32_t*>(meta);
+      float* facs = reinterpret_cast<float*>(meta + C::M * 4);
+#pragma unroll
+      for (int q4 = 0; q4 < C::M / 32; ++q4) {
+        rows[q4 * 32 + lane] = crow[q4];
+        facs[q4 * 32 + lane] = cfac[q4];
+      }
+      if (lane == 0) reinterpret_cast<int32_t*>(meta + C::M * 8)[0] = cur.z;
+      __syncwarp();
+      if (lane == 0) {
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&load_full[s], C::TX_BYTES);
+#pragma unroll
+        for (int a = 0; a < C::KATOMS; ++a) {
+          tma_load_2d(st + C::OFF_K + a * C::KV_ATOM, &tm_k, &load_full[s], a * 64, cur.y);
+          tma_load_2d(st + C::OFF_V + a * C::KV_ATOM, &tm_v, &load_full[s], a * 64, cur.y);
+        }
+        const uint32_t qdst = smem_u32(st + C::OFF_Q);
+#pragma unroll 4
+        for (int r = 0; r < C::M; r += 4) {
+#pragma unroll
+          for (int a = 0; a < C::KATOMS; ++a)
+            tma_gather4(qdst + a * C::Q_ATOM + r * 128, &tm_q, &load_full[s], a * 64, rows[r], rows[r + 1],
+                        rows[r + 2], rows[r + 3]);
+        }
+      }
+      __syncwarp();
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncthreads();
-    // S = Q K^T
-    if (tid == 0) {
-      ok = mbar_wait(kv_bar, kv_phase, abort_flag);
-      if (ok) {
+    if (lane == 0) *issued_slot = j;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int j = 0;
+      for (; j < n_my; ++j) {
+        const int s = j % C::NS, u = j / C::NS, b = j & 1, ub = j >> 1;
+        if (!mbar_wait(&load_full[s], u & 1, abort_flag)) break;
+        if (!mbar_wait(&t_empty[b], (ub & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::STAGE);
+        const uint32_t sq = st + C::OFF_Q, sk = st + C::OFF_K, sv = st + C::OFF_V, sp = st + C::OFF_P;
+        const uint32_t t_s = tmem + uint32_t(b * kChunk), t_o = tmem + uint32_t(2 * kChunk + b * D);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = uint32_t((kk >> 2) * C::Q_ATOM + (kk & 3) * 32);
           const uint32_t offk = uint32_t((kk >> 2) * C::KV_ATOM + (kk & 3) * 32);
-          mma_bf16(tmem, desc_sw128(sQ + off), desc_sw128(sK + offk), C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_bf16(t_s, desc_sw128(sq + off), desc_sw128(sk + offk), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(mma_bar);
-        issued_mma = true;
+        mma_commit(&s_full[b]);
+        if (!mbar_wait(&p_full[s], u & 1, abort_flag)) { ++j; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          mma_bf16(t_o, desc_sw128(sp + kk * 32), desc_sw128_mn(sv + kk * 2048, C::KV_ATOM), C::IDESC_O,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(&o_full[b]);
+        mma_commit(&load_empty[s]);
       }
+      *consumed_slot = j;
+      mma_commit(done);
     }
-    kv_phase ^= 1;
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    ok = mbar_wait(mma_bar, mma_phase, abort_flag);
-    mma_phase ^= 1;
-    tc_fence_after();
-    {
-      float s[64];
-      float tmp[32];
-      tmem_ld32(tmem + t_lane + 0, tmp);
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t t_lane = uint32_t(quarter * 32) << 16;
+    const float k2 = c.tau * 1.4426950408889634f;   // scores in log2 units
+    for (int j = 0; j < n_my; ++j) {
+      const int s = j % C::NS, u = j / C::NS, b = j & 1, ub = j >> 1;
+      if (!mbar_wait(&load_full[s], u & 1, abort_flag)) break;
+      const uint8_t* meta = smem + C::OFF_META + s * C::META;
+      const int n = reinterpret_cast<const int32_t*>(meta + C::M * 8)[0];
+      const bool live = r < n;
+      const int64_t grow = reinterpret_cast<const int32_t*>(meta)[r];
+      const float fac = reinterpret_cast<const float*>(meta + C::M * 4)[r];
+      if (!mbar_wait(&s_full[b], ub & 1, abort_flag)) break;
+      tc_fence_after();
+      float sc[64];
+      {
+        float tmp[32];
+        tmem_ld32(tmem + t_lane + uint32_t(b * kChunk), tmp);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) s[j] = tmp[j];
-      tmem_ld32(tmem + t_lane + 32, tmp);
+        for (int t = 0; t < 32; ++t) sc[t] = tmp[t];
+        tmem_ld32(tmem + t_lane + uint32_t(b * kChunk + 32), tmp);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) s[32 + j] = tmp[j];
-      const float k2 = c.tau * 1.4426950408889634f;   // scores in log2 units
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) m = fmaxf(m, s[j]);
-      const float mb = m * k2;
-      float l = 0.f;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        s[j] = exp2f(fmaf(s[j], k2, -mb));
-        l += s[j];
+        for (int t = 0; t < 32; ++t) sc[32 + t] = tmp[t];
       }
-      const float w = expf(fac) / l;
-      uint8_t* prow = smem + C::OFF_P + tid * 128;
+      uint8_t* prow = smem + s * C::STAGE + C::OFF_P + r * 128;
+      if (live) {
+        float m = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t wd[4] = {0u, 0u, 0u, 0u};
-        if (tid < n) {
+        for (int t = 0; t < 64; ++t) m = fmaxf(m, sc[t]);
+        const float mb = m * k2;
+        float l = 0.f;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(s[8 * j + 2 * u] * w, s[8 * j + 2 * u + 1] * w);
-            wd[u] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int t = 0; t < 64; ++t) {
+          sc[t] = ex2_approx(fmaf(sc[t], k2, -mb));
+          l += sc[t];
+        }
+        const float w = expf(fac) / l;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          uint32_t wd[4];
+#pragma unroll
+          for (int v2 = 0; v2 < 4; ++v2) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(sc[8 * t + 2 * v2] * w, sc[8 * t + 2 * v2 + 1] * w);
+            wd[v2] = *reinterpret_cast<uint32_t*>(&h2);
           }
+          *reinterpret_cast<uint4*>(prow + ((t ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
-        *reinterpret_cast<uint4*>(prow + ((j ^ (tid & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) *reinterpret_cast<uint4*>(prow + (t << 4)) = make_uint4(0u, 0u, 0u, 0u);
       }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    // O = P V
-    if (tid == 0) {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
+      if (!mbar_wait(&o_full[b], ub & 1, abort_flag)) break;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < kChunk / 16; ++kk)
-        mma_bf16(tmem + 64, desc_sw128(sP + kk * 32), desc_sw128_mn(sV + kk * 2048, C::KV_ATOM), C::IDESC_O,
-                 kk > 0 ? 1u : 0u);
-      mma_commit(mma_bar);
-    }
-    __syncwarp();
-    ok = mbar_wait(mma_bar, mma_phase, abort_flag);
-    mma_phase ^= 1;
-    tc_fence_after();
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + t_lane + uint32_t(2 * kChunk + b * D + cc * 32), o);
+        if (live) {
+          float* dst = p.oacc + grow * D + cc * 32;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      float o[32];
-      tmem_ld32(tmem + t_lane + 64 + cc * 32, o);
-      if (grow >= 0) {
-        float* dst = p.oacc + grow * D + cc * 32;
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) red_add_v4(dst + j, o[j], o[j + 1], o[j + 2], o[j + 3]);
+          for (int t = 0; t < 32; t += 4) red_add_v4(dst + t, o[t], o[t + 1], o[t + 2], o[t + 3]);
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[b]);
     }
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
   }
-  // teardown: no copy or MMA may still be in flight when TMEM is freed
+  // ------------------------------------------------------------ teardown
   __syncthreads();
   if (tid == 0) {
-    if (!ok) mbar_wait_drain(kv_bar, kv_phase ^ 1);
-    if (issued_mma) {
-      mma_commit(done_bar);
-      mbar_wait_drain(done_bar, 0);
-    }
+    // loads still in flight (only after an abort): wait for them to land
+    for (int j = *consumed_slot; j < *issued_slot; ++j) mbar_wait_drain(&load_full[j % C::NS], (j / C::NS) & 1);
   }
-  __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
+    if (lane == 0 && n_my > 0) mbar_wait_drain(done, 0);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -241,9 +241,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int64_t lim = n_cand - cbase;
         uint32_t bits = 0;
         if (lim > 0) {
-          // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr)
+          // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
+          // four independent 8-bit chains keep the dependency depth short
+          uint32_t part[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int e = 0; e < 32; ++e) bits = __funnelshift_l(__float_as_uint(fmaf(-tau, v[e], thr)), bits, 1);
+          for (int e = 0; e < 8; ++e) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              part[q4] = __funnelshift_l(__float_as_uint(fmaf(-tau, v[8 * q4 + e], thr)), part[q4], 1);
+          }
+          bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
           if (lim < 32) bits &= ~(0xFFFFFFFFu >> int(lim));
         }
         if (__any_sync(0xffffffffu, bits != 0)) {

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUP
 EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_prefill_workspace_bytes",
            "hils_attn_prefill",
            "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
-           "hils_get_status", "hils_strerror", "hils_kernel_launches")
+           "hils_get_status", "hils_selftest_bounded_wait", "hils_strerror", "hils_kernel_launches")
 DECODE_FIXED_SCRATCH_BYTES = 16 << 20
 
 
@@ -62,6 +62,7 @@ def lib():
         L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_attn_decode_fixed_scratch.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P]
         L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
+        L.hils_selftest_bounded_wait.argtypes = [ctypes.c_int32, P]
         L.hils_strerror.argtypes = [ctypes.c_int]
         L.hils_strerror.restype = ctypes.c_char_p
         L.hils_kernel_launches.restype = ctypes.c_uint64
@@ -173,6 +174,10 @@ def hils_get_status(stream=None) -> int:
     v = ctypes.c_int32(0)
     _check("hils_get_status", lib().hils_get_status(ctypes.byref(v), _stream(stream)))
     return int(v.value)
+
+
+def hils_selftest_bounded_wait(limit_ms: int = 50, stream=None):
+    _check("hils_selftest_bounded_wait", lib().hils_selftest_bounded_wait(int(limit_ms), _stream(stream)))
 
 
 def hils_kernel_launches() -> int:

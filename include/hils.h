@@ -216,6 +216,16 @@ int hils_attn_decode_fixed_scratch(const hils_dims* dims, const void* q, const v
  */
 int hils_get_status(int32_t* host_status, hils_stream_t stream);
 
+/*
+ * Self-test of the bounded device waits that every tcgen05 kernel uses (no
+ * counterpart in the paper).  Launches one CTA whose thread waits for an
+ * mbarrier phase that nothing completes, with a limit of limit_ms
+ * milliseconds (1..2000).  The wait gives up, records HILS_ERR_DEVICE_TIMEOUT
+ * in the device status word and the kernel returns normally, so the context
+ * stays usable; read the result with hils_get_status.  Nothing traps or hangs.
+ */
+int hils_selftest_bounded_wait(int32_t limit_ms, hils_stream_t stream);
+
 /* Static English description of a status code. */
 const char* hils_strerror(int status);
 

@@ -69,6 +69,8 @@ def test_null_and_misaligned_pointers_rejected(lib):
     small = hils.hils_decode_workspace_bytes(d) - 1
     assert lib.hils_attn_decode(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, p, small, None) == 4
     assert lib.hils_get_status(None, None) == 1
+    assert lib.hils_selftest_bounded_wait(0, None) == 1
+    assert lib.hils_selftest_bounded_wait(5000, None) == 1
     # bf16 prefill needs its workspace
     need = hils.hils_prefill_workspace_bytes(d)
     assert need > 0

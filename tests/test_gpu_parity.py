@@ -164,7 +164,9 @@ def test_out_of_range_id_is_recorded_and_skipped():
     assert hils.hils_get_status() == 0
     others = torch.ones(w.N, dtype=torch.bool)
     others[300] = False
-    assert torch.equal(o2[0, 0, others], o[0, 0, others])
+    # the bf16 path accumulates partial outputs with atomics in no fixed order,
+    # so untouched rows agree to rounding, not bit for bit
+    assert torch.max(torch.abs(o2[0, 0, others].float() - o[0, 0, others].float())).item() <= 1e-2
     assert torch.all(torch.isfinite(o2.float()))
 
 
@@ -179,3 +181,21 @@ def test_status_word_reports_bad_seqlen_and_clears():
     assert hils.hils_get_status() == 0
     assert torch.all(o[1] == 0) and torch.all(ids[1] == -1)
     assert torch.all(torch.isfinite(o[0].float()))
+
+
+def test_bounded_wait_times_out_cleanly_and_context_survives():
+    """A device wait on a phase that never completes gives up after its limit,
+    records HILS_ERR_DEVICE_TIMEOUT and returns; later work still runs."""
+    import time
+    t0 = time.time()
+    hils.hils_selftest_bounded_wait(50)
+    assert hils.hils_get_status() == 5
+    assert time.time() - t0 < 10
+    assert hils.hils_get_status() == 0
+    w = custom("after-timeout", B=1, Hq=2, Hkv=1, d=64, N=512, K=3, seed=71, dtype="bf16")
+    inp = generate(w)
+    q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
+    o = hils.prefill(q, k, v, lq, w.K)
+    torch.cuda.synchronize()
+    assert hils.hils_get_status() == 0
+    assert torch.all(torch.isfinite(o.float()))
