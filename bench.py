@@ -331,6 +331,95 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_selected_bytes(ids, w):
+    """Distinct K/V bytes a decode step must read: per (b, kv head) the union of
+    the G heads' kept chunks plus the own chunk, 64 keys x d x 2 bytes x (K, V)."""
+    B, Hq, K = ids.shape
+    total = 0
+    for b in range(B):
+        for h in range(w.Hkv):
+            sel = ids[b, h * w.G:(h + 1) * w.G].reshape(-1)
+            n_union = len(np.unique(sel[sel >= 0])) + 1
+            total += n_union * w.C * w.d * 2 * 2
+    return total
+
+
+def run_decode(args, w, rank, world, local_rank):
+    """One decode step per step for every sequence of the batch; the landmark
+    summaries of the cache are built in the untimed setup.  L2 is flushed
+    between steps (the compressed keys fit in L2)."""
+    import torch
+    from chunk_wise_sparse_b200 import hils
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hils.lib()
+    inp = generate(w)
+
+    def to_dev(name):
+        bits = getattr(inp, name + "_bits")
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(getattr(inp, name + "_f32")).to(dev)
+
+    q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
+    B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
+    summ = hils.landmark_summary(k, lq, K)
+    dims = hils.make_dims(B, Hq, Hkv, d, N, K, q.dtype)
+    seq = torch.full((B,), N, dtype=torch.int32, device=dev)
+    ws = torch.empty((hils.hils_decode_workspace_bytes(dims),), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    ids = torch.empty((B, Hq, K), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hils.hils_attn_decode(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, o, ids, sc, ws,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hils.hils_get_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    times = []
+    launches0 = hils.hils_kernel_launches()
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    launches = hils.hils_kernel_launches() - launches0
+    status = hils.hils_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} during the timed steps")
+    us = 1e3 * max_over_ranks(float(np.median(times)), world, dev)
+    if rank != 0:
+        return
+    sel_bytes = decode_selected_bytes(ids.cpu().numpy(), w)
+    kp_bytes = B * Hkv * w.nc * (d + 16) * 2
+    peaks = load_peaks()
+    gbs = sel_bytes / (us / 1e6) / 1e9
+    all_gbs = (sel_bytes + kp_bytes) / (us / 1e6) / 1e9
+    line = {
+        "metric": "HiLS decode us/step (one new token per sequence: scoring, top-K, sparse attention)",
+        "value": us, "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": f"synthetic: i.i.d. N(0,1), seed {w.seed}",
+        "config": dict(workload_config(w, world), l2="256 MiB buffer written between steps (L2 flush)"),
+        "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "bytes": "selected-KV (union of kept chunks + own chunk per (b, kv head))",
+                     "selected_kv_bytes": sel_bytes, "all_bytes_gbs": all_gbs},
+        "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,8 +432,6 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
-    if w.kind == "decode":
-        raise SystemExit("bench.py times prefill workloads; decode-only workloads are covered by the tests")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -358,7 +445,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if w.kind == "decode":
+            run_decode(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

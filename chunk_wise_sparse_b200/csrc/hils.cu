@@ -234,12 +234,19 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   op.oacc = oacc;
   op.rowstat = rowstat;
   op.lse_own = lse;
-  op.counts = counts;
-  op.ranks = ranks;
   op.P = P.P;
   op.n_tiles = P.own_tiles;
   own_fn<<<dim3(unsigned(P.own_tiles), unsigned(d->batch * d->heads_kv)), 128, CO::SMEM, st>>>(tq_tile, tk_own,
                                                                                             tv_own, op);
+  // two-level count when a CTA's rows stay in one window and the chunk histogram fits
+  const size_t hist_bytes = sizeof(int32_t) * size_t(P.c.nc);
+  if (d->seqlen % kCountRows == 0 && (int64_t(1) << P.c.win_shift) % kCountRows == 0 && hist_bytes <= 96 * 1024) {
+    constexpr auto cfn = cc_count_kernel;
+    if (hist_bytes > 48 * 1024 && set_smem_max<cfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    cfn<<<unsigned(P.rows / kCountRows), kCountThreads, hist_bytes, st>>>(ids, counts, ranks, P.c);
+  } else {
+    cc_count_direct_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, counts, ranks, P.c, P.n_slots);
+  }
   const unsigned nsb = unsigned(P.n_scan_blocks);
   cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
   cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
@@ -258,7 +265,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   fn<<<unsigned(sm_count() * C::MAX_CTAS), C::THREADS, C::SMEM, st>>>(tq_row, tk, tv, prm);
   const int64_t n8 = P.rows * D / 8;
   cc_final_kernel<D><<<unsigned((n8 + 255) / 256), 256, 0, st>>>(oacc, static_cast<__nv_bfloat16*>(o), n8);
-  return launched(8);
+  return launched(9);
 }
 
 template <typename T, int D>

@@ -80,10 +80,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // heads of one kv head.  The tile's keys are the NK = max(64, P) keys of the
 // chunks that hold those positions; S = Q K^T and O = P V run on tcgen05 and
 // one thread per row applies the causal own-chunk mask.  Per row it also forms
-// the fusion normaliser M' = log(sum_kept exp(s^) + exp(lse_own)), writes the
-// own chunk's weighted output exp(lse_own - M') softmax(s) V (= exp(s - M') V)
-// to the fp32 accumulator, and counts each kept (row, slot) pair under its key,
-// keeping the pair's rank within the key for the fill pass.
+// the fusion normaliser M' = log(sum_kept exp(s^) + exp(lse_own)) and writes
+// the own chunk's weighted output exp(lse_own - M') softmax(s) V
+// (= exp(s - M') V) to the fp32 accumulator.
 template <int D>
 struct CcOwn {
   static constexpr int M = 128;
@@ -107,8 +106,6 @@ struct CcOwnParams {
   float* oacc;
   float* rowstat;
   float* lse_own;
-  int32_t* counts;
-  int32_t* ranks;
   int P;            // positions per tile
   int n_tiles;      // tiles per kv head
 };
@@ -240,32 +237,14 @@ cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
   const float lse = m * c.tau + logf(l);   // log sum_j exp(tau s_j)
-  // fusion normaliser and pair counts
+  // fusion normaliser over the valid kept chunks and the own chunk
   float Mp = lse;
   if (live) {
     const float Mx = fmaxf(smax, lse);
     float Z = expf(lse - Mx);
-    const int64_t bhk = bh;
-    // eight slots at a time so that the counting atomics are in flight together
-    for (int t0 = 0; t0 < c.K; t0 += 8) {
-      int32_t rk[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = t0 + u;
-        rk[u] = -1;
-        if (t >= c.K) continue;
-        const int32_t ci = __ldg(p.ids + row * c.K + t);
-        if (ci < 0) continue;
-        if (ci >= own) {
-          record_error(HILS_ERR_DEVICE_BOUNDS);
-          continue;
-        }
-        Z += expf(__ldg(p.scores + row * c.K + t) - Mx);
-        rk[u] = atomicAdd(p.counts + cc_key(c, bhk, pos, ci), 1);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (rk[u] >= 0) p.ranks[row * c.K + t0 + u] = rk[u];
+    for (int t = 0; t < c.K; ++t) {
+      const int32_t ci = __ldg(p.ids + row * c.K + t);
+      if (ci >= 0 && ci < own) Z += expf(__ldg(p.scores + row * c.K + t) - Mx);
     }
     Mp = Mx + logf(Z);
     p.rowstat[row] = Mp;
@@ -334,6 +313,73 @@ cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------- pair counts
+// Each CTA takes kCountRows consecutive rows of one query head (inside one
+// window), counts their kept pairs per chunk in a shared-memory histogram,
+// then adds each touched chunk's count to the global per-key count with one
+// atomic, whose old value is the base of this CTA's pairs of that chunk.  A
+// pair's rank within its key is base + its rank in the histogram.  Ids outside
+// the row's candidates are recorded as HILS_ERR_DEVICE_BOUNDS and skipped.
+constexpr int kCountRows = 4096;
+constexpr int kCountThreads = 1024;
+
+__global__ void __launch_bounds__(kCountThreads)
+cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, int32_t* __restrict__ ranks,
+                const CcDims c) {
+  extern __shared__ int32_t hist[];   // [nc]
+  const int64_t row0 = int64_t(blockIdx.x) * kCountRows;   // rows of one (b, hq); kCountRows | n_tok
+  const int64_t bhq = row0 / c.n_tok, i0 = row0 % c.n_tok;
+  const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
+  const int64_t bh = b * c.Hkv + hq / c.G;
+  const int64_t key0 = cc_key(c, bh, i0, 0);
+  const int64_t nch = (i0 + kCountRows - 1) / kChunk;   // candidates of the last row
+  for (int64_t t = threadIdx.x; t < nch; t += blockDim.x) hist[t] = 0;
+  __syncthreads();
+  const int64_t n = int64_t(kCountRows) * c.K;
+  const int32_t* id0 = ids + row0 * c.K;
+  int32_t* rk0 = ranks + row0 * c.K;
+  for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
+    const int32_t ci = __ldg(id0 + t);
+    if (ci < 0) continue;
+    const int64_t i = i0 + t / c.K;
+    if (ci >= i / kChunk) {
+      record_error(HILS_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    rk0[t] = atomicAdd(hist + ci, 1);
+  }
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < nch; t += blockDim.x) {
+    const int32_t h = hist[t];
+    hist[t] = h > 0 ? atomicAdd(counts + key0 + t, h) : 0;
+  }
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
+    const int32_t ci = __ldg(id0 + t);
+    if (ci < 0 || ci >= (i0 + t / c.K) / kChunk) continue;
+    rk0[t] += hist[ci];
+  }
+}
+
+// Fallback for shapes the histogram does not fit: one global atomic per pair.
+__global__ void __launch_bounds__(256)
+cc_count_direct_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, int32_t* __restrict__ ranks,
+                       const CcDims c, int64_t n_slots) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n_slots) return;
+  const int32_t ci = __ldg(ids + idx);
+  if (ci < 0) return;
+  const int64_t row = idx / c.K;
+  const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
+  if (ci >= i / kChunk) {
+    record_error(HILS_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
+  const int64_t bh = b * c.Hkv + hq / c.G;
+  ranks[idx] = atomicAdd(counts + cc_key(c, bh, i, ci), 1);
 }
 
 // ---------------------------------------------------------------- scan (three passes)
@@ -491,9 +537,10 @@ cc_final_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ o, i
 // ---------------------------------------------------------------- chunk tiles on tcgen05
 // Warp-specialised, two-stage pipeline per CTA over its tiles (item = blockIdx.x
 // + j * gridDim.x):
-//   warp 0       producer: the tile's entries -> row ids (shared memory), then
-//                one lane issues TMA loads of the chunk's K and V and 32*d/64
-//                gather4 loads of the rows' queries (128B swizzle);
+//   warp 0       producer: the tile's entries (row ids, fusion factors) into
+//                shared memory (loaded one tile ahead), then one lane issues
+//                TMA loads of the chunk's K and V and 32*d/64 gather4 loads of
+//                the rows' queries (128B swizzle);
 //   warp 1       one lane issues S = Q K^T into TMEM buffer b, and once the
 //                softmax warps have written P, O = P V into TMEM buffer b;
 //   warps 2-5    one thread per row: the fusion factor s^ - M' (two loads),

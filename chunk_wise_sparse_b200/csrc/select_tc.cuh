@@ -83,6 +83,21 @@ struct SelTcParams {
   float* scores;
 };
 
+// sign bits (as words) of c - t*a0 and c - t*a1, one packed FMA
+__device__ __forceinline__ void fma2_signs(float a0, float a1, uint64_t nt2, uint64_t c2, uint32_t& s0, uint32_t& s1) {
+  asm("{\n\t.reg .b64 va, vd;\n\t"
+      "mov.b64 va, {%2, %3};\n\t"
+      "fma.rn.f32x2 vd, va, %4, %5;\n\t"
+      "mov.b64 {%0, %1}, vd;\n\t}"
+      : "=r"(s0), "=r"(s1)
+      : "f"(a0), "f"(a1), "l"(nt2), "l"(c2));
+}
+
+__device__ __forceinline__ uint64_t pack2(float x) {
+  const uint64_t u = __float_as_uint(x);
+  return (u << 32) | u;
+}
+
 template <int D, int KCAP>
 __global__ void __launch_bounds__(SelTc<D, KCAP>::THREADS, 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kb,
@@ -211,6 +226,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int64_t n_cand = valid ? pos / kChunk : 0;
     const int K = p.K;
     const float tau = p.tau;
+    const uint64_t ntau2 = pack2(-tau);
     float* my_stg = stg + r * C::STG_STRIDE;
     // Register list (KCAP > 0): sorted descending; slots [0, KCAP-K) hold +inf
     // so that the K-th best is always the last slot.  Shared-memory list
@@ -244,11 +260,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
           // four independent 8-bit chains keep the dependency depth short
           uint32_t part[4] = {0u, 0u, 0u, 0u};
+          const uint64_t thr2 = pack2(thr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 8; e += 2) {
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              part[q4] = __funnelshift_l(__float_as_uint(fmaf(-tau, v[8 * q4 + e], thr)), part[q4], 1);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t s0, s1;
+              fma2_signs(v[8 * q4 + e], v[8 * q4 + e + 1], ntau2, thr2, s0, s1);
+              part[q4] = __funnelshift_l(s0, part[q4], 1);
+              part[q4] = __funnelshift_l(s1, part[q4], 1);
+            }
           }
           bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
           if (lim < 32) bits &= ~(0xFFFFFFFFu >> int(lim));

@@ -90,6 +90,9 @@ SMALL = [
     custom("bf16-gqa3-cuda-core-select", B=1, Hq=6, Hkv=2, d=64, N=1600, K=7, seed=37, dtype="bf16", needles=2,
            needle_mode="random"),
     custom("bf16-gqa16-d128", B=1, Hq=16, Hkv=1, d=128, N=1024, K=12, seed=38, dtype="bf16"),
+    # N a multiple of 4096: pairs are counted through the shared-memory histogram
+    custom("bf16-gqa2-8k-hist-count", B=2, Hq=4, Hkv=2, d=64, N=8192, K=16, seed=39, dtype="bf16", needles=4,
+           needle_mode="random"),
 ]
 
 
