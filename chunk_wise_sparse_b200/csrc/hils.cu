@@ -179,8 +179,9 @@ CcPlan cc_plan(const hils_dims* d) {
   P.max_items = P.n_slots / kCcTileRows + P.c.n_keys + 1;
   P.off_items = take(sizeof(int4) * P.max_items);
   P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
-  P.off_erow = take(sizeof(int32_t) * P.n_slots);
-  P.off_efac = take(sizeof(float) * P.n_slots);
+  // entries are padded by one tile so that tile loads never run past the end
+  P.off_erow = take(sizeof(int32_t) * (P.n_slots + kCcTileRows));
+  P.off_efac = take(sizeof(float) * (P.n_slots + kCcTileRows));
   P.total = off;
   return P;
 }
@@ -225,6 +226,10 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
       !make_map_2d(&tv_own, v, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B))
     return HILS_ERR_CUDA;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess) return HILS_ERR_CUDA;
+  // the padding after the last entry must hold valid row ids (row 0)
+  if (cudaMemsetAsync(base + P.off_erow + sizeof(int32_t) * P.n_slots, 0, sizeof(int32_t) * kCcTileRows, st) !=
+      cudaSuccess)
+    return HILS_ERR_CUDA;
   constexpr auto own_fn = cc_own_tc_kernel<D>;
   if (set_smem_max<own_fn>() != cudaSuccess) return HILS_ERR_CUDA;
   CcOwnParams op;

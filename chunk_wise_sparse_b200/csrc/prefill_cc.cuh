@@ -642,64 +642,57 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Lane l owns rows 4l..4l+3 of every tile: it loads their row ids and
+    // fusion factors two tiles ahead and issues their gather4 itself, so the
+    // 32 gathers of a tile are issued in parallel.
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
     }
-    // metadata of tile j is loaded into registers while tile j-1 is issued
-    int4 rec = make_int4(0, 0, 1, 0);
-    int32_t nrow[C::M / 32];
-    float nfac[C::M / 32];
-    auto fetch = [&](int jj) {
+    int4 rec[2];
+    int32_t prow[2][4];
+    float pfac[2][4];
+    auto fetch = [&](int jj, int slot) {
       const int32_t item = int32_t(blockIdx.x) + jj * int32_t(gridDim.x);
-      rec = __ldg(p.items + item);
+      rec[slot] = __ldg(p.items + item);
 #pragma unroll
-      for (int q4 = 0; q4 < C::M / 32; ++q4) {
-        const int r = q4 * 32 + lane;
-        const int at = rec.x + (r < rec.z ? r : rec.z - 1);
-        nrow[q4] = __ldg(p.e_row + at);
-        nfac[q4] = __ldg(p.e_fac + at);
+      for (int t = 0; t < 4; ++t) {
+        const int at = rec[slot].x + 4 * lane + t;   // entries are padded past the last tile
+        prow[slot][t] = __ldg(p.e_row + at);
+        pfac[slot][t] = __ldg(p.e_fac + at);
       }
     };
-    if (n_my > 0) fetch(0);
+    if (n_my > 0) fetch(0, 0);
+    if (n_my > 1) fetch(1, 1);
     int j = 0;
     for (; j < n_my; ++j) {
-      const int s = j % C::NS, u = j / C::NS;
-      const int4 cur = rec;
-      int32_t crow[C::M / 32];
-      float cfac[C::M / 32];
+      const int s = j % C::NS, u = j / C::NS, cs = j & 1;
+      const int4 cur = rec[cs];
+      int32_t crow[4];
+      float cfac[4];
 #pragma unroll
-      for (int q4 = 0; q4 < C::M / 32; ++q4) { crow[q4] = nrow[q4]; cfac[q4] = nfac[q4]; }
-      if (j + 1 < n_my) fetch(j + 1);
+      for (int t = 0; t < 4; ++t) { crow[t] = prow[cs][t]; cfac[t] = pfac[cs][t]; }
+      if (j + 2 < n_my) fetch(j + 2, cs);
       if (!mbar_wait(&load_empty[s], (u & 1) ^ 1, abort_flag)) break;
       uint8_t* meta = smem + C::OFF_META + s * C::META;
-      int32_t* rows = reinterpret_cast<int32_t*>(meta);
-      float* facs = reinterpret_cast<float*>(meta + C::M * 4);
-#pragma unroll
-      for (int q4 = 0; q4 < C::M / 32; ++q4) {
-        rows[q4 * 32 + lane] = crow[q4];
-        facs[q4 * 32 + lane] = cfac[q4];
-      }
+      *reinterpret_cast<int4*>(meta + 16 * lane) = make_int4(crow[0], crow[1], crow[2], crow[3]);
+      *reinterpret_cast<float4*>(meta + C::M * 4 + 16 * lane) = make_float4(cfac[0], cfac[1], cfac[2], cfac[3]);
       if (lane == 0) reinterpret_cast<int32_t*>(meta + C::M * 8)[0] = cur.z;
-      __syncwarp();
+      uint8_t* st = smem + s * C::STAGE;
       if (lane == 0) {
-        uint8_t* st = smem + s * C::STAGE;
         mbar_arrive_expect_tx(&load_full[s], C::TX_BYTES);
 #pragma unroll
         for (int a = 0; a < C::KATOMS; ++a) {
           tma_load_2d(st + C::OFF_K + a * C::KV_ATOM, &tm_k, &load_full[s], a * 64, cur.y);
           tma_load_2d(st + C::OFF_V + a * C::KV_ATOM, &tm_v, &load_full[s], a * 64, cur.y);
         }
-        const uint32_t qdst = smem_u32(st + C::OFF_Q);
-#pragma unroll 4
-        for (int r = 0; r < C::M; r += 4) {
-#pragma unroll
-          for (int a = 0; a < C::KATOMS; ++a)
-            tma_gather4(qdst + a * C::Q_ATOM + r * 128, &tm_q, &load_full[s], a * 64, rows[r], rows[r + 1],
-                        rows[r + 2], rows[r + 3]);
-        }
       }
+      __syncwarp();
+      const uint32_t qdst = smem_u32(st + C::OFF_Q) + uint32_t(4 * lane) * 128;
+#pragma unroll
+      for (int a = 0; a < C::KATOMS; ++a)
+        tma_gather4(qdst + a * C::Q_ATOM, &tm_q, &load_full[s], a * 64, crow[0], crow[1], crow[2], crow[3]);
       __syncwarp();
     }
     if (lane == 0) *issued_slot = j;
