@@ -54,10 +54,20 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo) 
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+// global[dst .. dst+bytes) += shared[src .. src+bytes) as fp32, done by the
+// bulk-copy unit as whole-sector reductions in L2; per-thread bulk group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src_smem, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(src_smem), "r"(bytes)
                : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk groups except the newest n have finished reading shared memory
+template <int n>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Four rows y0..y3 of a tensor map whose box is one row of 64 elements.
 __device__ __forceinline__ void tma_gather4(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
@@ -558,8 +568,13 @@ struct CcTc {
   static constexpr uint32_t Q_BYTES = KATOMS * Q_ATOM;
   static constexpr uint32_t K_BYTES = KATOMS * KV_ATOM;
   static constexpr uint32_t P_BYTES = M * 128;      // 128 rows x 64 keys bf16
-  // P overwrites the stage's Q tile once S = Q K^T is done
-  static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES;
+  // P overwrites the stage's Q tile once S = Q K^T is done; once P V is done
+  // the whole stage holds the tile's fp32 output rows (4D bytes each, padded
+  // to a 4D + 16 byte stride so the row-per-thread stores of 8 consecutive
+  // rows hit distinct banks) until the bulk reductions have read them
+  static constexpr uint32_t O_ROW = D * 4;
+  static constexpr uint32_t O_STRIDE = O_ROW + 16;
+  static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES + 2048;
   static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES, OFF_P = 0;
   static constexpr uint32_t OFF_META = NS * STAGE;                // per stage: rows[128] i32, fac[128] f32, n
   static constexpr uint32_t META = M * 4 + M * 4 + 16;
@@ -577,6 +592,7 @@ struct CcTc {
   static constexpr uint32_t IDESC_O = sm100::idesc_bf16(M, D) | (1u << 16);
   static constexpr int THREADS = 192;
   static_assert(P_BYTES <= Q_BYTES, "P reuses the Q tile");
+  static_assert(M * O_STRIDE <= STAGE, "output rows fit the stage");
 };
 
 struct CcTcParams {
@@ -599,7 +615,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* load_full = bars;        // [NS] producer -> MMA, softmax
-  uint64_t* load_empty = bars + 3;   // [NS] MMA (after PV) -> producer
+  uint64_t* load_empty = bars + 3;   // [NS] epilogue (output rows read out) -> producer
   uint64_t* p_full = bars + 6;       // [NS] softmax -> MMA
   uint64_t* s_full = bars + 9;       // [2] MMA -> softmax
   uint64_t* o_full = bars + 11;      // [2] MMA -> epilogue
@@ -615,7 +631,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (tid == 0) {
     for (int t = 0; t < C::NS; ++t) {
       mbar_init(&load_full[t], 1);
-      mbar_init(&load_empty[t], 1);
+      mbar_init(&load_empty[t], 4);
       mbar_init(&p_full[t], 4);
     }
     for (int t = 0; t < 2; ++t) {
@@ -650,30 +666,44 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
     }
-    int4 rec[2];
-    int32_t prow[2][4];
-    float pfac[2][4];
-    auto fetch = [&](int jj, int slot) {
-      const int32_t item = int32_t(blockIdx.x) + jj * int32_t(gridDim.x);
-      rec[slot] = __ldg(p.items + item);
+    // Tile records are fetched three tiles ahead and their entries two tiles
+    // ahead, held in named registers that shift by one tile per iteration
+    // (an array indexed by the tile counter would live in local memory and
+    // make every load wait at once).
+    auto fetch_rec = [&](int jj) {
+      return __ldg(p.items + int32_t(blockIdx.x) + jj * int32_t(gridDim.x));
+    };
+    auto fetch_entries = [&](const int4& r, int32_t (&row)[4], float (&fac)[4]) {
+      const int base = r.x + 4 * lane;   // entries are padded past the last tile
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int at = rec[slot].x + 4 * lane + t;   // entries are padded past the last tile
-        prow[slot][t] = __ldg(p.e_row + at);
-        pfac[slot][t] = __ldg(p.e_fac + at);
+        row[t] = __ldg(p.e_row + base + t);
+        fac[t] = __ldg(p.e_fac + base + t);
       }
     };
-    if (n_my > 0) fetch(0, 0);
-    if (n_my > 1) fetch(1, 1);
+    int4 r0 = make_int4(0, 0, 0, 0), r1 = r0, r2 = r0;
+    int32_t row0[4] = {0, 0, 0, 0}, row1[4] = {0, 0, 0, 0};
+    float fac0[4] = {0.f, 0.f, 0.f, 0.f}, fac1[4] = {0.f, 0.f, 0.f, 0.f};
+    if (n_my > 0) { r0 = fetch_rec(0); fetch_entries(r0, row0, fac0); }
+    if (n_my > 1) { r1 = fetch_rec(1); fetch_entries(r1, row1, fac1); }
+    if (n_my > 2) r2 = fetch_rec(2);
     int j = 0;
     for (; j < n_my; ++j) {
-      const int s = j % C::NS, u = j / C::NS, cs = j & 1;
-      const int4 cur = rec[cs];
+      const int s = j % C::NS, u = j / C::NS;
+      const int4 cur = r0;
       int32_t crow[4];
       float cfac[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) { crow[t] = prow[cs][t]; cfac[t] = pfac[cs][t]; }
-      if (j + 2 < n_my) fetch(j + 2, cs);
+      for (int t = 0; t < 4; ++t) {
+        crow[t] = row0[t];
+        cfac[t] = fac0[t];
+        row0[t] = row1[t];
+        fac0[t] = fac1[t];
+      }
+      r0 = r1;
+      r1 = r2;
+      if (j + 3 < n_my) r2 = fetch_rec(j + 3);
+      if (j + 2 < n_my) fetch_entries(r1, row1, fac1);
       if (!mbar_wait(&load_empty[s], (u & 1) ^ 1, abort_flag)) break;
       uint8_t* meta = smem + C::OFF_META + s * C::META;
       *reinterpret_cast<int4*>(meta + 16 * lane) = make_int4(crow[0], crow[1], crow[2], crow[3]);
@@ -722,7 +752,6 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mma_bf16(t_o, desc_sw128(sp + kk * 32), desc_sw128_mn(sv + kk * 2048, C::KV_ATOM), C::IDESC_O,
                    kk > 0 ? 1u : 0u);
         mma_commit(&o_full[b]);
-        mma_commit(&load_empty[s]);
       }
       *consumed_slot = j;
       mma_commit(done);
@@ -786,20 +815,32 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (lane == 0) mbar_arrive(&p_full[s]);
       if (!mbar_wait(&o_full[b], ub & 1, abort_flag)) break;
       tc_fence_after();
+      // P V is done: the stage is free for this tile's output rows
+      const uint32_t orow = smem_u32(smem + s * C::STAGE) + uint32_t(r) * C::O_STRIDE;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         float o[32];
         tmem_ld32(tmem + t_lane + uint32_t(2 * kChunk + b * D + cc * 32), o);
-        if (live) {
-          float* dst = p.oacc + grow * D + cc * 32;
 #pragma unroll
-          for (int t = 0; t < 32; t += 4) red_add_v4(dst + t, o[t], o[t + 1], o[t + 2], o[t + 3]);
-        }
+        for (int t = 0; t < 32; t += 4)
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(orow + uint32_t(cc * 32 + t) * 4), "f"(o[t]),
+                       "f"(o[t + 1]), "f"(o[t + 2]), "f"(o[t + 3])
+                       : "memory");
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[b]);
+      fence_proxy_async_smem();
+      if (live) bulk_reduce_add_f32(p.oacc + grow * D, orow, C::O_ROW);
+      bulk_commit();
+      // the previous tile's rows have been read: hand its stage back
+      if (j > 0) {
+        bulk_wait_read<1>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&load_empty[(j - 1) % C::NS]);
+      }
     }
+    bulk_wait_all();
   }
   // ------------------------------------------------------------ teardown
   __syncthreads();
