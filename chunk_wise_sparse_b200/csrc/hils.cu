@@ -105,10 +105,15 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
       !make_map_2d(&tkb, kmma, D + kExt, rows_k, (D + kExt) * 2, 64, C::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tke, kmma, D + kExt, rows_k, (D + kExt) * 2, kExt, C::NT, CU_TENSOR_MAP_SWIZZLE_32B))
     return HILS_ERR_CUDA;
-  // d=64 fits two CTAs per SM with 3 stages; d=128 runs one CTA with up to 4.
-  int stages = D == 64 ? 3 : 4;
-  while (stages > 2 && C::layout(d->topk, stages).total > uint32_t(kMaxSmem)) --stages;
-  const uint32_t smem = C::layout(d->topk, stages).total;
+  // d=64 with K <= 16 keeps two CTAs per SM; the rest run one CTA per SM.
+  // Two k' stages; the top-K log takes what shared memory is left (it is
+  // compacted less often the longer it is), at most 128 entries.
+  const uint32_t per_cta = D == 64 && KCAP == 16 ? 115712u : uint32_t(kMaxSmem);
+  const int stages = 2;
+  int cap = KCAP > 0 ? C::MIN_CAP : 0;
+  if (KCAP > 0)
+    while (cap + 8 <= 128 && C::layout(d->topk, stages, cap + 8).total <= per_cta) cap += 8;
+  const uint32_t smem = C::layout(d->topk, stages, cap).total;
   if (smem > uint32_t(kMaxSmem)) return HILS_ERR_UNSUPPORTED;
   constexpr auto fn = select_tc_kernel<D, KCAP>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
@@ -122,6 +127,7 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
   p.P = P;
   p.n_row_tiles = int((N + P - 1) / P);
   p.stages = stages;
+  p.cap = cap;
   p.tau = 1.f / sqrtf(float(D));
   p.ids = ids;
   p.scores = scores;

@@ -22,10 +22,13 @@
 //   warps 2-5          epilogue, one thread per row (= TMEM lane): 32 scores
 //                      per tcgen05.ld; each is tested against the row's
 //                      current K-th best with one FFMA and its sign bit is
-//                      funnel-shifted into a 32-bit mask; only rows with set
-//                      bits stage their scores and insert them into a sorted
-//                      top-K list in shared memory.  Ties keep the lower
-//                      chunk id (chunks are visited in ascending order).
+//                      funnel-shifted into a 32-bit mask.  Passing scores go,
+//                      one per lane and round with all lanes in step, into a
+//                      values-only sorted list in registers (two min/max per
+//                      slot, no branches) and, with their chunk ids, into a
+//                      per-row log in shared memory; the result's ids are
+//                      read back from the log.  Ties keep the lower chunk id
+//                      (chunks are visited in ascending order).
 // Every wait is bounded in time; a time-out records HILS_ERR_DEVICE_TIMEOUT,
 // drains in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -46,7 +49,11 @@ struct SelTc {
   static constexpr uint32_t B_EXT = NT * 32;
   static constexpr uint32_t B_STAGE = B_MAIN + B_EXT;
   static constexpr int STG_STRIDE = 36;   // floats per thread in the staging area (conflict-free float4)
-  // KCAP > 0: the per-row top-K lives in registers (K <= KCAP); 0: in shared memory.
+  // KCAP > 0: the per-row top-K values live in registers (K <= KCAP) and the
+  // (score, chunk) pairs that entered them in a per-row shared-memory log of
+  // `cap` entries (K + 16 at least, host-chosen); KCAP == 0: a sorted
+  // (score, chunk) list of K entries in shared memory.
+  static constexpr int MIN_CAP = KCAP + 16;
   static constexpr uint32_t STG_BYTES = M * STG_STRIDE * 4;
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 2 * NT;
@@ -57,14 +64,14 @@ struct SelTc {
     int stages;
   };
   // Shared-memory layout (offsets from a 1024-byte aligned base).
-  __host__ __device__ static Layout layout(int K, int stages) {
+  __host__ __device__ static Layout layout(int K, int stages, int cap) {
     Layout L;
     L.stages = stages;
     L.a = 0;
     L.aext = A_BYTES;
     L.b = (L.aext + AEXT_BYTES + 1023u) & ~1023u;
     L.stg = L.b + uint32_t(stages) * B_STAGE;
-    const uint32_t list_bytes = KCAP > 0 ? 0u : uint32_t(K) * M * 4;
+    const uint32_t list_bytes = uint32_t(KCAP > 0 ? cap : K) * M * 4;
     L.topv = L.stg + STG_BYTES;
     L.topi = L.topv + list_bytes;
     L.bars = L.topi + list_bytes;
@@ -77,7 +84,7 @@ struct SelTc {
 struct SelTcParams {
   int64_t n_tok, nc;
   int Hq, Hkv, G, K, P;  // P = 128 / G positions per tile
-  int n_row_tiles, stages;
+  int n_row_tiles, stages, cap;
   float tau;
   int32_t* ids;
   float* scores;
@@ -107,7 +114,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
-  const typename C::Layout L = C::layout(p.K, p.stages);
+  const typename C::Layout L = C::layout(p.K, p.stages, p.cap);
   uint8_t* sA = smem + L.a;
   uint8_t* sAext = smem + L.aext;
   uint8_t* sB = smem + L.b;
@@ -134,6 +141,19 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int64_t pos_end = (pos0 + p.P < p.n_tok) ? pos0 + p.P : p.n_tok;
   const int64_t c_hi = (pos_end - 1) / kChunk;          // candidates of the tile's last row
   const int n_tiles = int((c_hi + C::NT - 1) / C::NT);
+  // K <= KCAP: when every row of the tile has at least 8 K candidates, a
+  // first pass over the chunks splits each row's scores into disjoint groups
+  // of g and finds the K-th largest group maximum: K distinct scores reach
+  // it, so it is a lower bound of the row's K-th best score, and the second
+  // pass keeps only the scores that reach it.  The MMAs of both passes are
+  // the same.  g: 128 from 128 K candidates on, else 32, 16 or 8 (the
+  // largest that leaves K groups); smaller groups bound tighter but cost a
+  // list insertion each, and on long rows a group of 128 is the cheaper.
+  const int64_t n_min = pos0 / kChunk;   // candidates of the tile's first row
+  const int64_t kk = p.K;
+  const int group = n_min >= 128 * kk ? 128 : n_min >= 32 * kk ? 32 : n_min >= 16 * kk ? 16 : n_min >= 8 * kk ? 8 : 0;
+  const int n_pass = (KCAP > 0 && group > 0) ? 2 : 1;
+  const int n_steps = n_pass * n_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.stages; ++s) {
@@ -181,12 +201,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int a = 0; a < C::KATOMS; ++a) tma_load_2d(sA + a * C::A_ATOM + g * p.P * 128, &tm_q, qfull, a * 64, y);
     }
     int j = 0;
-    for (; j < n_tiles; ++j) {
+    for (; j < n_steps; ++j) {
       const int s = j % L.stages, u = j / L.stages;
       if (!mbar_wait(&empty[s], (u & 1) ^ 1, abort_flag)) break;
       mbar_arrive_expect_tx(&full[s], C::B_STAGE);
       uint8_t* bs = sB + s * C::B_STAGE;
-      const int y = int(int64_t(bh) * p.nc + int64_t(j) * C::NT);
+      const int y = int(int64_t(bh) * p.nc + int64_t(j % n_tiles) * C::NT);
       for (int a = 0; a < C::KATOMS; ++a) tma_load_2d(bs + a * C::B_ATOM, &tm_kb, &full[s], a * 64, y);
       tma_load_2d(bs + C::B_MAIN, &tm_ke, &full[s], D, y);
     }
@@ -196,7 +216,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     int j = 0;
     if (mbar_wait(qfull, 0, abort_flag)) {
       const uint32_t a0 = smem_u32(sA), ae = smem_u32(sAext);
-      for (; j < n_tiles; ++j) {
+      for (; j < n_steps; ++j) {
         const int s = j % L.stages, u = j / L.stages, buf = j & 1, ub = j >> 1;
         if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
         if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, abort_flag)) break;
@@ -228,89 +248,209 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float tau = p.tau;
     const uint64_t ntau2 = pack2(-tau);
     float* my_stg = stg + r * C::STG_STRIDE;
-    // Register list (KCAP > 0): sorted descending; slots [0, KCAP-K) hold +inf
-    // so that the K-th best is always the last slot.  Shared-memory list
-    // (KCAP == 0): sorted descending, K slots, `count` filled.
-    constexpr int KR = KCAP > 0 ? KCAP : 1;
-    float rv[KR];
-    int32_t ri[KR];
-#pragma unroll
-    for (int t = 0; t < KR; ++t) {
-      const bool pad = t < KR - K;
-      rv[t] = pad ? INFINITY : -INFINITY;
-      ri[t] = pad ? -2 : -1;
-    }
     float* tv = topv + r;
     int32_t* ti = topi + r;
+    // KCAP > 0: tv/ti is the row's candidate buffer, (score, chunk) pairs in
+    // ascending chunk order; KCAP == 0: its sorted top-K list.  `count` entries.
     int count = 0;
+    // a score passes when tau * acc > thr, exactly (the sign of one FMA)
     float thr = -INFINITY;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int buf = j & 1, ub = j >> 1;
+    // KCAP > 0: values-only list sorted descending; slots [0, KCAP-K) hold
+    // +inf so that the K-th value is always the last slot.  It ranks the group
+    // maxima of the first pass and the candidate buffer.
+    constexpr int KR = KCAP > 0 ? KCAP : 1;
+    float rv[KR];
+    auto rv_reset = [&]() {
+#pragma unroll
+      for (int t = 0; t < KR; ++t) rv[t] = t < KR - K ? INFINITY : -INFINITY;
+    };
+    rv_reset();
+    // sorted insertion without branches: slot t takes max(old t, min(old t-1, x));
+    // x = -inf leaves the list unchanged
+    auto rv_insert = [&](float x) {
+#pragma unroll
+      for (int t = KR - 1; t >= 1; --t) rv[t] = fmaxf(rv[t], fminf(rv[t - 1], x));
+      rv[0] = fmaxf(rv[0], x);
+    };
+    // rv <- the best K scores of the buffer, all lanes in step
+    auto rank_buffer = [&]() {
+      rv_reset();
+      const int m = __reduce_max_sync(0xffffffffu, count);
+      for (int i = 0; i < m; ++i) rv_insert(i < count ? tv[i * C::M] : -INFINITY);
+    };
+    // Walk the buffer in chunk order and keep what its best K are: every
+    // score above their K-th value w, then the first scores equal to w.
+    // Compaction (emit false): the kept entries move to the front of the
+    // buffer and later scores must beat w.  Emission: they are written to
+    // out_i/out_s (if not null) in chunk order and padded with -1.  All lanes
+    // call it together.
+    auto keep_best = [&](bool emit, int32_t* out_i, float* out_s) {
+      rank_buffer();
+      const float w = rv[KR - 1];
+      int quota = K;
+#pragma unroll
+      for (int t = 0; t < KR; ++t) quota -= (t >= KR - K) & (rv[t] > w);
+      int n = 0;
+      for (int i = 0; i < count; ++i) {
+        const float val = tv[i * C::M];
+        const bool eq = val == w;
+        const bool keep = val > w || (eq && quota > 0);
+        quota -= eq && keep;
+        if (keep) {
+          const int32_t id = ti[i * C::M];
+          if (emit) {
+            if (out_i) out_i[n] = id;
+            if (out_s) out_s[n] = val;
+          } else {
+            tv[n * C::M] = val;
+            ti[n * C::M] = id;
+          }
+          ++n;
+        }
+      }
+      if (emit) {
+        for (int t = n; t < K && out_i; ++t) {
+          out_i[t] = -1;
+          if (out_s) out_s[t] = -INFINITY;
+        }
+      } else {
+        count = n;
+        thr = fmaxf(thr, w);
+      }
+    };
+    float tmax = -INFINITY;
+    for (int jg = 0; jg < n_steps; ++jg) {
+      const int buf = jg & 1, ub = jg >> 1;
+      const int j = jg % n_tiles;
       if (!mbar_wait(&tfull[buf], ub & 1, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(buf * C::NT);
+      const int64_t c0 = int64_t(j) * C::NT;
+      // candidates of this row left in the tile (clamped to 0..128)
+      const int64_t left64 = n_cand - c0;
+      const int left = left64 <= 0 ? 0 : (left64 >= C::NT ? C::NT : int(left64));
+      if (KCAP > 0 && n_pass == 2 && jg < n_tiles) {
+        // ---- first pass: the row's group maxima, ranked in rv
 #pragma unroll 1
-      for (int gi = 0; gi < C::NT / 32; ++gi) {
-        float v[32];
-        tmem_ld32(tb + gi * 32, v);
-        const int64_t cbase = int64_t(j) * C::NT + gi * 32;
-        const int64_t lim = n_cand - cbase;
-        uint32_t bits = 0;
-        if (lim > 0) {
-          // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
-          // four independent 8-bit chains keep the dependency depth short
-          uint32_t part[4] = {0u, 0u, 0u, 0u};
-          const uint64_t thr2 = pack2(thr);
+        for (int gi = 0; gi < C::NT / 32; ++gi) {
+          float v[32];
+          tmem_ld32(tb + gi * 32, v);
+          const int lim = left - gi * 32;
+          if (__any_sync(0xffffffffu, lim < 32)) {
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint32_t s0, s1;
-              fma2_signs(v[8 * q4 + e], v[8 * q4 + e + 1], ntau2, thr2, s0, s1);
-              part[q4] = __funnelshift_l(s0, part[q4], 1);
-              part[q4] = __funnelshift_l(s1, part[q4], 1);
-            }
+            for (int e = 0; e < 32; ++e) v[e] = e < lim ? v[e] : -INFINITY;
           }
-          bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
-          if (lim < 32) bits &= ~(0xFFFFFFFFu >> int(lim));
+          // max tree: after the step of width w, v[t] (t < w) is the maximum
+          // of the scores e = t (mod w) -- disjoint groups of 32 / w.
+          // tau > 0 and rounding is monotone: tau * max = max of the scores.
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = fmaxf(v[e], v[e + 16]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = fmaxf(v[e], v[e + 8]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = fmaxf(v[e], v[e + 4]);
+          if (group == 8) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rv_insert(tau * v[e]);
+            continue;
+          }
+          v[0] = fmaxf(v[0], v[2]);
+          v[1] = fmaxf(v[1], v[3]);
+          if (group == 16) {
+            rv_insert(tau * v[0]);
+            rv_insert(tau * v[1]);
+            continue;
+          }
+          v[0] = fmaxf(v[0], v[1]);
+          if (group == 32) {
+            rv_insert(tau * v[0]);
+            continue;
+          }
+          tmax = fmaxf(tmax, v[0]);
         }
-        if (__any_sync(0xffffffffu, bits != 0)) {
-          if (bits) {
+        if (group == C::NT) {
+          rv_insert(tau * tmax);
+          tmax = -INFINITY;
+        }
+      } else {
+        // ---- scan: test every score against thr, keep the passing ones
+#pragma unroll 1
+        for (int gi = 0; gi < C::NT / 32; ++gi) {
+          float v[32];
+          tmem_ld32(tb + gi * 32, v);
+          const int64_t cbase = c0 + gi * 32;
+          const int lim = left - gi * 32;
+          uint32_t bits = 0;
+          if (lim > 0) {
+            // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
+            // four independent 8-bit chains keep the dependency depth short
+            uint32_t part[4] = {0u, 0u, 0u, 0u};
+            const uint64_t thr2 = pack2(thr);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            for (int e = 0; e < 8; e += 2) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t s0, s1;
+                fma2_signs(v[8 * q4 + e], v[8 * q4 + e + 1], ntau2, thr2, s0, s1);
+                part[q4] = __funnelshift_l(s0, part[q4], 1);
+                part[q4] = __funnelshift_l(s1, part[q4], 1);
+              }
+            }
+            bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
+            if (lim < 32) bits &= ~(0xFFFFFFFFu >> lim);
           }
-          while (bits) {
-            const int e = __clz(bits);
-            bits &= ~(0x80000000u >> e);
-            const float sc = tau * my_stg[e];
-            const int32_t cid = int32_t(cbase + e);
-            if constexpr (KCAP > 0) {
-              if (!(sc > rv[KR - 1])) continue;
-              // insert keeping descending order; equal scores stay ahead (lower ids)
-              bool ge[KR];
+          if constexpr (KCAP > 0) {
+            // append the passing scores, one per lane and round; the score is
+            // picked out of the registers by a 5-level select on its column.
+            // All lanes compact their buffers together once one is full.
+            while (true) {
+              const uint32_t flags = (bits != 0u ? 1u : 0u) | (count == p.cap ? 2u : 0u);
+              const uint32_t any = __reduce_or_sync(0xffffffffu, flags);
+              if (!(any & 1u)) break;
+              if (any & 2u) keep_best(false, nullptr, nullptr);
+              const bool has = bits != 0u;
+              const int e = __clz(bits) & 31;
+              bits &= ~(0x80000000u >> e);
+              float w16[16], w8[8], w4[4], w2[2];
 #pragma unroll
-              for (int t = 0; t < KR; ++t) ge[t] = rv[t] >= sc;
+              for (int t = 0; t < 16; ++t) w16[t] = (e & 16) ? v[t + 16] : v[t];
 #pragma unroll
-              for (int t = KR - 1; t >= 1; --t) {
-                rv[t] = ge[t] ? rv[t] : (ge[t - 1] ? sc : rv[t - 1]);
-                ri[t] = ge[t] ? ri[t] : (ge[t - 1] ? cid : ri[t - 1]);
+              for (int t = 0; t < 8; ++t) w8[t] = (e & 8) ? w16[t + 8] : w16[t];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) w4[t] = (e & 4) ? w8[t + 4] : w8[t];
+#pragma unroll
+              for (int t = 0; t < 2; ++t) w2[t] = (e & 2) ? w4[t + 2] : w4[t];
+              const float x = tau * ((e & 1) ? w2[1] : w2[0]);
+              if (has) {
+                tv[count * C::M] = x;
+                ti[count * C::M] = int32_t(cbase + e);
+                ++count;
               }
-              rv[0] = ge[0] ? rv[0] : sc;
-              ri[0] = ge[0] ? ri[0] : cid;
-              thr = rv[KR - 1];
-            } else {
-              if (count == K && !(sc > thr)) continue;
-              int q = count < K ? count : K - 1;
-              while (q > 0 && tv[(q - 1) * C::M] < sc) {
-                tv[q * C::M] = tv[(q - 1) * C::M];
-                ti[q * C::M] = ti[(q - 1) * C::M];
-                --q;
+            }
+          } else if (__any_sync(0xffffffffu, bits != 0)) {
+            if (bits) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            }
+            {
+              while (bits) {
+                const int e = __clz(bits);
+                bits &= ~(0x80000000u >> e);
+                const float sc = tau * my_stg[e];
+                const int32_t cid = int32_t(cbase + e);
+                if (count == K && !(sc > thr)) continue;
+                int q = count < K ? count : K - 1;
+                while (q > 0 && tv[(q - 1) * C::M] < sc) {
+                  tv[q * C::M] = tv[(q - 1) * C::M];
+                  ti[q * C::M] = ti[(q - 1) * C::M];
+                  --q;
+                }
+                tv[q * C::M] = sc;
+                ti[q * C::M] = cid;
+                if (count < K) ++count;
+                if (count == K) thr = tv[(K - 1) * C::M];
               }
-              tv[q * C::M] = sc;
-              ti[q * C::M] = cid;
-              if (count < K) ++count;
-              if (count == K) thr = tv[(K - 1) * C::M];
             }
           }
         }
@@ -318,46 +458,33 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (KCAP > 0 && n_pass == 2 && jg == n_tiles - 1) {
+        // every score >= the K-th group maximum T passes: thr = the float below T
+        const float t_lb = rv[KR - 1];
+        thr = t_lb > -INFINITY ? nextafterf(t_lb, -INFINITY) : -INFINITY;
+      }
     }
-    if (valid) {
-      const int64_t row = (int64_t(b) * p.Hq + int64_t(h) * p.G + g) * p.n_tok + pos;
-      int32_t* out_i = p.ids + row * K;
-      float* out_s = p.scores ? p.scores + row * K : nullptr;
-      if constexpr (KCAP > 0) {
-        // ascending chunk id: each kept entry goes to its rank among the kept ids
-        int n_kept = 0;
-#pragma unroll
-        for (int t = 0; t < KR; ++t) n_kept += ri[t] >= 0;
-#pragma unroll
-        for (int t = 0; t < KR; ++t) {
-          if (ri[t] < 0) continue;
-          int rank = 0;
-#pragma unroll
-          for (int u = 0; u < KR; ++u) rank += (ri[u] >= 0) & (ri[u] < ri[t]);
-          out_i[rank] = ri[t];
-          if (out_s) out_s[rank] = rv[t];
+    const int64_t row = (int64_t(b) * p.Hq + int64_t(h) * p.G + g) * p.n_tok + pos;
+    int32_t* out_i = valid ? p.ids + row * K : nullptr;
+    float* out_s = valid && p.scores ? p.scores + row * K : nullptr;
+    if constexpr (KCAP > 0) {
+      keep_best(true, out_i, out_s);
+    } else if (valid) {
+      for (int a = 1; a < count; ++a) {
+        const int32_t ci = ti[a * C::M];
+        const float cv = tv[a * C::M];
+        int q = a;
+        while (q > 0 && ti[(q - 1) * C::M] > ci) {
+          ti[q * C::M] = ti[(q - 1) * C::M];
+          tv[q * C::M] = tv[(q - 1) * C::M];
+          --q;
         }
-        for (int t = n_kept; t < K; ++t) {
-          out_i[t] = -1;
-          if (out_s) out_s[t] = -INFINITY;
-        }
-      } else {
-        for (int a = 1; a < count; ++a) {
-          const int32_t ci = ti[a * C::M];
-          const float cv = tv[a * C::M];
-          int q = a;
-          while (q > 0 && ti[(q - 1) * C::M] > ci) {
-            ti[q * C::M] = ti[(q - 1) * C::M];
-            tv[q * C::M] = tv[(q - 1) * C::M];
-            --q;
-          }
-          ti[q * C::M] = ci;
-          tv[q * C::M] = cv;
-        }
-        for (int t = 0; t < K; ++t) {
-          out_i[t] = t < count ? ti[t * C::M] : -1;
-          if (out_s) out_s[t] = t < count ? tv[t * C::M] : -INFINITY;
-        }
+        ti[q * C::M] = ci;
+        tv[q * C::M] = cv;
+      }
+      for (int t = 0; t < K; ++t) {
+        out_i[t] = t < count ? ti[t * C::M] : -1;
+        if (out_s) out_s[t] = t < count ? tv[t * C::M] : -INFINITY;
       }
     }
   }
