@@ -16,6 +16,8 @@ same workload.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import subprocess
@@ -41,6 +43,31 @@ def load_peaks():
         return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
                     bf16_tflops_sustained=j.get("bf16_tflops_sustained", j["bf16_tflops"]), source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernels_sha256():
+    """Hash of the CUDA sources, to tell whether recorded counters still apply."""
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "chunk_wise_sparse_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(src, "*.cu")) + glob.glob(os.path.join(src, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, rows):
+    """DRAM bytes per launch of `kernel` from the committed ncu record (per
+    query row, scaled to `rows`), or None when there is none or the kernel
+    sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("kernels_sha256") != kernels_sha256() or kernel not in j.get("per_row_bytes", {}):
+        return None
+    return float(j["per_row_bytes"][kernel]) * rows
 
 
 def useful_work(w):
@@ -300,7 +327,8 @@ def run_ours(args, w, rank, world, local_rank):
         fl = work["flops_score"] if dom == "select" else work["flops_attn"]
         ach = fl / (kernels_ms[dom] / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "traffic": recorded_traffic(dom, B * w.Hq * N),
                 "peak_source": peaks["source"] + " bf16 dense burst"}
     else:
         by = work["bytes_summary"]

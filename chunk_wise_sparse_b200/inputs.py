@@ -73,7 +73,7 @@ class Workload:
         return self.N // self.C
 
 
-# The five workloads, named for what they are.
+# The workloads, named for what they are.
 WORKLOADS = {
     "tiny-fp32-1k": Workload("tiny-fp32-1k", 1, 1, 1, 64, 1024, 64, 3, 0,
                              "fp32", 3, "per_block", "prefill", 0),
@@ -85,6 +85,11 @@ WORKLOADS = {
                                        "bf16", 64, "random", "prefill", 4096),
     "prefill-512k-h16-d64": Workload("prefill-512k-h16-d64", 1, 16, 16, 64, 524288, 64, 16, 4,
                                      "bf16", 128, "random", "prefill+decode", 4096),
+    # the 512K workload's row lengths and kernels with two heads (about 0.3 GB
+    # on the device): the case that profiler captures of the long-context
+    # kernels run on
+    "prefill-256k-h2-d64": Workload("prefill-256k-h2-d64", 1, 2, 2, 64, 262144, 64, 16, 5,
+                                    "bf16", 16, "random", "prefill+decode", 4096),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
