@@ -105,9 +105,10 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
       !make_map_2d(&tkb, kmma, D + kExt, rows_k, (D + kExt) * 2, 64, C::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tke, kmma, D + kExt, rows_k, (D + kExt) * 2, kExt, C::NT, CU_TENSOR_MAP_SWIZZLE_32B))
     return HILS_ERR_CUDA;
-  // d=64 with K <= 16 keeps two CTAs per SM; the rest run one CTA per SM.
-  // Two k' stages; the top-K log takes what shared memory is left (it is
-  // compacted less often the longer it is), at most 128 entries.
+  // d = 64 with K <= 16 keeps two CTAs per SM (228 KB per SM, 1 KB of it
+  // reserved per CTA); the rest run one CTA per SM.  Two k' stages; the
+  // candidate buffer takes what shared memory is left (it is compacted less
+  // often the longer it is), at most 128 entries.
   const uint32_t per_cta = D == 64 && KCAP == 16 ? 115712u : uint32_t(kMaxSmem);
   const int stages = 2;
   int cap = KCAP > 0 ? C::MIN_CAP : 0;

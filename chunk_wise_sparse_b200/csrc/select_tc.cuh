@@ -54,9 +54,15 @@ struct SelTc {
   // `cap` entries (K + 16 at least, host-chosen); KCAP == 0: a sorted
   // (score, chunk) list of K entries in shared memory.
   static constexpr int MIN_CAP = KCAP + 16;
-  static constexpr uint32_t STG_BYTES = M * STG_STRIDE * 4;
+  // the staging area serves the shared-memory list path (K > 32) only
+  static constexpr uint32_t STG_BYTES = KCAP > 0 ? 0u : uint32_t(M) * STG_STRIDE * 4;
   static constexpr int THREADS = 192;
-  static constexpr uint32_t TMEM_COLS = 2 * NT;
+  // two CTAs per SM, two TMEM accumulators each (the MMA of tile j+1 runs
+  // during the epilogue of tile j; three CTAs with one accumulator each
+  // measured slower)
+  static constexpr int CTAS_PER_SM = 2;
+  static constexpr int BUFS = 2;
+  static constexpr uint32_t TMEM_COLS = BUFS * NT;
   static constexpr uint32_t IDESC = sm100::idesc_bf16(M, NT);
 
   struct Layout {
@@ -106,7 +112,7 @@ __device__ __forceinline__ uint64_t pack2(float x) {
 }
 
 template <int D, int KCAP>
-__global__ void __launch_bounds__(SelTc<D, KCAP>::THREADS, 2)
+__global__ void __launch_bounds__(SelTc<D, KCAP>::THREADS, SelTc<D, KCAP>::CTAS_PER_SM)
 select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kb,
                  const __grid_constant__ CUtensorMap tm_ke, const SelTcParams p) {
   using C = SelTc<D, KCAP>;
@@ -217,7 +223,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (mbar_wait(qfull, 0, abort_flag)) {
       const uint32_t a0 = smem_u32(sA), ae = smem_u32(sAext);
       for (; j < n_steps; ++j) {
-        const int s = j % L.stages, u = j / L.stages, buf = j & 1, ub = j >> 1;
+        const int s = j % L.stages, u = j / L.stages, buf = j % C::BUFS, ub = j / C::BUFS;
         if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
         if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
@@ -320,7 +326,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     };
     float tmax = -INFINITY;
     for (int jg = 0; jg < n_steps; ++jg) {
-      const int buf = jg & 1, ub = jg >> 1;
+      const int buf = jg % C::BUFS, ub = jg / C::BUFS;
       const int j = jg % n_tiles;
       if (!mbar_wait(&tfull[buf], ub & 1, abort_flag)) break;
       tc_fence_after();
