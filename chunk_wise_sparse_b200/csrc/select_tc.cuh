@@ -51,9 +51,9 @@ struct SelTc {
   static constexpr int STG_STRIDE = 36;   // floats per thread in the staging area (conflict-free float4)
   // KCAP > 0: the per-row top-K values live in registers (K <= KCAP) and the
   // (score, chunk) pairs that entered them in a per-row shared-memory log of
-  // `cap` entries (K + 16 at least, host-chosen); KCAP == 0: a sorted
+  // `cap` entries (K + 32 at least, host-chosen); KCAP == 0: a sorted
   // (score, chunk) list of K entries in shared memory.
-  static constexpr int MIN_CAP = KCAP + 16;
+  static constexpr int MIN_CAP = KCAP + 32;
   // the staging area serves the shared-memory list path (K > 32) only
   static constexpr uint32_t STG_BYTES = KCAP > 0 ? 0u : uint32_t(M) * STG_STRIDE * 4;
   static constexpr int THREADS = 192;
@@ -325,6 +325,117 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     };
     float tmax = -INFINITY;
+    // ---- first pass, one 32-column group: its maxima, ranked in rv
+    auto max_group = [&](uint32_t (&rg)[32], int lim) {
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rg[e]);
+      if (__any_sync(0xffffffffu, lim < 32)) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = e < lim ? v[e] : -INFINITY;
+      }
+      // max tree: after the step of width w, v[t] (t < w) is the maximum of
+      // the scores e = t (mod w) -- disjoint groups of 32 / w.
+      // tau > 0 and rounding is monotone: tau * max = max of the scores.
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = fmaxf(v[e], v[e + 16]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = fmaxf(v[e], v[e + 8]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = fmaxf(v[e], v[e + 4]);
+      if (group == 8) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rv_insert(tau * v[e]);
+        return;
+      }
+      v[0] = fmaxf(v[0], v[2]);
+      v[1] = fmaxf(v[1], v[3]);
+      if (group == 16) {
+        rv_insert(tau * v[0]);
+        rv_insert(tau * v[1]);
+        return;
+      }
+      v[0] = fmaxf(v[0], v[1]);
+      if (group == 32) rv_insert(tau * v[0]);
+      else tmax = fmaxf(tmax, v[0]);
+    };
+    // ---- scan, one 32-column group: test every score against thr, keep the
+    // passing ones
+    auto scan_group = [&](uint32_t (&rg)[32], int lim, int64_t cbase) {
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rg[e]);
+      uint32_t bits = 0;
+      if (lim > 0) {
+        // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
+        // four independent 8-bit chains keep the dependency depth short
+        uint32_t part[4] = {0u, 0u, 0u, 0u};
+        const uint64_t thr2 = pack2(thr);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t s0, s1;
+            fma2_signs(v[8 * q4 + e], v[8 * q4 + e + 1], ntau2, thr2, s0, s1);
+            part[q4] = __funnelshift_l(s0, part[q4], 1);
+            part[q4] = __funnelshift_l(s1, part[q4], 1);
+          }
+        }
+        bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
+        if (lim < 32) bits &= ~(0xFFFFFFFFu >> lim);
+      }
+      if constexpr (KCAP > 0) {
+        // the buffer holds at least K + 32 entries and a compaction leaves at
+        // most K, so one check per group makes room for all its scores
+        if (__any_sync(0xffffffffu, count + __popc(bits) > p.cap)) keep_best(false, nullptr, nullptr);
+        // append the passing scores, one per lane and round; the score is
+        // picked out of the registers by a 5-level select on its column
+        while (__any_sync(0xffffffffu, bits != 0u)) {
+          const bool has = bits != 0u;
+          const int e = __clz(bits) & 31;
+          bits &= ~(0x80000000u >> e);
+          float w16[16], w8[8], w4[4], w2[2];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) w16[t] = (e & 16) ? v[t + 16] : v[t];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) w8[t] = (e & 8) ? w16[t + 8] : w16[t];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) w4[t] = (e & 4) ? w8[t + 4] : w8[t];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) w2[t] = (e & 2) ? w4[t + 2] : w4[t];
+          const float x = tau * ((e & 1) ? w2[1] : w2[0]);
+          if (has) {
+            tv[count * C::M] = x;
+            ti[count * C::M] = int32_t(cbase + e);
+            ++count;
+          }
+        }
+      } else {
+        if (!__any_sync(0xffffffffu, bits != 0)) return;
+        if (bits) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+        while (bits) {
+          const int e = __clz(bits);
+          bits &= ~(0x80000000u >> e);
+          const float sc = tau * my_stg[e];
+          const int32_t cid = int32_t(cbase + e);
+          if (count == K && !(sc > thr)) continue;
+          int q = count < K ? count : K - 1;
+          while (q > 0 && tv[(q - 1) * C::M] < sc) {
+            tv[q * C::M] = tv[(q - 1) * C::M];
+            ti[q * C::M] = ti[(q - 1) * C::M];
+            --q;
+          }
+          tv[q * C::M] = sc;
+          ti[q * C::M] = cid;
+          if (count < K) ++count;
+          if (count == K) thr = tv[(K - 1) * C::M];
+        }
+      }
+    };
     for (int jg = 0; jg < n_steps; ++jg) {
       const int buf = jg % C::BUFS, ub = jg / C::BUFS;
       const int j = jg % n_tiles;
@@ -335,130 +446,26 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // candidates of this row left in the tile (clamped to 0..128)
       const int64_t left64 = n_cand - c0;
       const int left = left64 <= 0 ? 0 : (left64 >= C::NT ? C::NT : int(left64));
+      // the tile's four 32-column groups (loading the next group while one is
+      // processed measured slower: more registers, more code)
+      uint32_t ra[32];
       if (KCAP > 0 && n_pass == 2 && jg < n_tiles) {
-        // ---- first pass: the row's group maxima, ranked in rv
 #pragma unroll 1
         for (int gi = 0; gi < C::NT / 32; ++gi) {
-          float v[32];
-          tmem_ld32(tb + gi * 32, v);
-          const int lim = left - gi * 32;
-          if (__any_sync(0xffffffffu, lim < 32)) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = e < lim ? v[e] : -INFINITY;
-          }
-          // max tree: after the step of width w, v[t] (t < w) is the maximum
-          // of the scores e = t (mod w) -- disjoint groups of 32 / w.
-          // tau > 0 and rounding is monotone: tau * max = max of the scores.
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = fmaxf(v[e], v[e + 16]);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = fmaxf(v[e], v[e + 8]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[e] = fmaxf(v[e], v[e + 4]);
-          if (group == 8) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) rv_insert(tau * v[e]);
-            continue;
-          }
-          v[0] = fmaxf(v[0], v[2]);
-          v[1] = fmaxf(v[1], v[3]);
-          if (group == 16) {
-            rv_insert(tau * v[0]);
-            rv_insert(tau * v[1]);
-            continue;
-          }
-          v[0] = fmaxf(v[0], v[1]);
-          if (group == 32) {
-            rv_insert(tau * v[0]);
-            continue;
-          }
-          tmax = fmaxf(tmax, v[0]);
+          tmem_ld32_async(tb + gi * 32, ra);
+          tmem_ld_wait(ra);
+          max_group(ra, left - gi * 32);
         }
         if (group == C::NT) {
           rv_insert(tau * tmax);
           tmax = -INFINITY;
         }
       } else {
-        // ---- scan: test every score against thr, keep the passing ones
 #pragma unroll 1
         for (int gi = 0; gi < C::NT / 32; ++gi) {
-          float v[32];
-          tmem_ld32(tb + gi * 32, v);
-          const int64_t cbase = c0 + gi * 32;
-          const int lim = left - gi * 32;
-          uint32_t bits = 0;
-          if (lim > 0) {
-            // bit (31-e) = [tau * v[e] > thr], exactly: sign of fma(-tau, v, thr);
-            // four independent 8-bit chains keep the dependency depth short
-            uint32_t part[4] = {0u, 0u, 0u, 0u};
-            const uint64_t thr2 = pack2(thr);
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t s0, s1;
-                fma2_signs(v[8 * q4 + e], v[8 * q4 + e + 1], ntau2, thr2, s0, s1);
-                part[q4] = __funnelshift_l(s0, part[q4], 1);
-                part[q4] = __funnelshift_l(s1, part[q4], 1);
-              }
-            }
-            bits = (part[0] << 24) | ((part[1] & 0xFFu) << 16) | ((part[2] & 0xFFu) << 8) | (part[3] & 0xFFu);
-            if (lim < 32) bits &= ~(0xFFFFFFFFu >> lim);
-          }
-          if constexpr (KCAP > 0) {
-            // append the passing scores, one per lane and round; the score is
-            // picked out of the registers by a 5-level select on its column.
-            // All lanes compact their buffers together once one is full.
-            while (true) {
-              const uint32_t flags = (bits != 0u ? 1u : 0u) | (count == p.cap ? 2u : 0u);
-              const uint32_t any = __reduce_or_sync(0xffffffffu, flags);
-              if (!(any & 1u)) break;
-              if (any & 2u) keep_best(false, nullptr, nullptr);
-              const bool has = bits != 0u;
-              const int e = __clz(bits) & 31;
-              bits &= ~(0x80000000u >> e);
-              float w16[16], w8[8], w4[4], w2[2];
-#pragma unroll
-              for (int t = 0; t < 16; ++t) w16[t] = (e & 16) ? v[t + 16] : v[t];
-#pragma unroll
-              for (int t = 0; t < 8; ++t) w8[t] = (e & 8) ? w16[t + 8] : w16[t];
-#pragma unroll
-              for (int t = 0; t < 4; ++t) w4[t] = (e & 4) ? w8[t + 4] : w8[t];
-#pragma unroll
-              for (int t = 0; t < 2; ++t) w2[t] = (e & 2) ? w4[t + 2] : w4[t];
-              const float x = tau * ((e & 1) ? w2[1] : w2[0]);
-              if (has) {
-                tv[count * C::M] = x;
-                ti[count * C::M] = int32_t(cbase + e);
-                ++count;
-              }
-            }
-          } else if (__any_sync(0xffffffffu, bits != 0)) {
-            if (bits) {
-#pragma unroll
-              for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            }
-            {
-              while (bits) {
-                const int e = __clz(bits);
-                bits &= ~(0x80000000u >> e);
-                const float sc = tau * my_stg[e];
-                const int32_t cid = int32_t(cbase + e);
-                if (count == K && !(sc > thr)) continue;
-                int q = count < K ? count : K - 1;
-                while (q > 0 && tv[(q - 1) * C::M] < sc) {
-                  tv[q * C::M] = tv[(q - 1) * C::M];
-                  ti[q * C::M] = ti[(q - 1) * C::M];
-                  --q;
-                }
-                tv[q * C::M] = sc;
-                ti[q * C::M] = cid;
-                if (count < K) ++count;
-                if (count == K) thr = tv[(K - 1) * C::M];
-              }
-            }
-          }
+          tmem_ld32_async(tb + gi * 32, ra);
+          tmem_ld_wait(ra);
+          scan_group(ra, left - gi * 32, c0 + gi * 32);
         }
       }
       tc_fence_before();
