@@ -562,21 +562,24 @@ template <int D>
 struct CcTc {
   static constexpr int M = kCcTileRows;
   static constexpr int KATOMS = D / 64;
-  static constexpr int NS = 3;                      // shared-memory stages
+  static constexpr int NS = 2;                      // shared-memory load stages
   static constexpr uint32_t Q_ATOM = M * 128;       // 16 KB
   static constexpr uint32_t KV_ATOM = kChunk * 128; // 8 KB
   static constexpr uint32_t Q_BYTES = KATOMS * Q_ATOM;
   static constexpr uint32_t K_BYTES = KATOMS * KV_ATOM;
   static constexpr uint32_t P_BYTES = M * 128;      // 128 rows x 64 keys bf16
-  // P overwrites the stage's Q tile once S = Q K^T is done; once P V is done
-  // the whole stage holds the tile's fp32 output rows (4D bytes each, padded
-  // to a 4D + 16 byte stride so the row-per-thread stores of 8 consecutive
-  // rows hit distinct banks) until the bulk reductions have read them
+  // P overwrites the stage's Q tile once S = Q K^T is done; the stage goes
+  // back to the producer as soon as P V is done.  A separate buffer holds a
+  // tile's fp32 output rows (4D bytes each, padded to a 4D + 16 byte stride
+  // so the row-per-thread stores of 8 consecutive rows hit distinct banks)
+  // until the bulk reductions have read them.
   static constexpr uint32_t O_ROW = D * 4;
   static constexpr uint32_t O_STRIDE = O_ROW + 16;
-  static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES + 2048;
+  static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES;
   static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES, OFF_P = 0;
-  static constexpr uint32_t OFF_META = NS * STAGE;                // per stage: rows[128] i32, fac[128] f32, n
+  static constexpr uint32_t OFF_O = NS * STAGE;
+  static constexpr uint32_t O_BYTES = (M * O_STRIDE + 1023u) & ~1023u;
+  static constexpr uint32_t OFF_META = OFF_O + O_BYTES;           // per stage: rows[128] i32, fac[128] f32, n
   static constexpr uint32_t META = M * 4 + M * 4 + 16;
   static constexpr uint32_t OFF_BAR = OFF_META + NS * META;
   static constexpr uint32_t SMEM_MIN = OFF_BAR + 16 * 8 + 32 + 1024;
@@ -592,7 +595,6 @@ struct CcTc {
   static constexpr uint32_t IDESC_O = sm100::idesc_bf16(M, D) | (1u << 16);
   static constexpr int THREADS = 192;
   static_assert(P_BYTES <= Q_BYTES, "P reuses the Q tile");
-  static_assert(M * O_STRIDE <= STAGE, "output rows fit the stage");
 };
 
 struct CcTcParams {
@@ -615,7 +617,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* load_full = bars;        // [NS] producer -> MMA, softmax
-  uint64_t* load_empty = bars + 3;   // [NS] epilogue (output rows read out) -> producer
+  uint64_t* load_empty = bars + 3;   // [NS] MMA (after P V) -> producer
   uint64_t* p_full = bars + 6;       // [NS] softmax -> MMA
   uint64_t* s_full = bars + 9;       // [2] MMA -> softmax
   uint64_t* o_full = bars + 11;      // [2] MMA -> epilogue
@@ -631,7 +633,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (tid == 0) {
     for (int t = 0; t < C::NS; ++t) {
       mbar_init(&load_full[t], 1);
-      mbar_init(&load_empty[t], 4);
+      mbar_init(&load_empty[t], 1);
       mbar_init(&p_full[t], 4);
     }
     for (int t = 0; t < 2; ++t) {
@@ -752,25 +754,30 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mma_bf16(t_o, desc_sw128(sp + kk * 32), desc_sw128_mn(sv + kk * 2048, C::KV_ATOM), C::IDESC_O,
                    kk > 0 ? 1u : 0u);
         mma_commit(&o_full[b]);
+        mma_commit(&load_empty[s]);
       }
       *consumed_slot = j;
       mma_commit(done);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Software-pipelined: the softmax of tile j+1 runs while the tensor core
+    // does P V of tile j, then tile j's output is written.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t t_lane = uint32_t(quarter * 32) << 16;
     const float k2 = c.tau * 1.4426950408889634f;   // scores in log2 units
-    for (int j = 0; j < n_my; ++j) {
-      const int s = j % C::NS, u = j / C::NS, b = j & 1, ub = j >> 1;
-      if (!mbar_wait(&load_full[s], u & 1, abort_flag)) break;
+    // softmax of tile jj: P into the stage (over its Q tile); returns the
+    // row's global row id (-1 when the row is not live) or -2 on abort
+    auto softmax_tile = [&](int jj) -> int64_t {
+      const int s = jj % C::NS, u = jj / C::NS, b = jj & 1, ub = jj >> 1;
+      if (!mbar_wait(&load_full[s], u & 1, abort_flag)) return -2;
       const uint8_t* meta = smem + C::OFF_META + s * C::META;
       const int n = reinterpret_cast<const int32_t*>(meta + C::M * 8)[0];
       const bool live = r < n;
       const int64_t grow = reinterpret_cast<const int32_t*>(meta)[r];
       const float fac = reinterpret_cast<const float*>(meta + C::M * 4)[r];
-      if (!mbar_wait(&s_full[b], ub & 1, abort_flag)) break;
+      if (!mbar_wait(&s_full[b], ub & 1, abort_flag)) return -2;
       tc_fence_after();
       float sc[64];
       {
@@ -813,10 +820,17 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
-      if (!mbar_wait(&o_full[b], ub & 1, abort_flag)) break;
+      return live ? grow : -1;
+    };
+    // output of tile jj: the fp32 output rows go through the output buffer
+    // (once the previous tile's rows have been read out of it) and are added
+    // to the accumulator by one bulk reduction per row
+    const uint32_t orow = smem_u32(smem + C::OFF_O) + uint32_t(r) * C::O_STRIDE;
+    auto output_tile = [&](int jj, int64_t grow) -> bool {
+      const int b = jj & 1, ub = jj >> 1;
+      if (!mbar_wait(&o_full[b], ub & 1, abort_flag)) return false;
       tc_fence_after();
-      // P V is done: the stage is free for this tile's output rows
-      const uint32_t orow = smem_u32(smem + s * C::STAGE) + uint32_t(r) * C::O_STRIDE;
+      bulk_wait_read<0>();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         float o[32];
@@ -831,14 +845,16 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[b]);
       fence_proxy_async_smem();
-      if (live) bulk_reduce_add_f32(p.oacc + grow * D, orow, C::O_ROW);
+      if (grow >= 0) bulk_reduce_add_f32(p.oacc + grow * D, orow, C::O_ROW);
       bulk_commit();
-      // the previous tile's rows have been read: hand its stage back
-      if (j > 0) {
-        bulk_wait_read<1>();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&load_empty[(j - 1) % C::NS]);
-      }
+      return true;
+    };
+    int64_t g_cur = n_my > 0 ? softmax_tile(0) : -2;
+    for (int j = 0; j < n_my && g_cur != -2; ++j) {
+      const int64_t g_next = j + 1 < n_my ? softmax_tile(j + 1) : -1;
+      if (g_next == -2) break;
+      if (!output_tile(j, g_cur)) break;
+      g_cur = g_next;
     }
     bulk_wait_all();
   }
