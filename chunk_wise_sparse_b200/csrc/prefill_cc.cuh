@@ -61,6 +61,11 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src_sme
                "r"(src_smem), "r"(bytes)
                : "memory");
 }
+// global[addr .. addr+16) += {a, b, c, d} as fp32, in L2
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // this thread's bulk groups except the newest n have finished reading shared memory
 template <int n>
@@ -822,15 +827,23 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (lane == 0) mbar_arrive(&p_full[s]);
       return live ? grow : -1;
     };
-    // output of tile jj: the fp32 output rows go through the output buffer
-    // (once the previous tile's rows have been read out of it) and are added
-    // to the accumulator by one bulk reduction per row
+    // output of tile jj: each thread stages its fp32 output row in the output
+    // buffer (once the previous tile's rows have been read out of it), then
+    // the rows are added to the accumulator.  d = 64: one bulk reduction per
+    // row (256 B) by the bulk-copy unit.  d = 128: the warp reads its 32 rows
+    // back D / 4 lanes per row and adds them with coalesced 16-byte
+    // reductions, one row per instruction (measured faster at d = 128,
+    // slower at d = 64).
+    constexpr int LPR = D / 4;            // lanes per row
+    constexpr int RPI = 32 / LPR;         // rows per instruction
+    constexpr bool kBulk = D == 64;
     const uint32_t orow = smem_u32(smem + C::OFF_O) + uint32_t(r) * C::O_STRIDE;
+    const uint32_t obase = smem_u32(smem + C::OFF_O) + uint32_t(quarter * 32) * C::O_STRIDE;
     auto output_tile = [&](int jj, int64_t grow) -> bool {
       const int b = jj & 1, ub = jj >> 1;
       if (!mbar_wait(&o_full[b], ub & 1, abort_flag)) return false;
       tc_fence_after();
-      bulk_wait_read<0>();
+      if constexpr (kBulk) bulk_wait_read<0>();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         float o[32];
@@ -844,9 +857,26 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[b]);
-      fence_proxy_async_smem();
-      if (grow >= 0) bulk_reduce_add_f32(p.oacc + grow * D, orow, C::O_ROW);
-      bulk_commit();
+      if constexpr (kBulk) {
+        fence_proxy_async_smem();
+        if (grow >= 0) bulk_reduce_add_f32(p.oacc + grow * D, orow, C::O_ROW);
+        bulk_commit();
+      } else {
+        const int32_t g32 = int32_t(grow);   // rows < 2^31; -1 when the row is not live
+        const int sub = lane / LPR, col = (lane % LPR) * 4;
+#pragma unroll 4
+        for (int i = 0; i < 32; i += RPI) {
+          const int rr = i + sub;
+          const int32_t g = __shfl_sync(0xffffffffu, g32, rr);
+          float4 val;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(val.x), "=f"(val.y), "=f"(val.z), "=f"(val.w)
+                       : "r"(obase + uint32_t(rr) * C::O_STRIDE + uint32_t(col) * 4)
+                       : "memory");
+          if (g >= 0) red_add_v4(p.oacc + int64_t(g) * D + col, val.x, val.y, val.z, val.w);
+        }
+        __syncwarp();
+      }
       return true;
     };
     int64_t g_cur = n_my > 0 ? softmax_tile(0) : -2;
