@@ -16,9 +16,10 @@
 //                 order-preserving integer image of the score), then a
 //                 stable compaction in ascending chunk id; ties among equal
 //                 scores go to the lower ids.
-//   D3 partials : split-K over the K kept chunks plus the own chunk: one warp
-//                 per (row, chunk) computes the intra-chunk softmax output
-//                 and carries the chunk's fusion score.
+//   D3 partials : per (batch, kv head), each distinct chunk kept by any of the
+//                 G query heads (plus the own chunk) is read once and attended
+//                 by every head that kept it; one partial (score, output) per
+//                 (row, slot).
 //   D4 combine  : softmax over the chunk scores fuses the partials.
 #pragma once
 #include "attend_simt.cuh"
@@ -62,15 +63,18 @@ __device__ __forceinline__ int64_t decode_own_chunk(const int32_t* seqlens, int 
 
 constexpr int kDecChunksPerCta = 128;
 
+// One thread per candidate chunk: it reads the chunk's compressed-key row
+// once (16-byte loads) and scores it against the G query heads of the kv head
+// (query rows broadcast from shared memory), four heads per pass over the
+// row.  No cross-lane reductions.
 template <typename T, int D, bool MMA_OPERAND>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kDecChunksPerCta)
 decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, const float* __restrict__ bp,
                      const __nv_bfloat16* __restrict__ kmma, const int32_t* __restrict__ seqlens, int64_t cap,
                      int64_t nc, int Hq, int G, int Hkv, float tau, float* __restrict__ ws_scores) {
   using KT = typename std::conditional<MMA_OPERAND, __nv_bfloat16, float>::type;
-  using L = RowLayout<KT, D>;
-  constexpr int E = L::E, LPK = L::LPK, KPI = L::KPI;
-  constexpr int RS = MMA_OPERAND ? D + kExt : D;  // row stride of the k' rows
+  constexpr int E = Vec16<KT>::E;                   // elements per 16-byte load
+  constexpr int RS = MMA_OPERAND ? D + kExt : D;    // row stride of the k' rows
   extern __shared__ __align__(16) float sq[];       // [G][D]
   const int bh = blockIdx.y;
   const int b = bh / Hkv, h = bh % Hkv;
@@ -86,35 +90,36 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
     else sq[idx] = x;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int grp = lane / LPK, sub = lane % LPK;
-  const int64_t cw0 = int64_t(blockIdx.x) * kDecChunksPerCta + warp * 32;
-  const KT* base = MMA_OPERAND ? reinterpret_cast<const KT*>(kmma) : reinterpret_cast<const KT*>(kp);
-  base += int64_t(bh) * nc * RS;
-  for (int it = 0; it < 32 / KPI; ++it) {
-    const int64_t c = cw0 + it * KPI + grp;
-    if (cw0 + it * KPI >= own) break;               // uniform
-    const bool ok = c < own;
-    const int64_t cc = ok ? c : cw0;
-    float kv[E];
-    Vec16<KT>::load(base + cc * RS + sub * E, kv);
-    float bias;
-    if constexpr (MMA_OPERAND) {
-      const __nv_bfloat16* ext = kmma + (int64_t(bh) * nc + cc) * RS + D;
-      bias = __bfloat162float(ext[0]) + __bfloat162float(ext[1]);
-    } else {
-      bias = __ldg(bp + int64_t(bh) * nc + cc);
-    }
-    for (int g = 0; g < G; ++g) {
-      float part = 0.f;
+  const int64_t c = int64_t(blockIdx.x) * kDecChunksPerCta + threadIdx.x;
+  if (c >= own) return;
+  const KT* row = (MMA_OPERAND ? reinterpret_cast<const KT*>(kmma) : reinterpret_cast<const KT*>(kp)) +
+                  (int64_t(bh) * nc + c) * RS;
+  float bias;
+  if constexpr (MMA_OPERAND) {
+    const __nv_bfloat16* ext = kmma + (int64_t(bh) * nc + c) * RS + D;
+    bias = __bfloat162float(ext[0]) + __bfloat162float(ext[1]);
+  } else {
+    bias = __ldg(bp + int64_t(bh) * nc + c);
+  }
+  float* out = ws_scores + (int64_t(b) * Hq + h * G) * nc + c;
+  for (int g0 = 0; g0 < G; g0 += 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int k0 = 0; k0 < D; k0 += E) {
+      float kv[E];
+      Vec16<KT>::load(row + k0, kv);
 #pragma unroll
-      for (int e = 0; e < E; ++e) part = fmaf(sq[g * D + sub * E + e], kv[e], part);
-      const float dot = group_sum<LPK>(part);
-      if (ok && sub == 0) {
-        const float s = MMA_OPERAND ? tau * (dot + bias) : fmaf(tau, dot, bias);
-        ws_scores[(int64_t(b) * Hq + h * G + g) * nc + c] = s;
+      for (int j = 0; j < 4; ++j) {
+        if (g0 + j < G) {
+          const float* qg = sq + (g0 + j) * D + k0;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[j] = fmaf(qg[e], kv[e], acc[j]);
+        }
       }
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (g0 + j < G) out[int64_t(g0 + j) * nc] = MMA_OPERAND ? tau * (acc[j] + bias) : fmaf(tau, acc[j], bias);
   }
 }
 
@@ -227,52 +232,197 @@ decode_topk_kernel(const float* __restrict__ ws_scores, const int32_t* __restric
   }
 }
 
+// D3, grouped by kv head: the G query heads of a kv head select overlapping
+// chunk sets, so each distinct chunk is read once and attended by all heads
+// that kept it.  One single-warp CTA per candidate slot (g, k) of the
+// (b, kv head)'s G x K selections, plus one for the own chunk.  A slot whose
+// chunk already appears for an earlier head is skipped; otherwise the warp
+// finds the heads that kept the chunk (binary search in their ascending id
+// lists, one lane per head), brings the chunk's 64 key and value rows into
+// shared memory with all copies in flight at once (cp.async, 16 bytes per
+// copy; keys with the 16-byte blocks of row r rotated by r mod 8 so that the
+// key-per-lane reads hit distinct banks), then, four heads at a time,
+// computes the scores (lanes own keys), the softmax (warp reductions) and
+// P V (lanes own dims, weights broadcast by shuffle).  Each head's partial
+// goes to its own slot; invalid slots get score -inf.
+template <typename T, int D>
+struct DecUnion {
+  static constexpr int RB = D * int(sizeof(T));   // bytes per key / value row
+  static constexpr int NB = RB / 16;             // 16-byte blocks per row
+  static constexpr uint32_t TILE = uint32_t(kChunk) * RB;
+  // keys, values, queries, kept ids, then per-head slots and a flag (all dynamic:
+  // the kernel may be given the largest dynamic size, which leaves no room
+  // for static shared memory)
+  static size_t smem(int G, int K) {
+    return 2 * size_t(TILE) + sizeof(float) * size_t(G) * D + sizeof(int32_t) * size_t(G) * K +
+           sizeof(int32_t) * 33 + 16;
+  }
+};
+
+// 16 bytes from shared memory (shared-window address) as 8 bf16 or 4 fp32 values
+template <typename T>
+__device__ __forceinline__ void lds16(uint32_t saddr, float (&x)[16 / sizeof(T)]) {
+  uint32_t w[4];
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(saddr));
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+      x[2 * i] = __low2float(v);
+      x[2 * i + 1] = __high2float(v);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(w[i]);
+  }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
-decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                      const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int G, int Hkv, int K,
-                      float tau, const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
-                      float* __restrict__ part_u, float* __restrict__ part_o, int64_t n_units) {
-  using L = RowLayout<T, D>;
-  constexpr int E = L::E, LPK = L::LPK;
-  const int lane = threadIdx.x & 31, sub = lane % LPK;
-  const int64_t unit = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (unit >= n_units) return;
-  const int64_t row = unit / (K + 1);
-  const int slot = int(unit % (K + 1));
-  const int b = int(row / Hq), hq = int(row % Hq);
+decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+                            const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int G, int Hkv, int K,
+                            float tau, const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
+                            float* __restrict__ part_u, float* __restrict__ part_o) {
+  using U = DecUnion<T, D>;
+  constexpr int EL = D / 32;                 // output dims per lane
+  constexpr int EB = 16 / int(sizeof(T));    // elements per 16-byte block
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t* sk = dsm;                                            // [64][D] keys, blocks rotated
+  uint8_t* sv = dsm + U::TILE;                                  // [64][D] values
+  float* sq = reinterpret_cast<float*>(dsm + 2 * U::TILE);      // [G][D] queries
+  int32_t* sid = reinterpret_cast<int32_t*>(sq + G * D);        // [G][K] kept ids, ascending
+  int* s_slot = sid + G * K;   // [32] per head: the chunk's slot in its list, -1 if not kept
+  int& s_go = s_slot[32];
+  const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row0 = int64_t(b) * Hq + int64_t(h) * G;
+  const int pidx = blockIdx.x;   // candidate slot g * K + k, or G * K for the own chunk
   const int64_t own = decode_own_chunk(seqlens, b, cap);
-  float* uo = part_u + row * (K + 1) + slot;
-  float* po = part_o + (row * (K + 1) + slot) * D;
   if (own < 0) {
-    if (lane == 0) *uo = -INFINITY;
+    if (tid == 0 && pidx < G * K) part_u[(row0 + pidx / K) * (K + 1) + pidx % K] = -INFINITY;
+    if (tid < G && pidx == G * K) part_u[(row0 + tid) * (K + 1) + K] = -INFINITY;
     return;
   }
-  const int64_t t = int64_t(__ldg(seqlens + b)) - 1;
-  const int64_t bh = int64_t(b) * Hkv + hq / G;
-  const T* kbh = kc + bh * cap * D;
-  const T* vbh = vc + bh * cap * D;
-  float qv[E];
-  Vec16<T>::load(q + row * D + sub * E, qv);
-  float oc[E];
-  float u;
-  if (slot == K) {
-    u = attend_range<T, D>(qv, kbh, vbh, own * kChunk, t + 1, tau, oc);
+  for (int idx = tid; idx < G * K; idx += 128) sid[idx] = sel_ids[row0 * K + idx];
+  __syncthreads();
+  int64_t j0, j1;
+  if (pidx == G * K) {
+    j0 = own * kChunk;
+    j1 = int64_t(__ldg(seqlens + b));
+    if (tid < G) s_slot[tid] = K;
+    if (tid == 0) s_go = 1;
   } else {
-    const int32_t c = sel_ids[row * K + slot];
-    if (c < 0 || c >= own) {
-      if (lane == 0) *uo = -INFINITY;
-      return;
+    const int g = pidx / K, k = pidx % K;
+    const int32_t c = sid[g * K + k];
+    j0 = int64_t(c) * kChunk;
+    j1 = j0 + kChunk;
+    if (warp == 0) {
+      const bool bad = c < 0 || c >= own;
+      int my_slot = -1;
+      if (!bad && lane < G) {
+        const int32_t* ids = sid + lane * K;
+        int lo = 0, hi = K - 1;
+        while (lo <= hi) {
+          const int mid = (lo + hi) >> 1;
+          const int32_t v = ids[mid];
+          if (v == c) { my_slot = mid; break; }
+          // -1 padding sorts after the real ids
+          if (v >= 0 && v < c) lo = mid + 1; else hi = mid - 1;
+        }
+      }
+      const uint32_t mask = __ballot_sync(0xffffffffu, my_slot >= 0);
+      if (lane < G) s_slot[lane] = my_slot;
+      if (lane == 0) {
+        if (bad) {
+          part_u[(row0 + g) * (K + 1) + k] = -INFINITY;
+          if (c >= own) record_error(HILS_ERR_DEVICE_BOUNDS);
+        }
+        // an earlier head's CTA takes a chunk that head also kept
+        s_go = !bad && !(mask & ((1u << g) - 1u));
+      }
     }
-    attend_range<T, D>(qv, kbh, vbh, int64_t(c) * kChunk, int64_t(c + 1) * kChunk, tau, oc);
-    u = sel_scores[row * K + slot];
   }
-  if (lane < LPK) {
+  __syncthreads();
+  if (!s_go) return;
+  // the chunk's 64 key and value rows, all copies in flight at once (the own
+  // chunk lies inside the cache, whose capacity is a multiple of 64; keys
+  // after the query are masked below)
+  const int64_t bhk = int64_t(b) * Hkv + h;
+  const uint8_t* kg = reinterpret_cast<const uint8_t*>(kc + (bhk * cap + j0) * D);
+  const uint8_t* vg = reinterpret_cast<const uint8_t*>(vc + (bhk * cap + j0) * D);
+  const uint32_t sk_a = uint32_t(__cvta_generic_to_shared(sk)), sv_a = uint32_t(__cvta_generic_to_shared(sv));
+#pragma unroll 4
+  for (int t = tid; t < kChunk * U::NB; t += 128) {
+    const int r = t / U::NB, blk = t % U::NB;
+    cp_async16(sk_a + uint32_t(r * U::RB + ((blk ^ (r & 7)) << 4)), kg + size_t(t) * 16);
+    cp_async16(sv_a + uint32_t(t) * 16, vg + size_t(t) * 16);
+  }
+  for (int idx = tid; idx < G * D; idx += 128) {
+    const T x = q[row0 * D + idx];
+    if constexpr (sizeof(T) == 2) sq[idx] = __bfloat162float(x);
+    else sq[idx] = x;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int ra = lane, rb = lane + 32;
+  const bool va = j0 + ra < j1, vb = j0 + rb < j1;
+  for (int g = warp; g < G; g += 4) {
+    const int slot = s_slot[g];
+    if (slot < 0) continue;   // warp-uniform
+    // scores of the lane's two keys
+    float sa = 0.f, sb = 0.f;
+    const float* qg = sq + g * D;
+#pragma unroll 4
+    for (int blk = 0; blk < U::NB; ++blk) {
+      float xa[EB], xb[EB];
+      lds16<T>(sk_a + uint32_t(ra * U::RB + ((blk ^ (ra & 7)) << 4)), xa);
+      lds16<T>(sk_a + uint32_t(rb * U::RB + ((blk ^ (rb & 7)) << 4)), xb);
 #pragma unroll
-    for (int e = 0; e < E; e += 4)
-      *reinterpret_cast<float4*>(po + sub * E + e) = make_float4(oc[e], oc[e + 1], oc[e + 2], oc[e + 3]);
+      for (int e = 0; e < EB; ++e) {
+        sa = fmaf(qg[blk * EB + e], xa[e], sa);
+        sb = fmaf(qg[blk * EB + e], xb[e], sb);
+      }
+    }
+    // softmax over the chunk's keys (keys after the query excluded)
+    const float za = va ? sa * tau : -INFINITY, zb = vb ? sb * tau : -INFINITY;
+    float m = fmaxf(za, zb);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float pa = va ? expf(za - m) : 0.f, pb = vb ? expf(zb - m) : 0.f;
+    float l = pa + pb;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    // P V: lane owns dims lane * EL .. + EL - 1
+    float o[EL];
+#pragma unroll
+    for (int e = 0; e < EL; ++e) o[e] = 0.f;
+    const int nk = int(j1 - j0);
+#pragma unroll 8
+    for (int jj = 0; jj < nk; ++jj) {
+      const T* vrow = reinterpret_cast<const T*>(sv + jj * U::RB) + lane * EL;
+      const float pj = __shfl_sync(0xffffffffu, jj < 32 ? pa : pb, jj & 31);
+#pragma unroll
+      for (int e = 0; e < EL; ++e) {
+        float x;
+        if constexpr (sizeof(T) == 2) x = __bfloat162float(vrow[e]);
+        else x = vrow[e];
+        o[e] = fmaf(pj, x, o[e]);
+      }
+    }
+    const int64_t row = row0 + g;
+    float* po = part_o + (row * (K + 1) + slot) * D + lane * EL;
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int e = 0; e < EL; ++e) po[e] = o[e] * inv;
+    if (lane == 0) part_u[row * (K + 1) + slot] = slot == K ? m + logf(l) : sel_scores[row * K + slot];
   }
-  if (lane == 0) *uo = u;
 }
 
 template <typename T, int D>

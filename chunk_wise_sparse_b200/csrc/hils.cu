@@ -54,7 +54,11 @@ cudaError_t set_smem_max() {
   cudaGetDevice(&dev);
   const uint32_t bit = 1u << (dev & 31);
   if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(FN, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  // the per-block limit covers static and dynamic shared memory together
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, FN);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(FN, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem - int(fa.sharedSizeBytes));
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
   return e;
 }
@@ -335,10 +339,13 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores);
   decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
                                                       ws.sel_scores);
-  const int64_t units = rows * (K + 1);
-  decode_partial_kernel<T, D><<<unsigned((units + 3) / 4), 128, 0, st>>>(
+  const size_t smem3 = DecUnion<T, D>::smem(G, K);
+  constexpr auto k3 = decode_partial_union_kernel<T, D>;
+  if (smem3 > 48 * 1024 && set_smem_max<k3>() != cudaSuccess) return HILS_ERR_CUDA;
+  const dim3 g3(unsigned(G * K + 1), unsigned(d->batch * d->heads_kv));
+  k3<<<g3, 128, smem3, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
-      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, units);
+      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o);
   decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(
       ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
       ids_out, scores_out, rows);
@@ -442,6 +449,7 @@ int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, con
                      hils_stream_t stream) {
   int rc = check_dims(d);
   if (rc) return rc;
+  if (d->heads_q / d->heads_kv > 32) return HILS_ERR_UNSUPPORTED;   // one lane per query head of a kv head
   if (!ptr_ok(q) || !ptr_ok(k_cache) || !ptr_ok(v_cache) || !ptr_ok(seqlens) || !ptr_ok(o) || !ptr_ok(workspace))
     return HILS_ERR_INVALID_ARGUMENT;
   if ((ids_out != nullptr && !aligned16(ids_out)) || (scores_out != nullptr && !aligned16(scores_out)))
@@ -492,6 +500,7 @@ int hils_attn_decode_fixed_scratch(const hils_dims* d, const void* q, const void
                                    hils_stream_t stream) {
   int rc = check_dims(d);
   if (rc) return rc;
+  if (d->heads_q / d->heads_kv > 32) return HILS_ERR_UNSUPPORTED;
   const size_t need = hils_decode_workspace_bytes(d);
   if (need > size_t(HILS_DECODE_FIXED_SCRATCH_BYTES)) return HILS_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = decode_scratch_address();

@@ -173,6 +173,7 @@ size_t hils_decode_workspace_bytes(const hils_dims* dims);
  *   ids_out      [B, Hq, K] int32 out (nullable)
  *   scores_out   [B, Hq, K] fp32 out (nullable)
  *   workspace    device scratch of at least hils_decode_workspace_bytes(dims)
+ * heads_q / heads_kv must be at most 32 (HILS_ERR_UNSUPPORTED otherwise).
  */
 int hils_attn_decode(const hils_dims* dims, const void* q, const void* k_cache, const void* v_cache,
                      const float* kprime, const float* bprime, const void* kprime_mma,

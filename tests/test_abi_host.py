@@ -78,6 +78,14 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert hils.hils_prefill_workspace_bytes(dims(dtype=hils.FP32)) == 0
 
 
+def test_decode_rejects_more_than_32_query_heads_per_kv_head(lib):
+    d = dims(heads_q=64, heads_kv=1)
+    p = ctypes.c_void_p(256)     # never dereferenced: validation fails first
+    big = hils.hils_decode_workspace_bytes(d)
+    assert lib.hils_attn_decode(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, p, big, None) == 2
+    assert lib.hils_attn_decode_fixed_scratch(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, None) == 2
+
+
 def test_strerror(lib):
     for code in range(7):
         assert len(hils.strerror(code)) >= 2
