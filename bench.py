@@ -392,8 +392,25 @@ def run_decode(args, w, rank, world, local_rank):
 
     q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
     B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
-    summ = hils.landmark_summary(k, lq, K)
     dims = hils.make_dims(B, Hq, Hkv, d, N, K, q.dtype)
+    if w.paged:
+        # the cache in chunk pages of a pool, in a seeded random order (setup, untimed)
+        from chunk_wise_sparse_b200.inputs import page_table
+        table, n_pages = page_table(w)
+        nc = N // 64
+        idx = torch.from_numpy(table.reshape(-1).astype(np.int64)).to(dev)
+
+        def paginate(t):
+            pool = torch.empty((n_pages, Hkv, 64, d), dtype=t.dtype, device=dev)
+            pool[idx] = t.view(B, Hkv, nc, 64, d).permute(0, 2, 1, 3, 4).reshape(B * nc, Hkv, 64, d)
+            return pool
+
+        k, v = paginate(k), paginate(v)
+        tab = torch.from_numpy(table).to(dev)
+        summ = hils.Summary(dims, dev)
+        hils.hils_landmark_summary_paged(dims, k, tab, n_pages, lq, 0, nc, summ.kprime, summ.bprime, summ.kprime_mma)
+    else:
+        summ = hils.landmark_summary(k, lq, K)
     seq = torch.full((B,), N, dtype=torch.int32, device=dev)
     ws = torch.empty((hils.hils_decode_workspace_bytes(dims),), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
@@ -403,8 +420,12 @@ def run_decode(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def step():
-        hils.hils_attn_decode(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, o, ids, sc, ws,
-                              stream=stream)
+        if w.paged:
+            hils.hils_attn_decode_paged(dims, q, k, v, tab, n_pages, summ.kprime, summ.bprime, summ.kprime_mma, seq,
+                                        o, ids, sc, ws, stream=stream)
+        else:
+            hils.hils_attn_decode(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, o, ids, sc, ws,
+                                  stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -437,7 +458,8 @@ def run_decode(args, w, rank, world, local_rank):
         "metric": "HiLS decode us/step (one new token per sequence: scoring, top-K, sparse attention)",
         "value": us, "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": f"synthetic: i.i.d. N(0,1), seed {w.seed}",
+        "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": f"synthetic: i.i.d. N(0,1), seed {w.seed}" + (", KV cache in chunk pages (random order)" if w.paged else ""),
         "config": dict(workload_config(w, world), l2="256 MiB buffer written between steps (L2 flush)"),
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,

@@ -21,6 +21,27 @@ __device__ int32_t g_status;
 
 __device__ __forceinline__ void record_error(int32_t code) { atomicCAS(&g_status, 0, code); }
 
+// Where the keys / values of chunk c of (b, h) live.  Contiguous cache
+// (table == nullptr): [B, Hkv, n_tok, d], chunk c at token c*C.  Chunk-paged
+// cache: a pool [n_pages, Hkv, C, d] and table[b * nc + c] = the page of
+// logical chunk c of sequence b.
+struct PagedKv {
+  const int32_t* table;
+  int64_t n_pages;
+};
+// Element offset of the chunk's first row, or -1 (recorded as
+// HILS_ERR_DEVICE_BOUNDS) when its page is outside the pool.
+__device__ __forceinline__ int64_t kv_chunk_offset(const PagedKv& pk, int64_t b, int64_t h, int64_t c, int64_t Hkv,
+                                                   int64_t n_tok, int64_t nc, int64_t D) {
+  if (pk.table == nullptr) return ((b * Hkv + h) * n_tok + c * kChunk) * D;
+  const int64_t page = __ldg(pk.table + b * nc + c);
+  if (page < 0 || page >= pk.n_pages) {
+    record_error(HILS_ERR_DEVICE_BOUNDS);
+    return -1;
+  }
+  return (page * Hkv + h) * kChunk * D;
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte vectors of bf16 (8 elements) or fp32 (4 elements), widened to fp32.
 template <typename T> struct Vec16;

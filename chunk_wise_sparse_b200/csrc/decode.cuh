@@ -255,7 +255,7 @@ struct DecUnion {
   // for static shared memory)
   static size_t smem(int G, int K) {
     return 2 * size_t(TILE) + sizeof(float) * size_t(G) * D + sizeof(int32_t) * size_t(G) * K +
-           sizeof(int32_t) * 33 + 16;
+           sizeof(int32_t) * 36 + 16;
   }
 };
 
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(128)
 decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                             const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int G, int Hkv, int K,
                             float tau, const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
-                            float* __restrict__ part_u, float* __restrict__ part_o) {
+                            float* __restrict__ part_u, float* __restrict__ part_o, PagedKv pk) {
   using U = DecUnion<T, D>;
   constexpr int EL = D / 32;                 // output dims per lane
   constexpr int EB = 16 / int(sizeof(T));    // elements per 16-byte block
@@ -300,6 +300,7 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   int32_t* sid = reinterpret_cast<int32_t*>(sq + G * D);        // [G][K] kept ids, ascending
   int* s_slot = sid + G * K;   // [32] per head: the chunk's slot in its list, -1 if not kept
   int& s_go = s_slot[32];
+  int* s_off = s_slot + 34;   // [2] element offset of the chunk's rows, low and high words
   const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t row0 = int64_t(b) * Hq + int64_t(h) * G;
@@ -351,12 +352,25 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   }
   __syncthreads();
   if (!s_go) return;
+  // where the chunk's rows live (contiguous cache or chunk page); a page
+  // outside the pool is recorded and the chunk counts as not kept
+  if (tid == 0) {
+    const int64_t off = kv_chunk_offset(pk, b, h, j0 / kChunk, Hkv, cap, cap / kChunk, D);
+    s_off[0] = int(uint32_t(uint64_t(off)));
+    s_off[1] = int(uint32_t(uint64_t(off) >> 32));
+    if (off < 0) {
+      for (int g = 0; g < G; ++g)
+        if (s_slot[g] >= 0) part_u[(row0 + g) * (K + 1) + s_slot[g]] = -INFINITY;
+    }
+  }
+  __syncthreads();
+  const int64_t koff = int64_t((uint64_t(uint32_t(s_off[1])) << 32) | uint64_t(uint32_t(s_off[0])));
+  if (koff < 0) return;
   // the chunk's 64 key and value rows, all copies in flight at once (the own
   // chunk lies inside the cache, whose capacity is a multiple of 64; keys
   // after the query are masked below)
-  const int64_t bhk = int64_t(b) * Hkv + h;
-  const uint8_t* kg = reinterpret_cast<const uint8_t*>(kc + (bhk * cap + j0) * D);
-  const uint8_t* vg = reinterpret_cast<const uint8_t*>(vc + (bhk * cap + j0) * D);
+  const uint8_t* kg = reinterpret_cast<const uint8_t*>(kc + koff);
+  const uint8_t* vg = reinterpret_cast<const uint8_t*>(vc + koff);
   const uint32_t sk_a = uint32_t(__cvta_generic_to_shared(sk)), sv_a = uint32_t(__cvta_generic_to_shared(sv));
 #pragma unroll 4
   for (int t = tid; t < kChunk * U::NB; t += 128) {

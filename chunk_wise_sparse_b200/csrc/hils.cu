@@ -286,13 +286,13 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
 
 template <typename T, int D>
 int launch_summary(const hils_dims* d, const void* k, const void* lq, int64_t c0, int64_t c1, float* kp,
-                   float* bp, void* kmma, cudaStream_t st) {
+                   float* bp, void* kmma, cudaStream_t st, PagedKv pk = PagedKv{nullptr, 0}) {
   const int64_t nc = d->seqlen / kChunk, span = c1 - c0;
   const int64_t units = int64_t(d->batch) * d->heads_kv * span;
   const int64_t blocks = (units * 32 + 255) / 256;
   summary_kernel<T, D><<<dim3(unsigned(blocks)), 256, 0, st>>>(
       static_cast<const T*>(k), static_cast<const T*>(lq), d->seqlen, nc, c0, span, units, kp, bp,
-      static_cast<__nv_bfloat16*>(kmma), 1.f / sqrtf(float(D)));
+      static_cast<__nv_bfloat16*>(kmma), 1.f / sqrtf(float(D)), pk, d->heads_kv);
   return launched(1);
 }
 
@@ -324,7 +324,7 @@ int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const 
 template <typename T, int D>
 int launch_decode(const hils_dims* d, const void* q, const void* kc, const void* vc, const float* kp,
                   const float* bp, const void* kmma, const int32_t* seqlens, void* o, int32_t* ids_out,
-                  float* scores_out, void* ws_ptr, cudaStream_t st) {
+                  float* scores_out, void* ws_ptr, cudaStream_t st, PagedKv pk = PagedKv{nullptr, 0}) {
   constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
   const int64_t nc = d->seqlen / kChunk, rows = int64_t(d->batch) * d->heads_q;
   const int G = d->heads_q / d->heads_kv, K = d->topk;
@@ -345,7 +345,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   const dim3 g3(unsigned(G * K + 1), unsigned(d->batch * d->heads_kv));
   k3<<<g3, 128, smem3, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
-      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o);
+      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, pk);
   decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(
       ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
       ids_out, scores_out, rows);
@@ -356,9 +356,9 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
 
 extern "C" {
 
-int hils_landmark_summary(const hils_dims* d, const void* k, const void* lq, int64_t chunk_begin,
-                          int64_t chunk_end, float* kprime, float* bprime, void* kprime_mma,
-                          hils_stream_t stream) {
+static int summary_entry(const hils_dims* d, const void* k, const void* lq, int64_t chunk_begin,
+                         int64_t chunk_end, float* kprime, float* bprime, void* kprime_mma, hils_stream_t stream,
+                         PagedKv pk) {
   int rc = check_dims(d);
   if (rc) return rc;
   const int64_t nc = d->seqlen / kChunk;
@@ -368,11 +368,25 @@ int hils_landmark_summary(const hils_dims* d, const void* k, const void* lq, int
   if (chunk_end == chunk_begin) return HILS_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d->dtype == HILS_BF16) {
-    if (d->head_dim == 64) return launch_summary<__nv_bfloat16, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st);
-    return launch_summary<__nv_bfloat16, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st);
+    if (d->head_dim == 64) return launch_summary<__nv_bfloat16, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st, pk);
+    return launch_summary<__nv_bfloat16, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, st, pk);
   }
-  if (d->head_dim == 64) return launch_summary<float, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st);
-  return launch_summary<float, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st);
+  if (d->head_dim == 64) return launch_summary<float, 64>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st, pk);
+  return launch_summary<float, 128>(d, k, lq, chunk_begin, chunk_end, kprime, bprime, nullptr, st, pk);
+}
+
+int hils_landmark_summary(const hils_dims* d, const void* k, const void* lq, int64_t chunk_begin,
+                          int64_t chunk_end, float* kprime, float* bprime, void* kprime_mma,
+                          hils_stream_t stream) {
+  return summary_entry(d, k, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, stream, PagedKv{nullptr, 0});
+}
+
+int hils_landmark_summary_paged(const hils_dims* d, const void* k_pages, const int32_t* page_table, int64_t n_pages,
+                                const void* lq, int64_t chunk_begin, int64_t chunk_end, float* kprime,
+                                float* bprime, void* kprime_mma, hils_stream_t stream) {
+  if (page_table == nullptr || n_pages < 1) return HILS_ERR_INVALID_ARGUMENT;
+  return summary_entry(d, k_pages, lq, chunk_begin, chunk_end, kprime, bprime, kprime_mma, stream,
+                       PagedKv{page_table, n_pages});
 }
 
 size_t hils_kprime_mma_bytes(const hils_dims* d) {
@@ -443,10 +457,10 @@ size_t hils_decode_workspace_bytes(const hils_dims* d) {
   return decode_ws_layout(int64_t(d->batch) * d->heads_q, d->seqlen / kChunk, d->topk, d->head_dim, nullptr, nullptr);
 }
 
-int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
-                     const float* kprime, const float* bprime, const void* kprime_mma, const int32_t* seqlens,
-                     void* o, int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
-                     hils_stream_t stream) {
+static int decode_entry(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
+                        const float* kprime, const float* bprime, const void* kprime_mma, const int32_t* seqlens,
+                        void* o, int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                        hils_stream_t stream, PagedKv pk) {
   int rc = check_dims(d);
   if (rc) return rc;
   if (d->heads_q / d->heads_kv > 32) return HILS_ERR_UNSUPPORTED;   // one lane per query head of a kv head
@@ -459,13 +473,30 @@ int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, con
   if (d->dtype == HILS_BF16) {
     if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
     if (d->head_dim == 64)
-      return launch_decode<__nv_bfloat16, 64>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st);
-    return launch_decode<__nv_bfloat16, 128>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st);
+      return launch_decode<__nv_bfloat16, 64>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk);
+    return launch_decode<__nv_bfloat16, 128>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk);
   }
   if (!ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
   if (d->head_dim == 64)
-    return launch_decode<float, 64>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st);
-  return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st);
+    return launch_decode<float, 64>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk);
+  return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk);
+}
+
+int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
+                     const float* kprime, const float* bprime, const void* kprime_mma, const int32_t* seqlens,
+                     void* o, int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                     hils_stream_t stream) {
+  return decode_entry(d, q, k_cache, v_cache, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out, workspace,
+                      workspace_bytes, stream, PagedKv{nullptr, 0});
+}
+
+int hils_attn_decode_paged(const hils_dims* d, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* page_table, int64_t n_pages, const float* kprime, const float* bprime,
+                           const void* kprime_mma, const int32_t* seqlens, void* o, int32_t* ids_out,
+                           float* scores_out, void* workspace, size_t workspace_bytes, hils_stream_t stream) {
+  if (page_table == nullptr || n_pages < 1) return HILS_ERR_INVALID_ARGUMENT;
+  return decode_entry(d, q, k_pages, v_pages, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out, workspace,
+                      workspace_bytes, stream, PagedKv{page_table, n_pages});
 }
 
 }  // extern "C"

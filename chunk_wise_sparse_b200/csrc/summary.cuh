@@ -21,7 +21,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256)
 summary_kernel(const T* __restrict__ k, const T* __restrict__ lq, int64_t n_tok, int64_t nc,
                int64_t chunk_begin, int64_t span, int64_t n_units, float* __restrict__ kp,
-               float* __restrict__ bp, __nv_bfloat16* __restrict__ kmma, float tau) {
+               float* __restrict__ bp, __nv_bfloat16* __restrict__ kmma, float tau, PagedKv pk, int Hkv) {
   using L = RowLayout<T, D>;
   constexpr int E = L::E, LPK = L::LPK, KPI = L::KPI;
   constexpr int ITERS = kChunk / KPI;
@@ -32,9 +32,11 @@ summary_kernel(const T* __restrict__ k, const T* __restrict__ lq, int64_t n_tok,
   const int64_t bh = unit / span, c = chunk_begin + unit % span;
   const int grp = lane / LPK, sub = lane % LPK;
 
+  const int64_t koff = kv_chunk_offset(pk, bh / Hkv, bh % Hkv, c, Hkv, n_tok, nc, D);
+  if (koff < 0) return;   // page outside the pool: recorded, chunk left unwritten
   float lqv[E];
   Vec16<T>::load(lq + (bh * nc + c) * D + sub * E, lqv);
-  const T* kc = k + (bh * n_tok + c * kChunk) * D + sub * E;
+  const T* kc = k + koff + sub * E;
 
   // online state of this key group: max m, sum l of exp(z-m), sum s of exp(z-m)*z, acc of exp(z-m)*k
   float m = -INFINITY, l = 0.f, s = 0.f, acc[E];

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUP
 EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_prefill_workspace_bytes",
            "hils_attn_prefill",
            "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
+           "hils_landmark_summary_paged", "hils_attn_decode_paged",
            "hils_get_status", "hils_selftest_bounded_wait", "hils_strerror", "hils_kernel_launches")
 DECODE_FIXED_SCRATCH_BYTES = 16 << 20
 
@@ -61,6 +62,8 @@ def lib():
         L.hils_decode_workspace_bytes.restype = SZ
         L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_attn_decode_fixed_scratch.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P]
+        L.hils_landmark_summary_paged.argtypes = [D, P, P, I64, P, I64, I64, P, P, P, P]
+        L.hils_attn_decode_paged.argtypes = [D, P, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
         L.hils_selftest_bounded_wait.argtypes = [ctypes.c_int32, P]
         L.hils_strerror.argtypes = [ctypes.c_int]
@@ -168,6 +171,24 @@ def hils_attn_decode_fixed_scratch(dims, q, k_cache, v_cache, kprime, bprime, kp
            lib().hils_attn_decode_fixed_scratch(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                                 _ptr(kprime), _ptr(bprime), _ptr(kprime_mma), _ptr(seqlens),
                                                 _ptr(o), _ptr(ids_out), _ptr(scores_out), _stream(stream)))
+
+
+def hils_landmark_summary_paged(dims, k_pages, page_table, n_pages, lq, chunk_begin, chunk_end, kprime, bprime,
+                                kprime_mma=None, stream=None):
+    _check("hils_landmark_summary_paged",
+           lib().hils_landmark_summary_paged(ctypes.byref(dims), _ptr(k_pages), _ptr(page_table), int(n_pages),
+                                             _ptr(lq), int(chunk_begin), int(chunk_end), _ptr(kprime), _ptr(bprime),
+                                             _ptr(kprime_mma), _stream(stream)))
+
+
+def hils_attn_decode_paged(dims, q, k_pages, v_pages, page_table, n_pages, kprime, bprime, kprime_mma, seqlens, o,
+                           ids_out, scores_out, workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("hils_attn_decode_paged",
+           lib().hils_attn_decode_paged(ctypes.byref(dims), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                        int(n_pages), _ptr(kprime), _ptr(bprime), _ptr(kprime_mma), _ptr(seqlens),
+                                        _ptr(o), _ptr(ids_out), _ptr(scores_out), _ptr(workspace), int(nbytes),
+                                        _stream(stream)))
 
 
 def hils_get_status(stream=None) -> int:

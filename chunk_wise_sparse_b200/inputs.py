@@ -63,6 +63,7 @@ class Workload:
     needle_mode: str    # "per_block", "random" or "none"
     kind: str           # "prefill", "decode" or "prefill+decode"
     sample_rows: int    # rows the oracle checks (0 = all rows)
+    paged: bool = False  # decode: the KV cache in chunk pages (page_table)
 
     @property
     def G(self) -> int:
@@ -81,6 +82,9 @@ WORKLOADS = {
                                     "bf16", 32, "random", "prefill", 4096),
     "decode-128k-b8-gqa4-d128": Workload("decode-128k-b8-gqa4-d128", 8, 32, 8, 128, 131072, 64, 32, 2,
                                          "bf16", 0, "none", "decode", 0),
+    # the same decode step with the KV cache in chunk pages drawn in random order
+    "decode-128k-b8-gqa4-d128-paged": Workload("decode-128k-b8-gqa4-d128-paged", 8, 32, 8, 128, 131072, 64, 32, 2,
+                                               "bf16", 0, "none", "decode", 0, paged=True),
     "prefill-128k-gqa4-d128": Workload("prefill-128k-gqa4-d128", 1, 32, 8, 128, 131072, 64, 32, 3,
                                        "bf16", 64, "random", "prefill", 4096),
     "prefill-512k-h16-d64": Workload("prefill-512k-h16-d64", 1, 16, 16, 64, 524288, 64, 16, 4,
@@ -227,6 +231,16 @@ def generate(w: Workload) -> Inputs:
     elif w.dtype != "fp32":
         raise ValueError(w.dtype)
     return inp
+
+
+def page_table(w: Workload, spare: int = 0) -> tuple[np.ndarray, int]:
+    """A chunk page table [B, nc] int32 for a pool of B * nc + spare pages:
+    every logical chunk of every sequence gets a distinct page, in an order
+    drawn from the workload's seed.  Returns (table, n_pages)."""
+    n_pages = w.B * w.nc + spare
+    rng = np.random.default_rng(np.random.SeedSequence([w.seed, 5]))
+    table = rng.permutation(n_pages)[: w.B * w.nc].astype(np.int32).reshape(w.B, w.nc)
+    return table, n_pages
 
 
 def sample_rows(w: Workload, n: int | None = None) -> np.ndarray:

@@ -210,6 +210,36 @@ int hils_attn_decode_fixed_scratch(const hils_dims* dims, const void* q, const v
                                    int32_t* ids_out, float* scores_out, hils_stream_t stream);
 
 /*
+ * Chunk-paged KV cache -- [AIT-Tech] lists chunk-unit KV paging among what
+ * the implementation needs (its limits section counts it as engineering cost
+ * of deployment).  Here each page holds one chunk (C = 64 tokens) of all kv
+ * heads of one sequence, taken from a pool; a page table maps every
+ * sequence's logical chunks to pages.
+ *   k_pages, v_pages  [n_pages, Hkv, C, d] dtype (16-byte aligned)
+ *   page_table        device int32 [B, seqlen/C] (dims.seqlen is the
+ *                     capacity in tokens): page of logical chunk c of
+ *                     sequence b; only the entries of chunks the call reads
+ *                     are looked at
+ *   n_pages           pool size, >= 1
+ * All other arguments, layouts and results are those of
+ * hils_landmark_summary / hils_attn_decode: both compute exactly what the
+ * contiguous calls compute on the cache the table describes (same kernels,
+ * same arithmetic; only the addresses of the key and value rows differ).  A
+ * table entry outside [0, n_pages) is recorded as HILS_ERR_DEVICE_BOUNDS:
+ * the summary leaves that chunk's k', b' unwritten; the decode step leaves
+ * that chunk out of every query's fusion.  NULL page_table or n_pages < 1:
+ * HILS_ERR_INVALID_ARGUMENT.
+ */
+int hils_landmark_summary_paged(const hils_dims* dims, const void* k_pages, const int32_t* page_table,
+                                int64_t n_pages, const void* lq, int64_t chunk_begin, int64_t chunk_end,
+                                float* kprime, float* bprime, void* kprime_mma, hils_stream_t stream);
+int hils_attn_decode_paged(const hils_dims* dims, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* page_table, int64_t n_pages, const float* kprime,
+                           const float* bprime, const void* kprime_mma, const int32_t* seqlens, void* o,
+                           int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                           hils_stream_t stream);
+
+/*
  * Synchronises `stream`, copies the device status word of the current device
  * into *host_status (HILS_OK or a HILS_ERR_DEVICE_* code recorded by a kernel
  * since the last call) and clears it.  Returns HILS_ERR_CUDA if the

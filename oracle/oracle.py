@@ -189,3 +189,18 @@ class Oracle:
         B, Hq, d = q.shape
         return dict(ids=ids.reshape(B, Hq, -1), sel=sel.reshape(B, Hq, -1), gap=gap.reshape(B, Hq),
                     O=O.reshape(B, Hq, d), lse_own=lse.reshape(B, Hq), rows=rows)
+
+
+def gather_pages(pages: np.ndarray, table: np.ndarray) -> np.ndarray:
+    """The contiguous cache [B, Hkv, nc*C, d] that a chunk-paged pool
+    [n_pages, Hkv, C, d] and a page table [B, nc] describe: logical chunk c of
+    sequence b is page table[b, c] (aitrends.kr article, section "기술 상세":
+    chunk-unit KV paging).  Every paged call is defined as the contiguous call
+    on this cache."""
+    B, nc = table.shape
+    n_pages, H, C, d = pages.shape
+    out = np.empty((B, H, nc * C, d), dtype=pages.dtype)
+    for b in range(B):
+        for c in range(nc):
+            out[b, :, c * C:(c + 1) * C, :] = pages[int(table[b, c])]
+    return out
