@@ -64,6 +64,7 @@ class Workload:
     kind: str           # "prefill", "decode" or "prefill+decode"
     sample_rows: int    # rows the oracle checks (0 = all rows)
     paged: bool = False  # decode: the KV cache in chunk pages (page_table)
+    window: int = 0      # local window in tokens (0: the own chunk alone)
 
     @property
     def G(self) -> int:
@@ -99,11 +100,12 @@ WORKLOAD_ORDER = list(WORKLOADS)
 
 
 def custom(name="custom", *, B=1, Hq=1, Hkv=1, d=64, N=1024, C=64, K=3, seed=0,
-           dtype="bf16", needles=0, needle_mode="none", kind="prefill", sample_rows=0) -> Workload:
+           dtype="bf16", needles=0, needle_mode="none", kind="prefill", sample_rows=0, window=0) -> Workload:
     """A workload with arbitrary sizes (used for small parity cases)."""
     if needles == 0:
         needle_mode = "none"
-    return Workload(name, B, Hq, Hkv, d, N, C, K, seed, dtype, needles, needle_mode, kind, sample_rows)
+    return Workload(name, B, Hq, Hkv, d, N, C, K, seed, dtype, needles, needle_mode, kind, sample_rows,
+                    window=window)
 
 
 def round_bf16_bits(x: np.ndarray) -> np.ndarray:

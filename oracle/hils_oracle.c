@@ -36,8 +36,14 @@
  *   - candidates of a query at position i are the chunks c < floor(i/C)
  *     (fully past); the query's own chunk is always attended under the
  *     causal mask and enters the fusion with its exact log-sum-exp as score;
+ *   - with a local window of W tokens (W a multiple of C; [AIT-Tech] gives a
+ *     sliding window of 512) the window is chunk-aligned: the own chunk o
+ *     and the W/C - 1 chunks before it, keys max(0, (o - W/C + 1) C) .. i.
+ *     The window is one fusion branch scored by its exact log-sum-exp (it
+ *     replaces the own-chunk branch), and the candidates are the chunks
+ *     before it, c < o - W/C + 1.  W = 0 or W = C is the own chunk alone;
  *   - the fusion softmax runs over the selected chunks and the own chunk
- *     only;
+ *     (the window) only;
  *   - query head hq reads kv head floor(hq / G);
  *   - top-K ties: the lower chunk id wins; fewer than K candidates: keep
  *     them all, pad the id list with -1; ids are reported in ascending order.
@@ -60,7 +66,17 @@
 
 typedef struct hils_oracle_dims {
   int64_t B, Hq, Hkv, N, d, C, K;
+  int64_t W;   /* local window in tokens (0 or C: the own chunk only) */
 } hils_oracle_dims;
+
+/* chunks in the local window, own chunk included */
+static int64_t window_chunks(const hils_oracle_dims* D) { return D->W > D->C ? D->W / D->C : 1; }
+
+/* candidates of a query at position i: the chunks before its window */
+static int64_t n_candidates(const hils_oracle_dims* D, int64_t i) {
+  const int64_t n = i / D->C - (window_chunks(D) - 1);
+  return n > 0 ? n : 0;
+}
 
 static double dot_fd(const float* a, const float* b, int64_t d) {
   double s = 0.0;
@@ -130,7 +146,7 @@ void hils_oracle_scores(const hils_oracle_dims* D, const double* kp, const doubl
 #pragma omp parallel for schedule(dynamic, 16)
   for (int64_t r = 0; r < n_rows; ++r) {
     const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
-    const int64_t own = rpos[r] / D->C;
+    const int64_t own = n_candidates(D, rpos[r]);   /* scores exist for c < own */
     const float* q = qrows + r * d;
     for (int64_t c = 0; c < nc; ++c) {
       out[r * nc + c] = (c < own) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]
@@ -171,7 +187,7 @@ void hils_oracle_select(const hils_oracle_dims* D, const double* kp, const doubl
 #pragma omp parallel for schedule(dynamic, 16)
   for (int64_t r = 0; r < n_rows; ++r) {
     const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
-    const int64_t n_cand = rpos[r] / D->C;   /* candidates: the fully-past chunks 0 .. n_cand-1 */
+    const int64_t n_cand = n_candidates(D, rpos[r]);   /* candidates: the chunks 0 .. n_cand-1 */
     const float* q = qrows + r * d;
     scored_chunk* cand = (scored_chunk*)malloc(sizeof(scored_chunk) * (size_t)(n_cand + 1));
     for (int64_t c = 0; c < n_cand; ++c) {
@@ -243,7 +259,7 @@ void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* 
     const int64_t nsel = ids_stride;
     double* u = (double*)malloc(sizeof(double) * (size_t)(nsel + 1));
     double* oc = (double*)malloc(sizeof(double) * (size_t)((nsel + 1) * d));
-    double* s = (double*)malloc(sizeof(double) * (size_t)C);
+    double* s = (double*)malloc(sizeof(double) * (size_t)(C * window_chunks(D)));
     int64_t m_used = 0;
     for (int64_t t = 0; t < nsel; ++t) {
       const int64_t c = ids[r * ids_stride + t];
@@ -253,7 +269,10 @@ void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* 
                                     : lse;
       ++m_used;
     }
-    const double lo = attend_keys(q, Kbh, Vbh, own * C, i + 1, d, tau, s, oc + m_used * d);
+    /* the own chunk, or with a window the W/C chunks ending at it (causal) */
+    int64_t w0 = (own - (window_chunks(D) - 1)) * C;
+    if (w0 < 0) w0 = 0;
+    const double lo = attend_keys(q, Kbh, Vbh, w0, i + 1, d, tau, s, oc + m_used * d);
     u[m_used] = lo;
     if (lse_own) lse_own[r] = lo;
     ++m_used;

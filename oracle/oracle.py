@@ -24,7 +24,7 @@ _lib = None
 
 
 class _Dims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int64) for n in ("B", "Hq", "Hkv", "N", "d", "C", "K")]
+    _fields_ = [(n, ctypes.c_int64) for n in ("B", "Hq", "Hkv", "N", "d", "C", "K", "W")]
 
 
 def _lib_path() -> str:
@@ -64,8 +64,8 @@ def max_threads() -> int:
     return int(_load().hils_oracle_max_threads())
 
 
-def _dims(B, Hq, Hkv, N, d, C, K):
-    return _Dims(B, Hq, Hkv, N, d, C, K)
+def _dims(B, Hq, Hkv, N, d, C, K, W=0):
+    return _Dims(B, Hq, Hkv, N, d, C, K, W)
 
 
 def _p(a: np.ndarray | None):
@@ -111,16 +111,17 @@ class Rows:
 class Oracle:
     """fp64 oracle bound to one set of sizes (K/V arrays have N token slots)."""
 
-    def __init__(self, B, Hq, Hkv, N, d, C, K):
-        assert Hq % Hkv == 0 and N % C == 0
-        self.B, self.Hq, self.Hkv, self.N, self.d, self.C, self.K = B, Hq, Hkv, N, d, C, K
+    def __init__(self, B, Hq, Hkv, N, d, C, K, W=0):
+        """W: local window in tokens, a multiple of C (0 or C: the own chunk alone)."""
+        assert Hq % Hkv == 0 and N % C == 0 and W % C == 0
+        self.B, self.Hq, self.Hkv, self.N, self.d, self.C, self.K, self.W = B, Hq, Hkv, N, d, C, K, W
         self.nc = N // C
-        self._d = _dims(B, Hq, Hkv, N, d, C, K)
+        self._d = _dims(B, Hq, Hkv, N, d, C, K, W)
         self._lib = _load()
 
     @staticmethod
     def for_workload(w, K=None) -> "Oracle":
-        return Oracle(w.B, w.Hq, w.Hkv, w.N, w.d, w.C, w.K if K is None else K)
+        return Oracle(w.B, w.Hq, w.Hkv, w.N, w.d, w.C, w.K if K is None else K, w.window)
 
     def summary(self, Kt, LQ, chunk_begin=0, chunk_end=None):
         """Compressed keys kp [B,Hkv,nc,d] and entropy biases bp [B,Hkv,nc]."""

@@ -328,3 +328,52 @@ def test_partial_summary_range():
     kp2, bp2 = o.summary(K, LQ, 3, 5)
     assert np.array_equal(kp2[:, :, 3:5], kp[:, :, 3:5]) and np.array_equal(bp2[:, :, 3:5], bp[:, :, 3:5])
     assert not kp2[:, :, :3].any() and not kp2[:, :, 5:].any()
+
+
+@pytest.mark.parametrize("W", [64, 128, 320, 512])
+def test_pin_window_plus_all_exact_chunks_is_dense_attention(W):
+    """Local window (aitrends.kr article, section "기술 상세": sliding window
+    512; read as chunk-aligned, the own chunk and the W/C - 1 chunks before it,
+    one fusion branch scored by its exact log-sum-exp).  Keeping every
+    candidate (the chunks before the window) with exact chunk log-sum-exps
+    must reproduce dense causal attention for any W: window and candidates
+    cover every past key exactly once."""
+    rng = np.random.default_rng(31 + W)
+    B, Hq, Hkv, N, d, C = 1, 2, 1, 768, 16, 64
+    nc = N // C
+    Q, K, V = rand(rng, B, Hq, N, d), rand(rng, B, Hkv, N, d), rand(rng, B, Hkv, N, d)
+    LQ = rand(rng, B, Hkv, nc, d)
+    o = Oracle(B, Hq, Hkv, N, d, C, nc, W)
+    kp, bp = o.summary(K, LQ)
+    rows = Rows.from_prefill(Q, np.arange(B * Hq * N))
+    ids, _, _ = o.select(kp, bp, rows)
+    wc = W // C
+    for r in range(len(rows)):
+        # candidates: the chunks before the window, all kept (K = nc)
+        n_cand = max(0, rows.pos[r] // C - (wc - 1))
+        assert np.array_equal(ids[r, :n_cand], np.arange(n_cand))
+        assert np.all(ids[r, n_cand:] == -1)
+    O, lse_w = o.attend(K, V, kp, bp, rows, ids, score_mode=1)
+    assert np.max(np.abs(O - dense_causal(Q, K, V, Hq // Hkv).reshape(-1, d))) < 1e-12
+    # the window branch's score is the exact log-sum-exp over its keys
+    for r in (0, 100, 700, 767 + 768):
+        i, h = rows.pos[r], rows.hq[r] // (Hq // Hkv)
+        w0 = max(0, (i // C - (wc - 1)) * C)
+        s = (K[0, h, w0:i + 1].astype(np.float64) @ Q[0, rows.hq[r], i].astype(np.float64)) / math.sqrt(d)
+        assert abs(lse_w[r] - logsumexp(s)) < 1e-12
+
+
+def test_pin_window_over_the_whole_sequence_is_dense_attention():
+    """A window that covers every past key leaves no candidates: the output is
+    dense causal attention whatever the summaries and K."""
+    rng = np.random.default_rng(37)
+    B, H, N, d, C = 1, 1, 512, 16, 64
+    Q, K, V = rand(rng, B, H, N, d), rand(rng, B, H, N, d), rand(rng, B, H, N, d)
+    LQ = rand(rng, B, H, N // C, d)
+    o = Oracle(B, H, H, N, d, C, 3, N)
+    kp, bp = o.summary(K, LQ)
+    rows = Rows.from_prefill(Q, np.arange(N))
+    ids, _, _ = o.select(kp, bp, rows)
+    assert np.all(ids == -1)
+    O, _ = o.attend(K, V, kp, bp, rows, ids, score_mode=0)
+    assert np.max(np.abs(O - dense_causal(Q, K, V, 1).reshape(-1, d))) < 1e-12

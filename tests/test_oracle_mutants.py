@@ -21,12 +21,17 @@ MUTANTS = {
                             "(score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d)"),
     "fusion_surrogate_unscaled": ("(score_mode == 0) ? tau * dot_fdd(", "(score_mode == 0) ? dot_fdd("),
     "compressed_key_wrong_index": ("out[t] += p * (double)kc[j * d + t];", "out[t] += p * (double)kc[t * d + j % d];"),
-    "causal_mask_off_by_one": ("own * C, i + 1, d, tau", "own * C, i, d, tau"),
+    "causal_mask_off_by_one": ("w0, i + 1, d, tau", "w0, i, d, tau"),
     "kv_head_mapping_modulo": ("const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;\n    const int64_t i = rpos[r]",
                                "const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] % D->Hkv;\n    const int64_t i = rpos[r]"),
     "select_ascending": ("if (a->s > b->s) return -1;\n  if (a->s < b->s) return 1;",
                          "if (a->s < b->s) return -1;\n  if (a->s > b->s) return 1;"),
-    "own_chunk_is_candidate": ("const int64_t n_cand = rpos[r] / D->C;", "const int64_t n_cand = rpos[r] / D->C + 1;"),
+    "own_chunk_is_candidate": ("const int64_t n_cand = n_candidates(D, rpos[r]);",
+                               "const int64_t n_cand = n_candidates(D, rpos[r]) + 1;"),
+    "window_starts_a_chunk_late": ("int64_t w0 = (own - (window_chunks(D) - 1)) * C;",
+                                   "int64_t w0 = (own - (window_chunks(D) - 2)) * C;"),
+    "window_candidates_overlap": ("const int64_t n = i / D->C - (window_chunks(D) - 1);",
+                                  "const int64_t n = i / D->C - (window_chunks(D) - 2);"),
     "fusion_uniform_weights": ("const double w = exp(u[t] - M) / Z;", "const double w = 1.0 / (double)m_used;"),
     "fusion_drops_own_chunk": ("u[m_used] = lo;", "u[m_used] = -INFINITY;"),
 }
