@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(128)
 prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                     const int32_t* __restrict__ ids, const float* __restrict__ scores, T* __restrict__ o,
                     float* __restrict__ lse_own, int64_t n_tok, int Hq, int G, int Hkv, int K, float tau,
-                    int64_t n_rows) {
+                    int64_t n_rows, int wm1) {
   using L = RowLayout<T, D>;
   constexpr int E = L::E, LPK = L::LPK;
   const int lane = threadIdx.x & 31;
@@ -95,13 +95,22 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
   const int64_t own = i / kChunk;
 
   float oc[E];
-  const float lo = attend_range<T, D>(qv, kbh, vbh, own * kChunk, i + 1, tau, oc);
+  // the local window: the own chunk (causal) and the wm1 chunks before it,
+  // each fused at its exact log-sum-exp, which together is one branch over
+  // the window's keys at the window's log-sum-exp lo
+  float lo = attend_range<T, D>(qv, kbh, vbh, own * kChunk, i + 1, tau, oc);
   Fusion<E> f;
   f.init(lo, oc);
+  for (int64_t c = own - 1; c >= 0 && c >= own - wm1; --c) {
+    const float lc = attend_range<T, D>(qv, kbh, vbh, c * kChunk, (c + 1) * kChunk, tau, oc);
+    f.add(lc, oc);
+    lo = fmaxf(lo, lc) + log1pf(expf(-fabsf(lo - lc)));
+  }
+  const int64_t n_cand = n_candidates(i, wm1);
   for (int t = 0; t < K; ++t) {
     const int32_t c = __ldg(ids + row * K + t);
     if (c < 0) continue;
-    if (c >= own) {
+    if (c >= n_cand) {
       if (lane == 0) record_error(HILS_ERR_DEVICE_BOUNDS);
       continue;
     }

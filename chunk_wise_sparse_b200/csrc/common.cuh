@@ -21,6 +21,14 @@ __device__ int32_t g_status;
 
 __device__ __forceinline__ void record_error(int32_t code) { atomicCAS(&g_status, 0, code); }
 
+// Candidates of a query at position i: the chunks before its local window,
+// which spans the own chunk and the wm1 chunks before it (wm1 = 0: the own
+// chunk alone).
+__host__ __device__ __forceinline__ int64_t n_candidates(int64_t i, int wm1) {
+  const int64_t n = i / kChunk - wm1;
+  return n > 0 ? n : 0;
+}
+
 // Where the keys / values of chunk c of (b, h) live.  Contiguous cache
 // (table == nullptr): [B, Hkv, n_tok, d], chunk c at token c*C.  Chunk-paged
 // cache: a pool [n_pages, Hkv, C, d] and table[b * nc + c] = the page of

@@ -3,9 +3,10 @@
 // HiLS paper, aitrends.kr article, section "방법론" (Methodology) for the
 // scoring and top-K, and ai-papers.net article, section "実験結果と性能",
 // for the per-token decode with sparse KV access.  The query of (b, hq) sits
-// at position t = seqlens[b]-1; its candidates are the fully-past chunks
-// c < floor(t/C); its own chunk (keys floor(t/C)*C .. t) is attended under
-// the causal mask.
+// at position t = seqlens[b]-1.  Its local window is the own chunk
+// o = floor(t/C) and the wm1 chunks before it (keys max(0, (o - wm1) C) .. t,
+// causal), one fusion branch whose score is its exact log-sum-exp; its top-K
+// candidates are the chunks before the window, c < o - wm1.
 //
 // Four short kernels, all HBM- or latency-bound:
 //   D1 scores   : s^ for every candidate chunk of every query head; one warp
@@ -17,9 +18,11 @@
 //                 stable compaction in ascending chunk id; ties among equal
 //                 scores go to the lower ids.
 //   D3 partials : per (batch, kv head), each distinct chunk kept by any of the
-//                 G query heads (plus the own chunk) is read once and attended
-//                 by every head that kept it; one partial (score, output) per
-//                 (row, slot).
+//                 G query heads (plus each chunk of the local window) is read
+//                 once and attended by every head that kept it; one partial
+//                 (score, output) per (row, slot).  A window chunk's score is
+//                 its exact log-sum-exp, so the window chunks' partials fuse
+//                 to the one window branch.
 //   D4 combine  : softmax over the chunk scores fuses the partials.
 #pragma once
 #include "attend_simt.cuh"
@@ -30,20 +33,20 @@ struct DecodeWs {
   float* scores;      // [B*Hq, nc]
   int32_t* sel_ids;   // [B*Hq, K]
   float* sel_scores;  // [B*Hq, K]
-  float* part_u;      // [B*Hq, K+1]
-  float* part_o;      // [B*Hq, K+1, D]
+  float* part_u;      // [B*Hq, K+WC]: K selected slots, then the WC window chunks
+  float* part_o;      // [B*Hq, K+WC, D]
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline size_t decode_ws_layout(int64_t rows, int64_t nc, int K, int D, char* base, DecodeWs* ws) {
+inline size_t decode_ws_layout(int64_t rows, int64_t nc, int K, int WC, int D, char* base, DecodeWs* ws) {
   size_t off = 0;
   auto take = [&](size_t bytes) { char* p = base ? base + off : nullptr; off += align256(bytes); return p; };
   char* a = take(sizeof(float) * rows * nc);
   char* b = take(sizeof(int32_t) * rows * K);
   char* c = take(sizeof(float) * rows * K);
-  char* d = take(sizeof(float) * rows * (K + 1));
-  char* e = take(sizeof(float) * rows * (K + 1) * D);
+  char* d = take(sizeof(float) * rows * (K + WC));
+  char* e = take(sizeof(float) * rows * (K + WC) * D);
   if (ws) {
     ws->scores = reinterpret_cast<float*>(a);
     ws->sel_ids = reinterpret_cast<int32_t*>(b);
@@ -54,7 +57,7 @@ inline size_t decode_ws_layout(int64_t rows, int64_t nc, int K, int D, char* bas
   return off;
 }
 
-// Number of candidate chunks of batch b (own chunk index); -1 if seqlens[b] is invalid.
+// Own chunk of batch b's query; -1 if seqlens[b] is invalid.
 __device__ __forceinline__ int64_t decode_own_chunk(const int32_t* seqlens, int b, int64_t cap) {
   const int32_t s = __ldg(seqlens + b);
   if (s < 1 || int64_t(s) > cap) return -1;
@@ -71,7 +74,7 @@ template <typename T, int D, bool MMA_OPERAND>
 __global__ void __launch_bounds__(kDecChunksPerCta)
 decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, const float* __restrict__ bp,
                      const __nv_bfloat16* __restrict__ kmma, const int32_t* __restrict__ seqlens, int64_t cap,
-                     int64_t nc, int Hq, int G, int Hkv, float tau, float* __restrict__ ws_scores) {
+                     int64_t nc, int Hq, int G, int Hkv, float tau, float* __restrict__ ws_scores, int wm1) {
   using KT = typename std::conditional<MMA_OPERAND, __nv_bfloat16, float>::type;
   constexpr int E = Vec16<KT>::E;                   // elements per 16-byte load
   constexpr int RS = MMA_OPERAND ? D + kExt : D;    // row stride of the k' rows
@@ -91,7 +94,7 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
   }
   __syncthreads();
   const int64_t c = int64_t(blockIdx.x) * kDecChunksPerCta + threadIdx.x;
-  if (c >= own) return;
+  if (c >= own - wm1) return;
   const KT* row = (MMA_OPERAND ? reinterpret_cast<const KT*>(kmma) : reinterpret_cast<const KT*>(kp)) +
                   (int64_t(bh) * nc + c) * RS;
   float bias;
@@ -153,12 +156,13 @@ __device__ __forceinline__ int block_exclusive_scan256(int x, int* warp_tot, int
 
 __global__ void __launch_bounds__(256)
 decode_topk_kernel(const float* __restrict__ ws_scores, const int32_t* __restrict__ seqlens, int64_t cap,
-                   int64_t nc, int Hq, int K, int32_t* __restrict__ sel_ids, float* __restrict__ sel_scores) {
+                   int64_t nc, int Hq, int K, int32_t* __restrict__ sel_ids, float* __restrict__ sel_scores,
+                   int wm1) {
   __shared__ uint32_t hist[256];
   __shared__ int warp_tot[8];
   __shared__ uint32_t s_digit, s_above;
   const int row = blockIdx.x, b = row / Hq, tid = threadIdx.x;
-  int64_t n = decode_own_chunk(seqlens, b, cap);
+  int64_t n = decode_own_chunk(seqlens, b, cap) - wm1;   // candidates
   if (n < 0) n = 0;
   const float* sc = ws_scores + int64_t(row) * nc;
   int32_t* oid = sel_ids + int64_t(row) * K;
@@ -234,8 +238,8 @@ decode_topk_kernel(const float* __restrict__ ws_scores, const int32_t* __restric
 
 // D3, grouped by kv head: the G query heads of a kv head select overlapping
 // chunk sets, so each distinct chunk is read once and attended by all heads
-// that kept it.  One single-warp CTA per candidate slot (g, k) of the
-// (b, kv head)'s G x K selections, plus one for the own chunk.  A slot whose
+// that kept it.  One CTA per candidate slot (g, k) of the (b, kv head)'s
+// G x K selections, plus one per chunk of the local window.  A slot whose
 // chunk already appears for an earlier head is skipped; otherwise the warp
 // finds the heads that kept the chunk (binary search in their ascending id
 // lists, one lane per head), brings the chunk's 64 key and value rows into
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(128)
 decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                             const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int G, int Hkv, int K,
                             float tau, const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
-                            float* __restrict__ part_u, float* __restrict__ part_o, PagedKv pk) {
+                            float* __restrict__ part_u, float* __restrict__ part_o, PagedKv pk, int wm1) {
   using U = DecUnion<T, D>;
   constexpr int EL = D / 32;                 // output dims per lane
   constexpr int EB = 16 / int(sizeof(T));    // elements per 16-byte block
@@ -304,20 +308,24 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t row0 = int64_t(b) * Hq + int64_t(h) * G;
-  const int pidx = blockIdx.x;   // candidate slot g * K + k, or G * K for the own chunk
+  const int PS = K + wm1 + 1;    // partial slots per row
+  // candidate slot g * K + k, or G * K + w for window chunk own - w
+  const int pidx = blockIdx.x;
   const int64_t own = decode_own_chunk(seqlens, b, cap);
-  if (own < 0) {
-    if (tid == 0 && pidx < G * K) part_u[(row0 + pidx / K) * (K + 1) + pidx % K] = -INFINITY;
-    if (tid < G && pidx == G * K) part_u[(row0 + tid) * (K + 1) + K] = -INFINITY;
+  if (own < 0 || (pidx >= G * K && own < pidx - G * K)) {
+    if (tid == 0 && pidx < G * K) part_u[(row0 + pidx / K) * PS + pidx % K] = -INFINITY;
+    if (tid < G && pidx >= G * K) part_u[(row0 + tid) * PS + K + (pidx - G * K)] = -INFINITY;
     return;
   }
+  const int64_t n_cand = own - wm1 > 0 ? own - wm1 : 0;
   for (int idx = tid; idx < G * K; idx += 128) sid[idx] = sel_ids[row0 * K + idx];
   __syncthreads();
   int64_t j0, j1;
-  if (pidx == G * K) {
-    j0 = own * kChunk;
-    j1 = int64_t(__ldg(seqlens + b));
-    if (tid < G) s_slot[tid] = K;
+  if (pidx >= G * K) {
+    const int w = pidx - G * K;
+    j0 = (own - w) * kChunk;
+    j1 = w == 0 ? int64_t(__ldg(seqlens + b)) : j0 + kChunk;
+    if (tid < G) s_slot[tid] = K + w;
     if (tid == 0) s_go = 1;
   } else {
     const int g = pidx / K, k = pidx % K;
@@ -325,7 +333,7 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
     j0 = int64_t(c) * kChunk;
     j1 = j0 + kChunk;
     if (warp == 0) {
-      const bool bad = c < 0 || c >= own;
+      const bool bad = c < 0 || c >= n_cand;
       int my_slot = -1;
       if (!bad && lane < G) {
         const int32_t* ids = sid + lane * K;
@@ -342,8 +350,8 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
       if (lane < G) s_slot[lane] = my_slot;
       if (lane == 0) {
         if (bad) {
-          part_u[(row0 + g) * (K + 1) + k] = -INFINITY;
-          if (c >= own) record_error(HILS_ERR_DEVICE_BOUNDS);
+          part_u[(row0 + g) * PS + k] = -INFINITY;
+          if (c >= n_cand) record_error(HILS_ERR_DEVICE_BOUNDS);
         }
         // an earlier head's CTA takes a chunk that head also kept
         s_go = !bad && !(mask & ((1u << g) - 1u));
@@ -360,7 +368,7 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
     s_off[1] = int(uint32_t(uint64_t(off) >> 32));
     if (off < 0) {
       for (int g = 0; g < G; ++g)
-        if (s_slot[g] >= 0) part_u[(row0 + g) * (K + 1) + s_slot[g]] = -INFINITY;
+        if (s_slot[g] >= 0) part_u[(row0 + g) * PS + s_slot[g]] = -INFINITY;
     }
   }
   __syncthreads();
@@ -431,11 +439,11 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
       }
     }
     const int64_t row = row0 + g;
-    float* po = part_o + (row * (K + 1) + slot) * D + lane * EL;
+    float* po = part_o + (row * PS + slot) * D + lane * EL;
     const float inv = 1.f / l;
 #pragma unroll
     for (int e = 0; e < EL; ++e) po[e] = o[e] * inv;
-    if (lane == 0) part_u[row * (K + 1) + slot] = slot == K ? m + logf(l) : sel_scores[row * K + slot];
+    if (lane == 0) part_u[row * PS + slot] = slot >= K ? m + logf(l) : sel_scores[row * K + slot];
   }
 }
 
@@ -445,25 +453,26 @@ decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict_
                       const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int K,
                       const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
                       T* __restrict__ o, int32_t* __restrict__ ids_out, float* __restrict__ scores_out,
-                      int64_t n_rows) {
+                      int64_t n_rows, int wm1) {
   constexpr int EL = D / 32;   // output elements per lane
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (row >= n_rows) return;
   const int b = int(row / Hq);
   const bool valid = decode_own_chunk(seqlens, b, cap) >= 0;
+  const int PS = K + wm1 + 1;
   float M = -INFINITY;
-  for (int s = 0; s <= K; ++s) M = fmaxf(M, part_u[row * (K + 1) + s]);
+  for (int s = 0; s < PS; ++s) M = fmaxf(M, part_u[row * PS + s]);
   float Z = 0.f, acc[EL];
 #pragma unroll
   for (int e = 0; e < EL; ++e) acc[e] = 0.f;
   if (valid) {
-    for (int s = 0; s <= K; ++s) {
-      const float u = part_u[row * (K + 1) + s];
+    for (int s = 0; s < PS; ++s) {
+      const float u = part_u[row * PS + s];
       if (u == -INFINITY) continue;
       const float w = expf(u - M);
       Z += w;
-      const float* po = part_o + (row * (K + 1) + s) * D + lane * EL;
+      const float* po = part_o + (row * PS + s) * D + lane * EL;
 #pragma unroll
       for (int e = 0; e < EL; ++e) acc[e] += w * po[e];
     }

@@ -29,7 +29,9 @@ int check_dims(const hils_dims* d) {
   if (d == nullptr) return HILS_ERR_INVALID_ARGUMENT;
   if (d->batch < 1 || d->heads_q < 1 || d->heads_kv < 1 || d->heads_q % d->heads_kv != 0)
     return HILS_ERR_INVALID_ARGUMENT;
-  if (d->seqlen < 1 || d->chunk < 1 || d->reserved != 0) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->seqlen < 1 || d->chunk < 1) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->window < 0 || d->window % kChunk != 0) return HILS_ERR_INVALID_ARGUMENT;
+  if (d->window > 16 * kChunk) return HILS_ERR_UNSUPPORTED;
   if (d->dtype != HILS_BF16 && d->dtype != HILS_FP32) return HILS_ERR_INVALID_ARGUMENT;
   if (d->chunk != kChunk) return HILS_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return HILS_ERR_UNSUPPORTED;
@@ -38,6 +40,9 @@ int check_dims(const hils_dims* d) {
   if (d->seqlen > (int64_t(1) << 31)) return HILS_ERR_UNSUPPORTED;
   return HILS_OK;
 }
+
+// chunks of the local window before the own chunk
+inline int window_wm1(const hils_dims* d) { return d->window > kChunk ? d->window / kChunk - 1 : 0; }
 
 inline int launched(int n) {
   g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed);
@@ -133,6 +138,7 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
   p.n_row_tiles = int((N + P - 1) / P);
   p.stages = stages;
   p.cap = cap;
+  p.wm1 = window_wm1(d);
   p.tau = 1.f / sqrtf(float(D));
   p.ids = ids;
   p.scores = scores;
@@ -153,7 +159,9 @@ struct CcPlan {
 bool cc_supported(const hils_dims* d) {
   const int64_t G = d->heads_q / d->heads_kv;
   const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
-  return d->dtype == HILS_BF16 && G <= 16 && (G & (G - 1)) == 0 && G * d->seqlen <= (int64_t(1) << 25) &&
+  // a local window beyond the own chunk runs on the CUDA-core prefill
+  return d->dtype == HILS_BF16 && window_wm1(d) == 0 && G <= 16 && (G & (G - 1)) == 0 &&
+         G * d->seqlen <= (int64_t(1) << 25) &&
          rows * d->topk < (int64_t(1) << 31);
 }
 
@@ -305,7 +313,7 @@ int launch_select_simt(const hils_dims* d, const void* q, const float* kp, const
   dim3 grid(unsigned((d->seqlen + kSelRows - 1) / kSelRows), unsigned(d->batch * d->heads_q));
   fn<<<grid, kSelRows, smem, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma),
                                   d->seqlen, d->seqlen / kChunk, d->heads_q, d->heads_q / d->heads_kv,
-                                  d->heads_kv, d->topk, 1.f / sqrtf(float(D)), ids, scores);
+                                  d->heads_kv, d->topk, 1.f / sqrtf(float(D)), ids, scores, window_wm1(d));
   return launched(1);
 }
 
@@ -317,7 +325,7 @@ int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const 
   prefill_simt_kernel<T, D><<<dim3(unsigned(blocks)), 128, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ids, scores,
       static_cast<T*>(o), lse, d->seqlen, d->heads_q, d->heads_q / d->heads_kv, d->heads_kv, d->topk,
-      1.f / sqrtf(float(D)), rows);
+      1.f / sqrtf(float(D)), rows, window_wm1(d));
   return launched(1);
 }
 
@@ -330,25 +338,26 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   const int G = d->heads_q / d->heads_kv, K = d->topk;
   const float tau = 1.f / sqrtf(float(D));
   DecodeWs ws;
-  decode_ws_layout(rows, nc, K, D, static_cast<char*>(ws_ptr), &ws);
+  const int wm1 = window_wm1(d);
+  decode_ws_layout(rows, nc, K, wm1 + 1, D, static_cast<char*>(ws_ptr), &ws);
   const size_t smem1 = sizeof(float) * size_t(G) * D;
   constexpr auto k1 = decode_scores_kernel<T, D, BF>;
   if (smem1 > 48 * 1024 && set_smem_max<k1>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
   k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
-                            d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores);
+                            d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores, wm1);
   decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
-                                                      ws.sel_scores);
+                                                      ws.sel_scores, wm1);
   const size_t smem3 = DecUnion<T, D>::smem(G, K);
   constexpr auto k3 = decode_partial_union_kernel<T, D>;
   if (smem3 > 48 * 1024 && set_smem_max<k3>() != cudaSuccess) return HILS_ERR_CUDA;
-  const dim3 g3(unsigned(G * K + 1), unsigned(d->batch * d->heads_kv));
+  const dim3 g3(unsigned(G * K + wm1 + 1), unsigned(d->batch * d->heads_kv));
   k3<<<g3, 128, smem3, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
-      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, pk);
+      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, pk, wm1);
   decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(
       ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
-      ids_out, scores_out, rows);
+      ids_out, scores_out, rows, wm1);
   return launched(4);
 }
 
@@ -454,7 +463,8 @@ int hils_attn_prefill(const hils_dims* d, const void* q, const void* k, const vo
 
 size_t hils_decode_workspace_bytes(const hils_dims* d) {
   if (check_dims(d) != HILS_OK) return 0;
-  return decode_ws_layout(int64_t(d->batch) * d->heads_q, d->seqlen / kChunk, d->topk, d->head_dim, nullptr, nullptr);
+  return decode_ws_layout(int64_t(d->batch) * d->heads_q, d->seqlen / kChunk, d->topk, window_wm1(d) + 1,
+                          d->head_dim, nullptr, nullptr);
 }
 
 static int decode_entry(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,

@@ -32,7 +32,7 @@ template <typename T, int D, bool MMA_OPERAND>
 __global__ void __launch_bounds__(kSelRows)
 select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const float* __restrict__ bp,
                    const __nv_bfloat16* __restrict__ kmma, int64_t n_tok, int64_t nc, int Hq, int G,
-                   int Hkv, int K, float tau, int32_t* __restrict__ ids, float* __restrict__ scores) {
+                   int Hkv, int K, float tau, int32_t* __restrict__ ids, float* __restrict__ scores, int wm1) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* qT = reinterpret_cast<float*>(smem_raw);          // [D][128]
   float* kT = qT + D * kSelRows;                           // [D][32]
@@ -47,7 +47,7 @@ select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const 
   const int64_t i0 = int64_t(blockIdx.x) * kSelRows;
   const int64_t i = i0 + tid;
   const bool valid = i < n_tok;
-  const int64_t n_cand = valid ? i / kChunk : 0;
+  const int64_t n_cand = valid ? n_candidates(i, wm1) : 0;
 
   // stage q (transposed)
   for (int idx = tid; idx < kSelRows * D; idx += kSelRows) {
@@ -63,7 +63,7 @@ select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const 
   int count = 0;
   float thr = -INFINITY;
   const int64_t i_last = (i0 + kSelRows - 1 < n_tok - 1) ? i0 + kSelRows - 1 : n_tok - 1;
-  const int64_t c_end = i_last / kChunk;  // candidates of the last row of the tile
+  const int64_t c_end = n_candidates(i_last, wm1);  // candidates of the last row of the tile
 
   for (int64_t c0 = 0; c0 < c_end; c0 += kSelTile) {
     __syncthreads();

@@ -91,6 +91,7 @@ struct SelTcParams {
   int64_t n_tok, nc;
   int Hq, Hkv, G, K, P;  // P = 128 / G positions per tile
   int n_row_tiles, stages, cap;
+  int wm1;   // chunks of the local window before the own chunk
   float tau;
   int32_t* ids;
   float* scores;
@@ -145,7 +146,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int b = bh / p.Hkv, h = bh % p.Hkv;
   const int64_t pos0 = int64_t(tile) * p.P;
   const int64_t pos_end = (pos0 + p.P < p.n_tok) ? pos0 + p.P : p.n_tok;
-  const int64_t c_hi = (pos_end - 1) / kChunk;          // candidates of the tile's last row
+  const int64_t c_hi = n_candidates(pos_end - 1, p.wm1);   // candidates of the tile's last row
   const int n_tiles = int((c_hi + C::NT - 1) / C::NT);
   // K <= KCAP: when every row of the tile has at least 8 K candidates, a
   // first pass over the chunks splits each row's scores into disjoint groups
@@ -155,7 +156,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   // the same.  g: 128 from 128 K candidates on, else 32, 16 or 8 (the
   // largest that leaves K groups); smaller groups bound tighter but cost a
   // list insertion each, and on long rows a group of 128 is the cheaper.
-  const int64_t n_min = pos0 / kChunk;   // candidates of the tile's first row
+  const int64_t n_min = n_candidates(pos0, p.wm1);   // candidates of the tile's first row
   const int64_t kk = p.K;
   const int group = n_min >= 128 * kk ? 128 : n_min >= 32 * kk ? 32 : n_min >= 16 * kk ? 16 : n_min >= 8 * kk ? 8 : 0;
   const int n_pass = (KCAP > 0 && group > 0) ? 2 : 1;
@@ -249,7 +250,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int g = r / p.P;
     const int64_t pos = pos0 + r % p.P;
     const bool valid = pos < p.n_tok;
-    const int64_t n_cand = valid ? pos / kChunk : 0;
+    const int64_t n_cand = valid ? n_candidates(pos, p.wm1) : 0;
     const int K = p.K;
     const float tau = p.tau;
     const uint64_t ntau2 = pack2(-tau);

@@ -36,7 +36,7 @@ class HilsError(RuntimeError):
 class hils_dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("chunk", ctypes.c_int32), ("topk", ctypes.c_int32),
-                ("seqlen", ctypes.c_int64), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("seqlen", ctypes.c_int64), ("dtype", ctypes.c_int32), ("window", ctypes.c_int32)]
 
 
 _lib = None
@@ -98,16 +98,18 @@ def _check(call, rc):
         raise HilsError(call, rc)
 
 
-def make_dims(batch, heads_q, heads_kv, head_dim, seqlen, topk, dtype, chunk=CHUNK) -> hils_dims:
+def make_dims(batch, heads_q, heads_kv, head_dim, seqlen, topk, dtype, chunk=CHUNK, window=0) -> hils_dims:
+    """window: local window in tokens (0 = the own chunk alone; else a multiple
+    of the chunk, at most 16 chunks)."""
     if isinstance(dtype, torch.dtype):
         dtype = BF16 if dtype == torch.bfloat16 else FP32 if dtype == torch.float32 else -1
-    return hils_dims(batch, heads_q, heads_kv, head_dim, chunk, topk, seqlen, dtype, 0)
+    return hils_dims(batch, heads_q, heads_kv, head_dim, chunk, topk, seqlen, dtype, window)
 
 
-def dims_for(q, k, topk) -> hils_dims:
+def dims_for(q, k, topk, window=0) -> hils_dims:
     """Dims of a prefill from q [B,Hq,N,d] and k [B,Hkv,N,d]."""
     B, Hq, N, d = q.shape
-    return make_dims(B, Hq, k.shape[1], d, N, topk, q.dtype)
+    return make_dims(B, Hq, k.shape[1], d, N, topk, q.dtype, window=window)
 
 
 # ---------------------------------------------------------------------------
@@ -231,21 +233,22 @@ def landmark_summary(k, lq, topk=1, chunk_begin=0, chunk_end=None, out: Summary 
     return out
 
 
-def select(q, summ: Summary, heads_kv, topk, stream=None):
+def select(q, summ: Summary, heads_kv, topk, stream=None, window=0):
     B, Hq, N, d = q.shape
-    dims = make_dims(B, Hq, heads_kv, d, N, topk, q.dtype)
+    dims = make_dims(B, Hq, heads_kv, d, N, topk, q.dtype, window=window)
     ids = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device)
     scores = torch.empty((B, Hq, N, topk), dtype=torch.float32, device=q.device)
     hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
     return ids, scores
 
 
-def prefill(q, k, v, lq, topk, stream=None, return_all=False):
+def prefill(q, k, v, lq, topk, stream=None, return_all=False, window=0):
     """Full HiLS prefill: summary -> select -> sparse attention.  Returns O
-    (and, with return_all, the summary, ids, scores and lse_own)."""
-    dims = dims_for(q, k, topk)
+    (and, with return_all, the summary, ids, scores and the local branch's
+    log-sum-exp)."""
+    dims = dims_for(q, k, topk, window)
     summ = landmark_summary(k, lq, topk, stream=stream)
-    ids, scores = select(q, summ, k.shape[1], topk, stream)
+    ids, scores = select(q, summ, k.shape[1], topk, stream, window)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, prefill_workspace(dims, q.device), stream=stream)
@@ -254,11 +257,11 @@ def prefill(q, k, v, lq, topk, stream=None, return_all=False):
     return o
 
 
-def decode_step(q, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None):
+def decode_step(q, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None, window=0):
     """One decode step for q [B,Hq,d] against caches [B,Hkv,cap,d]."""
     B, Hq, d = q.shape
     Hkv, cap = k_cache.shape[1], k_cache.shape[2]
-    dims = make_dims(B, Hq, Hkv, d, cap, topk, q.dtype)
+    dims = make_dims(B, Hq, Hkv, d, cap, topk, q.dtype, window=window)
     if workspace is None:
         workspace = torch.empty((hils_decode_workspace_bytes(dims),), dtype=torch.uint8, device=q.device)
     o = torch.empty_like(q)

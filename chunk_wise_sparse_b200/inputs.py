@@ -86,6 +86,11 @@ WORKLOADS = {
     # the same decode step with the KV cache in chunk pages drawn in random order
     "decode-128k-b8-gqa4-d128-paged": Workload("decode-128k-b8-gqa4-d128-paged", 8, 32, 8, 128, 131072, 64, 32, 2,
                                                "bf16", 0, "none", "decode", 0, paged=True),
+    # the same steps with the 512-token local window beside the selected chunks
+    "prefill-32k-h16-d64-w512": Workload("prefill-32k-h16-d64-w512", 1, 16, 16, 64, 32768, 64, 16, 1,
+                                         "bf16", 32, "random", "prefill", 4096, window=512),
+    "decode-128k-b8-gqa4-d128-w512": Workload("decode-128k-b8-gqa4-d128-w512", 8, 32, 8, 128, 131072, 64, 32, 2,
+                                              "bf16", 0, "none", "decode", 0, window=512),
     "prefill-128k-gqa4-d128": Workload("prefill-128k-gqa4-d128", 1, 32, 8, 128, 131072, 64, 32, 3,
                                        "bf16", 64, "random", "prefill", 4096),
     "prefill-512k-h16-d64": Workload("prefill-512k-h16-d64", 1, 16, 16, 64, 524288, 64, 16, 4,

@@ -36,8 +36,10 @@
  *   streams (they keep no host state besides a launch counter).
  * - Row = (b, hq, i).  Its kv head is h = hq / G with G = heads_q/heads_kv
  *   (contiguous query-head groups share a kv head).  Its own chunk is
- *   floor(i/chunk); its candidate chunks are the fully-past ones,
- *   c < floor(i/chunk).  tau = 1/sqrt(head_dim).
+ *   o = floor(i/chunk); its local window is o and the W-1 chunks before it
+ *   (W = max(1, dims.window/chunk)), keys max(0, (o-W+1) chunk) .. i; its
+ *   candidate chunks are the ones before the window, c < o - W + 1.
+ *   tau = 1/sqrt(head_dim).
  */
 #ifndef HILS_H_
 #define HILS_H_
@@ -73,7 +75,13 @@ typedef struct hils_dims {
   int64_t seqlen;    /* prefill: N tokens; decode: KV-cache capacity in tokens.
                         Must be a positive multiple of chunk. */
   int32_t dtype;     /* HILS_BF16 (bf16 storage, fp32 accumulation) or HILS_FP32 */
-  int32_t reserved;  /* must be 0 */
+  int32_t window;    /* local window in tokens ([AIT-Tech]: a sliding window of
+                        512): 0 or chunk = the own chunk alone; else a multiple
+                        of chunk, at most 16 chunks.  Read chunk-aligned: the
+                        own chunk o and the window/C - 1 chunks before it, keys
+                        max(0, (o - window/C + 1) C) .. i, one fusion branch
+                        scored by its exact log-sum-exp; the top-K candidates
+                        are the chunks before the window. */
 } hils_dims;
 
 /*
@@ -107,7 +115,8 @@ size_t hils_kprime_mma_bytes(const hils_dims* dims);
 /*
  * Chunk scoring and top-K selection for every query row of a prefill --
  * [AIT-Meth]: s^_{i,c} = tau*<q_i, k'_c> + b'_c over the candidates
- * c < floor(i/C); keep the K largest.  Ties go to the lower chunk id.
+ * c < floor(i/C) - W + 1 (W = window chunks); keep the K largest.  Ties go to
+ * the lower chunk id.
  *   q          [B, Hq, seqlen, d] dtype
  *   kprime     fp32 [B,Hkv,nc,d]  (fp32 path; may be NULL for bf16)
  *   bprime     fp32 [B,Hkv,nc]    (fp32 path; may be NULL for bf16)
@@ -133,18 +142,20 @@ size_t hils_prefill_workspace_bytes(const hils_dims* dims);
 /*
  * Prefill sparse attention with hierarchical fusion -- [HP-Abs], [AIT-Meth],
  * [AIT-Gloss]: for each row and each kept chunk c, an intra-chunk softmax
- * over the chunk's C keys gives o_c and its log-sum-exp; the row's own chunk
- * is attended under the causal mask (keys floor(i/C)*C .. i) and enters the
- * fusion with its exact log-sum-exp lse_own as score; the fusion weights are
- * a softmax over {s^_c : c kept} U {lse_own}:
+ * over the chunk's C keys gives o_c and its log-sum-exp; the row's local
+ * window (keys max(0, (floor(i/C)-W+1) C) .. i, causal) is one branch that
+ * enters the fusion with its exact log-sum-exp lse_own as score; the fusion
+ * weights are a softmax over {s^_c : c kept} U {lse_own}:
  *     O_i = sum_c w_c o_c + w_own o_own.
+ * With a window beyond the own chunk the bf16 call runs on CUDA cores and
+ * needs no workspace.
  *   q, k, v   [B,Hq,N,d] / [B,Hkv,N,d] / [B,Hkv,N,d] dtype
  *   ids       [B,Hq,N,K] int32 from hils_select (-1 entries are skipped; an id
- *             outside [0, floor(i/C)) is recorded as HILS_ERR_DEVICE_BOUNDS
- *             and skipped)
+ *             outside the candidates [0, floor(i/C)-W+1) is recorded as
+ *             HILS_ERR_DEVICE_BOUNDS and skipped)
  *   scores    [B,Hq,N,K] fp32 from hils_select (required)
  *   o         [B,Hq,N,d] dtype out
- *   lse_own   [B,Hq,N] fp32 out (nullable)
+ *   lse_own   [B,Hq,N] fp32 out (nullable): log-sum-exp of the local window
  *   workspace device scratch of at least hils_prefill_workspace_bytes(dims)
  *             (may be NULL when that is 0); HILS_ERR_WORKSPACE_TOO_SMALL
  *             otherwise
@@ -160,8 +171,8 @@ size_t hils_decode_workspace_bytes(const hils_dims* dims);
  * One decode step -- [AIT-Meth] scoring and selection plus the fused sparse
  * attention of hils_attn_prefill, for one new query per (b, hq) at position
  * t_b = seqlens[b] - 1 whose key/value are already in the cache ([AIP-Perf]:
- * per-token decode with sparse KV access).  Chunks 0 .. floor(t_b/C)-1 must
- * have summaries.
+ * per-token decode with sparse KV access).  The candidate chunks
+ * 0 .. floor(t_b/C)-W must have summaries.
  *   dims.seqlen  KV-cache capacity in tokens
  *   q            [B, Hq, d] dtype
  *   k_cache, v_cache [B, Hkv, seqlen, d] dtype

@@ -35,7 +35,7 @@ def dims(**kw):
     base = dict(batch=1, heads_q=2, heads_kv=1, head_dim=64, seqlen=1024, topk=4, dtype=hils.BF16)
     base.update(kw)
     return hils.make_dims(base["batch"], base["heads_q"], base["heads_kv"], base["head_dim"], base["seqlen"],
-                          base["topk"], base["dtype"], base.get("chunk", 64))
+                          base["topk"], base["dtype"], base.get("chunk", 64), base.get("window", 0))
 
 
 def test_sizes(lib):
@@ -48,6 +48,7 @@ def test_sizes(lib):
 @pytest.mark.parametrize("kw,code", [
     (dict(chunk=32), 2), (dict(head_dim=96), 2), (dict(topk=0), 2), (dict(topk=65), 2),
     (dict(seqlen=1000), 1), (dict(heads_q=3, heads_kv=2), 1), (dict(dtype=7), 1), (dict(batch=0), 1),
+    (dict(window=100), 1), (dict(window=-64), 1), (dict(window=17 * 64), 2),
 ])
 def test_bad_dims_rejected_before_launch(lib, kw, code):
     d = dims(**kw)
@@ -84,6 +85,17 @@ def test_decode_rejects_more_than_32_query_heads_per_kv_head(lib):
     big = hils.hils_decode_workspace_bytes(d)
     assert lib.hils_attn_decode(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, p, big, None) == 2
     assert lib.hils_attn_decode_fixed_scratch(ctypes.byref(d), p, p, p, None, None, p, p, p, None, None, None) == 2
+
+
+def test_window_sizes(lib):
+    """A window beyond the own chunk runs the bf16 prefill on CUDA cores (no
+    workspace) and gives the decode one partial slot per window chunk."""
+    assert hils.hils_prefill_workspace_bytes(dims(window=64)) == hils.hils_prefill_workspace_bytes(dims())
+    assert hils.hils_prefill_workspace_bytes(dims(window=512)) == 0
+    d0, d8 = dims(window=0), dims(window=512)
+    assert hils.hils_decode_workspace_bytes(d8) > hils.hils_decode_workspace_bytes(d0)
+    d16 = dims(window=1024)
+    assert lib.hils_select(ctypes.byref(d16), None, None, None, None, None, None, None) == 1   # dims pass, q NULL
 
 
 def test_strerror(lib):

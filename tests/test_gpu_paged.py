@@ -30,6 +30,7 @@ def _pool(cache, table, n_pages):
 
 
 def _run(w, seqlens, spare=9, corrupt=None):
+    win = w.window
     inp = generate(w)
     q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
     table, n_pages = page_table(w, spare)
@@ -39,11 +40,11 @@ def _run(w, seqlens, spare=9, corrupt=None):
         table = table.copy()
         table[corrupt] = n_pages + 3
     tab = torch.from_numpy(table).cuda()
-    dims = hils.make_dims(w.B, w.Hq, w.Hkv, w.d, w.N, w.K, q.dtype)
+    dims = hils.make_dims(w.B, w.Hq, w.Hkv, w.d, w.N, w.K, q.dtype, window=win)
     seq = torch.from_numpy(seqlens.astype(np.int32)).cuda()
     # contiguous reference calls
     summ = hils.landmark_summary(k, lq, w.K)
-    o_c, ids_c, sc_c = hils.decode_step(q, k, v, summ, seq, w.K)
+    o_c, ids_c, sc_c = hils.decode_step(q, k, v, summ, seq, w.K, window=win)
     torch.cuda.synchronize()
     assert hils.hils_get_status() == 0
     # paged calls
@@ -65,9 +66,10 @@ def _run(w, seqlens, spare=9, corrupt=None):
                 o_c=o_c, ids_c=ids_c, sc_c=sc_c, o_p=o_p, ids_p=ids_p, sc_p=sc_p, status=status)
 
 
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("fp32", 64)])
-def test_paged_equals_contiguous_and_matches_the_oracle(dtype, d):
-    w = custom(f"paged-{dtype}-{d}", B=3, Hq=8, Hkv=2, d=d, N=16384, K=16, seed=71, dtype=dtype, kind="decode")
+@pytest.mark.parametrize("dtype,d,window", [("bf16", 128, 0), ("bf16", 64, 0), ("fp32", 64, 0), ("bf16", 128, 512)])
+def test_paged_equals_contiguous_and_matches_the_oracle(dtype, d, window):
+    w = custom(f"paged-{dtype}-{d}-w{window}", B=3, Hq=8, Hkv=2, d=d, N=16384, K=16, seed=71, dtype=dtype,
+               kind="decode", window=window)
     seqlens = np.array([16384, 16384 - 45, 700], np.int32)
     r = _run(w, seqlens)
     assert r["status"] == 0

@@ -63,7 +63,7 @@ def check_rows(w, inp, oracle, kp, bp, flat, ids_t, scores_t, o_t, lse_t=None, r
 def run_prefill_case(w):
     inp = generate(w)
     q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
-    o, aux = hils.prefill(q, k, v, lq, w.K, return_all=True)
+    o, aux = hils.prefill(q, k, v, lq, w.K, return_all=True, window=w.window)
     torch.cuda.synchronize()
     assert hils.hils_get_status() == 0
     oracle = Oracle.for_workload(w)
@@ -108,7 +108,7 @@ def test_prefill_full_size(name):
 
 def run_decode_check(w, inp, q_dev, kc, vc, summ, seqlens, oracle, kp, bp, q_f32):
     seq_dev = torch.from_numpy(seqlens.astype(np.int32)).cuda()
-    o, ids, scores = hils.decode_step(q_dev, kc, vc, summ, seq_dev, w.K)
+    o, ids, scores = hils.decode_step(q_dev, kc, vc, summ, seq_dev, w.K, window=w.window)
     torch.cuda.synchronize()
     assert hils.hils_get_status() == 0
     rows = Rows.from_decode(q_f32, seqlens)
