@@ -487,7 +487,7 @@ def run_decode(args, w, rank, world, local_rank):
         "config": dict(workload_config(w, world), l2="256 MiB buffer written between steps (L2 flush)"),
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                     "bytes": "selected-KV (union of kept chunks + own chunk per (b, kv head))",
+                     "bytes": "selected-KV (union of kept chunks + local window chunks per (b, kv head))",
                      "selected_kv_bytes": sel_bytes, "all_bytes_gbs": all_gbs},
         "gpu_launches": int(launches),
     }

@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "select_tc.cuh"
 #include "prefill_cc.cuh"
+#include "prefill_local.cuh"
 
 using namespace hils;
 
@@ -159,8 +160,7 @@ struct CcPlan {
 bool cc_supported(const hils_dims* d) {
   const int64_t G = d->heads_q / d->heads_kv;
   const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
-  // a local window beyond the own chunk runs on the CUDA-core prefill
-  return d->dtype == HILS_BF16 && window_wm1(d) == 0 && G <= 16 && (G & (G - 1)) == 0 &&
+  return d->dtype == HILS_BF16 && G <= 16 && (G & (G - 1)) == 0 &&
          G * d->seqlen <= (int64_t(1) << 25) &&
          rows * d->topk < (int64_t(1) << 31);
 }
@@ -174,6 +174,7 @@ CcPlan cc_plan(const hils_dims* d) {
   P.c.Hkv = d->heads_kv;
   P.c.G = int(G);
   P.c.K = d->topk;
+  P.c.wm1 = window_wm1(d);
   P.c.tau = 1.f / sqrtf(float(D));
   // window: the fp32 accumulators and bf16 queries of one window of one kv head
   // (G x W positions) stay within 64 MiB of L2
@@ -249,8 +250,6 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   if (cudaMemsetAsync(base + P.off_erow + sizeof(int32_t) * P.n_slots, 0, sizeof(int32_t) * kCcTileRows, st) !=
       cudaSuccess)
     return HILS_ERR_CUDA;
-  constexpr auto own_fn = cc_own_tc_kernel<D>;
-  if (set_smem_max<own_fn>() != cudaSuccess) return HILS_ERR_CUDA;
   CcOwnParams op;
   op.c = P.c;
   op.ids = ids;
@@ -260,8 +259,18 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   op.lse_own = lse;
   op.P = P.P;
   op.n_tiles = P.own_tiles;
-  own_fn<<<dim3(unsigned(P.own_tiles), unsigned(d->batch * d->heads_kv)), 128, CO::SMEM, st>>>(tq_tile, tk_own,
-                                                                                            tv_own, op);
+  const dim3 own_grid(unsigned(P.own_tiles), unsigned(d->batch * d->heads_kv));
+  if (P.c.wm1 == 0) {
+    constexpr auto own_fn = cc_own_tc_kernel<D>;
+    if (set_smem_max<own_fn>() != cudaSuccess) return HILS_ERR_CUDA;
+    own_fn<<<own_grid, 128, CO::SMEM, st>>>(tq_tile, tk_own, tv_own, op);
+  } else {
+    // the local window spans more than the own chunk
+    using CL = CcLocal<D>;
+    constexpr auto loc_fn = cc_local_tc_kernel<D>;
+    if (set_smem_max<loc_fn>() != cudaSuccess) return HILS_ERR_CUDA;
+    loc_fn<<<own_grid, CL::THREADS, CL::SMEM, st>>>(tq_tile, tk, tv, op);
+  }
   // two-level count when a CTA's rows stay in one window and the chunk histogram fits
   const size_t hist_bytes = sizeof(int32_t) * size_t(P.c.nc);
   if (d->seqlen % kCountRows == 0 && (int64_t(1) << P.c.win_shift) % kCountRows == 0 && hist_bytes <= 96 * 1024) {

@@ -37,7 +37,8 @@ namespace hils {
 struct CcDims {
   int64_t n_tok, nc;
   int Hq, Hkv, G, K;
-  int win_shift;   // window = pos >> win_shift
+  int wm1;         // chunks of the local window before the own chunk
+  int win_shift;   // L2 window of a row = pos >> win_shift
   int n_win;
   int64_t n_keys;  // B*Hkv*n_win*nc
   float tau;
@@ -359,7 +360,7 @@ cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, i
     const int32_t ci = __ldg(id0 + t);
     if (ci < 0) continue;
     const int64_t i = i0 + t / c.K;
-    if (ci >= i / kChunk) {
+    if (ci >= n_candidates(i, c.wm1)) {
       record_error(HILS_ERR_DEVICE_BOUNDS);
       continue;
     }
@@ -373,7 +374,7 @@ cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, i
   __syncthreads();
   for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
     const int32_t ci = __ldg(id0 + t);
-    if (ci < 0 || ci >= (i0 + t / c.K) / kChunk) continue;
+    if (ci < 0 || ci >= n_candidates(i0 + t / c.K, c.wm1)) continue;
     rk0[t] += hist[ci];
   }
 }
@@ -388,7 +389,7 @@ cc_count_direct_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ co
   if (ci < 0) return;
   const int64_t row = idx / c.K;
   const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
-  if (ci >= i / kChunk) {
+  if (ci >= n_candidates(i, c.wm1)) {
     record_error(HILS_ERR_DEVICE_BOUNDS);
     return;
   }
@@ -529,7 +530,7 @@ cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ rank
   if (ci < 0) return;
   const int64_t row = idx / c.K;
   const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
-  if (ci >= i / kChunk) return;   // out of range: recorded when counting
+  if (ci >= n_candidates(i, c.wm1)) return;   // out of range: recorded when counting
   const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
   const int64_t bh = b * c.Hkv + hq / c.G;
   const int64_t at = offsets[cc_key(c, bh, i, ci)] + __ldg(ranks + idx);

@@ -147,8 +147,6 @@ size_t hils_prefill_workspace_bytes(const hils_dims* dims);
  * enters the fusion with its exact log-sum-exp lse_own as score; the fusion
  * weights are a softmax over {s^_c : c kept} U {lse_own}:
  *     O_i = sum_c w_c o_c + w_own o_own.
- * With a window beyond the own chunk the bf16 call runs on CUDA cores and
- * needs no workspace.
  *   q, k, v   [B,Hq,N,d] / [B,Hkv,N,d] / [B,Hkv,N,d] dtype
  *   ids       [B,Hq,N,K] int32 from hils_select (-1 entries are skipped; an id
  *             outside the candidates [0, floor(i/C)-W+1) is recorded as

@@ -88,10 +88,10 @@ def test_decode_rejects_more_than_32_query_heads_per_kv_head(lib):
 
 
 def test_window_sizes(lib):
-    """A window beyond the own chunk runs the bf16 prefill on CUDA cores (no
-    workspace) and gives the decode one partial slot per window chunk."""
+    """The window leaves the prefill workspace unchanged and gives the decode
+    one partial slot per window chunk."""
     assert hils.hils_prefill_workspace_bytes(dims(window=64)) == hils.hils_prefill_workspace_bytes(dims())
-    assert hils.hils_prefill_workspace_bytes(dims(window=512)) == 0
+    assert hils.hils_prefill_workspace_bytes(dims(window=512)) == hils.hils_prefill_workspace_bytes(dims())
     d0, d8 = dims(window=0), dims(window=512)
     assert hils.hils_decode_workspace_bytes(d8) > hils.hils_decode_workspace_bytes(d0)
     d16 = dims(window=1024)

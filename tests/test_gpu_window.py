@@ -23,7 +23,13 @@ PREFILL = [
            needle_mode="random", window=512),
     custom("win128-bf16-d128-gqa4", B=1, Hq=8, Hkv=2, d=128, N=2112, K=8, seed=82, dtype="bf16", needles=2,
            needle_mode="random", window=128),
-    # CUDA-core selection (G = 3) under a window
+    # G = 1: 128-position tiles that span two chunks; ragged last tile
+    custom("win192-bf16-g1-ragged", B=2, Hq=2, Hkv=2, d=64, N=1600, K=8, seed=91, dtype="bf16", needles=2,
+           needle_mode="random", window=192),
+    # G = 16 (8-position tiles), d = 128, the longest window (15 chunks before the own one)
+    custom("win1024-bf16-gqa16-d128", B=1, Hq=16, Hkv=1, d=128, N=2048, K=4, seed=92, dtype="bf16",
+           window=1024),
+    # CUDA-core selection and prefill (G = 3) under a window
     custom("win256-bf16-gqa3", B=1, Hq=6, Hkv=2, d=64, N=1600, K=7, seed=83, dtype="bf16", window=256),
     custom("win320-fp32-d64", B=2, Hq=2, Hkv=1, d=64, N=1024, K=5, seed=84, dtype="fp32", needles=2,
            needle_mode="random", window=320),
