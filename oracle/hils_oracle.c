@@ -27,6 +27,10 @@
  *   [AIT-Gloss] same article, glossary entry "계층적 소프트맥스"
  *              (hierarchical softmax): an inter-chunk softmax over the chunk
  *              scores, then an intra-chunk softmax.
+ *   [AIT-QCal] same article, section "방법론" and glossary entry "저계수
+ *              쿼리 보정" (low-rank query calibration): a light adapter that
+ *              applies a low-rank down/up projection to the query, giving a
+ *              calibrated query for the chunk-level scores.
  *
  * Readings where the pages are silent (each is also listed in the design
  * notes of the repository):
@@ -46,7 +50,12 @@
  *     (the window) only;
  *   - query head hq reads kv head floor(hq / G);
  *   - top-K ties: the lower chunk id wins; fewer than K candidates: keep
- *     them all, pad the id list with -1; ids are reported in ascending order.
+ *     them all, pad the id list with -1; ids are reported in ascending order;
+ *   - Q-Cal ([AIT-QCal]) is residual, per query head, and acts on the query
+ *     (not on a hidden state, which this path does not see):
+ *     q^ = q + W_up (W_down q), W_down [r x d], W_up [d x r].  q^ replaces q
+ *     in the chunk score s^ = tau <q^, k'_c> + b'_c, so it steers both the
+ *     selection and the fusion weights; the attention inside chunks keeps q.
  *
  * Everything is computed in double precision from the exact stored input
  * values (bf16 and fp32 values are exactly representable in double).
@@ -232,7 +241,9 @@ static double attend_keys(const float* q, const float* Kbh, const float* Vbh, in
  * Hierarchical attention of the given rows ([HP-Abs], [AIT-Meth], [AIT-Gloss]):
  *   for each selected chunk c (ids[r, :], -1 entries skipped):
  *       o_c = softmax_j(<q, k_j>/sqrt(d)) V   over the chunk's C keys
- *       u_c = s^_{i,c}                      (score_mode 0: the surrogate)
+ *       u_c = s^_{i,c}                      (score_mode 0: the surrogate,
+ *                                              with the scoring query qscore
+ *                                              when given, else q)
  *           = log sum_j exp(<q,k_j>/sqrt(d))  (score_mode 1: the exact chunk
  *                                              log-sum-exp; used by the
  *                                              dense-equivalence pin)
@@ -245,8 +256,8 @@ static double attend_keys(const float* q, const float* Kbh, const float* Vbh, in
 void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* V,
                         const double* kp, const double* bp,
                         int64_t n_rows, const int32_t* rb, const int32_t* rhq, const int64_t* rpos,
-                        const float* qrows, const int32_t* ids, int64_t ids_stride, int score_mode,
-                        double* O, double* lse_own) {
+                        const float* qrows, const float* qscore, const int32_t* ids, int64_t ids_stride,
+                        int score_mode, double* O, double* lse_own) {
   const int64_t d = D->d, C = D->C, nc = D->N / D->C, G = D->Hq / D->Hkv;
   const double tau = 1.0 / sqrt((double)d);
 #pragma omp parallel for schedule(dynamic, 8)
@@ -254,6 +265,7 @@ void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* 
     const int64_t bh = (int64_t)rb[r] * D->Hkv + rhq[r] / G;
     const int64_t i = rpos[r], own = i / C;
     const float* q = qrows + r * d;
+    const float* qs = qscore ? qscore + r * d : q;
     const float* Kbh = K + bh * D->N * d;
     const float* Vbh = V + bh * D->N * d;
     const int64_t nsel = ids_stride;
@@ -265,7 +277,7 @@ void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* 
       const int64_t c = ids[r * ids_stride + t];
       if (c < 0) continue;
       const double lse = attend_keys(q, Kbh, Vbh, c * C, (c + 1) * C, d, tau, s, oc + m_used * d);
-      u[m_used] = (score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]
+      u[m_used] = (score_mode == 0) ? tau * dot_fdd(qs, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]
                                     : lse;
       ++m_used;
     }
@@ -289,6 +301,35 @@ void hils_oracle_attend(const hils_oracle_dims* D, const float* K, const float* 
     free(u);
     free(oc);
     free(s);
+  }
+}
+
+/*
+ * Q-Cal ([AIT-QCal]): q^ = q + W_up (W_down q) for each row, with the
+ * projections of the row's query head.
+ *   q      [n_rows, d] float      rhq [n_rows] query head of each row
+ *   w_down [Hq, r, d] float       w_up [Hq, d, r] float
+ *   out    [n_rows, d] double
+ */
+void hils_oracle_qcal(int64_t n_rows, int64_t d, int64_t r, const int32_t* rhq, const float* q,
+                      const float* w_down, const float* w_up, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t row = 0; row < n_rows; ++row) {
+    const float* x = q + row * d;
+    const float* Wd = w_down + (int64_t)rhq[row] * r * d;
+    const float* Wu = w_up + (int64_t)rhq[row] * d * r;
+    double* y = out + row * d;
+    double z[256];   /* W_down q, r <= 256 */
+    for (int64_t a = 0; a < r; ++a) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < d; ++t) acc += (double)Wd[a * d + t] * (double)x[t];
+      z[a] = acc;
+    }
+    for (int64_t t = 0; t < d; ++t) {
+      double acc = (double)x[t];
+      for (int64_t a = 0; a < r; ++a) acc += (double)Wu[t * r + a] * z[a];
+      y[t] = acc;
+    }
   }
 }
 

@@ -53,8 +53,9 @@ def _load():
         lib.hils_oracle_summary.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64, P, P]
         lib.hils_oracle_scores.argtypes = [P, P, P, ctypes.c_int64, P, P, P, P, P]
         lib.hils_oracle_select.argtypes = [P, P, P, ctypes.c_int64, P, P, P, P, P, P, P]
-        lib.hils_oracle_attend.argtypes = [P, P, P, P, P, ctypes.c_int64, P, P, P, P, P,
+        lib.hils_oracle_attend.argtypes = [P, P, P, P, P, ctypes.c_int64, P, P, P, P, P, P,
                                            ctypes.c_int64, ctypes.c_int, P, P]
+        lib.hils_oracle_qcal.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P, P, P]
         lib.hils_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -160,8 +161,10 @@ class Oracle:
                                      _p(rows.pos), _p(rows.q), _p(ids), _p(sel), _p(gap))
         return ids, sel, gap
 
-    def attend(self, Kt, Vt, kp, bp, rows: Rows, ids, score_mode=0):
-        """Fused output O [n,d] and own-chunk log-sum-exp [n] for given ids."""
+    def attend(self, Kt, Vt, kp, bp, rows: Rows, ids, score_mode=0, qscore=None):
+        """Fused output O [n,d] and local-branch log-sum-exp [n] for given ids.
+        qscore [n,d] (optional): the scoring query of each row (Q-Cal), used
+        for the chunk scores in the fusion; rows.q attends."""
         Kt, Vt = _f32(Kt), _f32(Vt)
         assert Kt.shape == (self.B, self.Hkv, self.N, self.d) and Vt.shape == Kt.shape
         kp, bp = self._kb(kp, bp)
@@ -170,8 +173,11 @@ class Oracle:
         assert ids.shape[0] == n
         O = np.empty((n, self.d), np.float64)
         lse = np.empty((n,), np.float64)
+        if qscore is not None:
+            qscore = _f32(qscore)
+            assert qscore.shape == rows.q.shape
         self._lib.hils_oracle_attend(ctypes.byref(self._d), _p(Kt), _p(Vt), _p(kp), _p(bp), n,
-                                     _p(rows.b), _p(rows.hq), _p(rows.pos), _p(rows.q), _p(ids),
+                                     _p(rows.b), _p(rows.hq), _p(rows.pos), _p(rows.q), _p(qscore), _p(ids),
                                      ids.shape[1], int(score_mode), _p(O), _p(lse))
         return O, lse
 
@@ -190,6 +196,22 @@ class Oracle:
         B, Hq, d = q.shape
         return dict(ids=ids.reshape(B, Hq, -1), sel=sel.reshape(B, Hq, -1), gap=gap.reshape(B, Hq),
                     O=O.reshape(B, Hq, d), lse_own=lse.reshape(B, Hq), rows=rows)
+
+
+def qcal(q: np.ndarray, hq: np.ndarray, w_down: np.ndarray, w_up: np.ndarray) -> np.ndarray:
+    """Q-Cal (aitrends.kr article, section "방법론" and glossary entry
+    "저계수 쿼리 보정"): q^ = q + W_up (W_down q) per row with the projections
+    of the row's query head.  q [n,d], hq [n], w_down [Hq,r,d], w_up [Hq,d,r];
+    returns q^ [n,d] in double."""
+    q, w_down, w_up = _f32(q), _f32(w_down), _f32(w_up)
+    hq = np.ascontiguousarray(hq, dtype=np.int32)
+    n, d = q.shape
+    Hq, r, d2 = w_down.shape
+    assert d2 == d and w_up.shape == (Hq, d, r) and len(hq) == n and r <= 256
+    assert n == 0 or (hq.min() >= 0 and hq.max() < Hq)
+    out = np.empty((n, d), np.float64)
+    _load().hils_oracle_qcal(n, d, r, _p(hq), _p(q), _p(w_down), _p(w_up), _p(out))
+    return out
 
 
 def gather_pages(pages: np.ndarray, table: np.ndarray) -> np.ndarray:

@@ -377,3 +377,72 @@ def test_pin_window_over_the_whole_sequence_is_dense_attention():
     assert np.all(ids == -1)
     O, _ = o.attend(K, V, kp, bp, rows, ids, score_mode=0)
     assert np.max(np.abs(O - dense_causal(Q, K, V, 1).reshape(-1, d))) < 1e-12
+
+
+# ---------------------------------------------------------------- Q-Cal
+# aitrends.kr article, section "방법론" and glossary entry "저계수 쿼리 보정":
+# a low-rank down/up projection of the query gives the calibrated query that
+# scores the chunks.
+
+def test_pin_qcal_hand_built_projection():
+    """W_down picks q0 and 2 q2, W_up sends them to dims 1 and 4 with factors
+    3 and -1: q^ = q + (0, 3 q0, 0, 0, -2 q2, 0), worked out by hand."""
+    from oracle.oracle import qcal
+    wd = np.zeros((1, 2, 6), np.float32)
+    wd[0, 0, 0], wd[0, 1, 2] = 1.0, 2.0
+    wu = np.zeros((1, 6, 2), np.float32)
+    wu[0, 1, 0], wu[0, 4, 1] = 3.0, -1.0
+    q = np.array([[0.5, -1.0, 2.0, 0.25, 4.0, -3.0], [1.0, 1.0, -1.5, 0.0, 0.5, 2.0]], np.float32)
+    out = qcal(q, np.zeros(2, np.int32), wd, wu)
+    want = q.astype(np.float64).copy()
+    want[:, 1] += 3.0 * want[:, 0]
+    want[:, 4] += -2.0 * q[:, 2]
+    assert np.array_equal(out, want)
+
+
+def test_pin_qcal_orthogonal_projection_per_head():
+    """With orthonormal rows U_h^T as W_down and -U_h as W_up, q^ is q with its
+    component in span(U_h) removed: U_h^T q^ = 0, and calibrating q^ again
+    changes nothing (a projection is idempotent).  Heads use their own U_h."""
+    from oracle.oracle import qcal
+    rng = np.random.default_rng(23)
+    Hq, d, r, n = 3, 16, 4, 40
+    U = np.stack([np.linalg.qr(rng.standard_normal((d, r)))[0] for _ in range(Hq)])   # [Hq, d, r]
+    wd = np.ascontiguousarray(U.transpose(0, 2, 1)).astype(np.float32)
+    wu = (-U).astype(np.float32)
+    hq = rng.integers(0, Hq, n).astype(np.int32)
+    q = rand(rng, n, d)
+    out = qcal(q, hq, wd, wu)
+    Uf = U.astype(np.float32).astype(np.float64)
+    for i in range(n):
+        assert np.max(np.abs(Uf[hq[i]].T @ out[i])) < 1e-6
+    assert np.max(np.abs(out - q)) > 0.1
+    again = qcal(out.astype(np.float32), hq, wd, wu)
+    assert np.max(np.abs(again - out)) < 1e-5
+
+
+def test_pin_scoring_query_steers_only_the_fusion():
+    """A scoring query pushed far along k'_c makes chunk c's fusion weight 1,
+    so O is chunk c's own softmax attention computed with the attending query
+    q (a textbook softmax over 64 keys), not with the scoring query."""
+    rng = np.random.default_rng(29)
+    B, Hq, Hkv, N, d, C = 1, 2, 1, 512, 32, 64
+    K, V = rand(rng, B, Hkv, N, d), rand(rng, B, Hkv, N, d)
+    LQ = rand(rng, B, Hkv, N // C, d)
+    o = Oracle(B, Hq, Hkv, N, d, C, 1)
+    kp, bp = o.summary(K, LQ)
+    c, pos = 3, 7 * C + 20
+    q = rand(rng, 2, d)
+    qs = q + 400.0 * (kp[0, 0, c] / np.linalg.norm(kp[0, 0, c])).astype(np.float32)
+    rows = Rows([0, 0], [0, 1], [pos, pos], q)
+    ids = np.array([[c], [c]], np.int32)
+    O, _ = o.attend(K, V, kp, bp, rows, ids, qscore=qs)
+    keys = K[0, 0, c * C:(c + 1) * C].astype(np.float64)
+    for r in range(2):
+        s = keys @ q[r].astype(np.float64) / math.sqrt(d)
+        p = np.exp(s - s.max())
+        want = (p / p.sum()) @ V[0, 0, c * C:(c + 1) * C].astype(np.float64)
+        assert np.max(np.abs(O[r] - want)) < 1e-9
+    # the same rows without the scoring query mix in the own chunk
+    O2, _ = o.attend(K, V, kp, bp, rows, ids)
+    assert np.max(np.abs(O2 - O)) > 1e-3

@@ -17,8 +17,8 @@ MUTANTS = {
                            "(c < own) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d)"),
     "select_without_bias": ("cand[c].s = tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c];",
                             "cand[c].s = tau * dot_fdd(q, kp + (bh * nc + c) * d, d);"),
-    "fusion_without_bias": ("(score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]",
-                            "(score_mode == 0) ? tau * dot_fdd(q, kp + (bh * nc + c) * d, d)"),
+    "fusion_without_bias": ("(score_mode == 0) ? tau * dot_fdd(qs, kp + (bh * nc + c) * d, d) + bp[bh * nc + c]",
+                            "(score_mode == 0) ? tau * dot_fdd(qs, kp + (bh * nc + c) * d, d)"),
     "fusion_surrogate_unscaled": ("(score_mode == 0) ? tau * dot_fdd(", "(score_mode == 0) ? dot_fdd("),
     "compressed_key_wrong_index": ("out[t] += p * (double)kc[j * d + t];", "out[t] += p * (double)kc[t * d + j % d];"),
     "causal_mask_off_by_one": ("w0, i + 1, d, tau", "w0, i, d, tau"),
@@ -34,6 +34,12 @@ MUTANTS = {
                                   "const int64_t n = i / D->C - (window_chunks(D) - 2);"),
     "fusion_uniform_weights": ("const double w = exp(u[t] - M) / Z;", "const double w = 1.0 / (double)m_used;"),
     "fusion_drops_own_chunk": ("u[m_used] = lo;", "u[m_used] = -INFINITY;"),
+    "qcal_not_residual": ("double acc = (double)x[t];", "double acc = 0.0;"),
+    "qcal_up_transposed": ("acc += (double)Wu[t * r + a] * z[a];", "acc += (double)Wu[a * d + t] * z[a];"),
+    "qcal_down_transposed": ("acc += (double)Wd[a * d + t] * (double)x[t];",
+                             "acc += (double)Wd[t * r + a] * (double)x[t];"),
+    "qcal_one_head_for_all": ("const float* Wd = w_down + (int64_t)rhq[row] * r * d;", "const float* Wd = w_down;"),
+    "fusion_ignores_scoring_query": ("const float* qs = qscore ? qscore + r * d : q;", "const float* qs = q;"),
 }
 
 
