@@ -16,6 +16,7 @@
 #include "select_tc.cuh"
 #include "prefill_cc.cuh"
 #include "prefill_local.cuh"
+#include "qcal.cuh"
 
 using namespace hils;
 
@@ -93,6 +94,20 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 tensor map [planes][rows][inner], 128-byte swizzle, box {64, box_rows, 1}.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                 uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {inner, rows, planes};
+  cuuint64_t strides[2] = {inner * 2, inner * 2 * rows};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -341,7 +356,8 @@ int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const 
 template <typename T, int D>
 int launch_decode(const hils_dims* d, const void* q, const void* kc, const void* vc, const float* kp,
                   const float* bp, const void* kmma, const int32_t* seqlens, void* o, int32_t* ids_out,
-                  float* scores_out, void* ws_ptr, cudaStream_t st, PagedKv pk = PagedKv{nullptr, 0}) {
+                  float* scores_out, void* ws_ptr, cudaStream_t st, PagedKv pk = PagedKv{nullptr, 0},
+                  const void* q_score = nullptr) {
   constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
   const int64_t nc = d->seqlen / kChunk, rows = int64_t(d->batch) * d->heads_q;
   const int G = d->heads_q / d->heads_kv, K = d->topk;
@@ -353,7 +369,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   constexpr auto k1 = decode_scores_kernel<T, D, BF>;
   if (smem1 > 48 * 1024 && set_smem_max<k1>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
-  k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
+  k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q_score ? q_score : q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores, wm1);
   decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
                                                       ws.sel_scores, wm1);
@@ -479,12 +495,13 @@ size_t hils_decode_workspace_bytes(const hils_dims* d) {
 static int decode_entry(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
                         const float* kprime, const float* bprime, const void* kprime_mma, const int32_t* seqlens,
                         void* o, int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
-                        hils_stream_t stream, PagedKv pk) {
+                        hils_stream_t stream, PagedKv pk, const void* q_score = nullptr) {
   int rc = check_dims(d);
   if (rc) return rc;
   if (d->heads_q / d->heads_kv > 32) return HILS_ERR_UNSUPPORTED;   // one lane per query head of a kv head
   if (!ptr_ok(q) || !ptr_ok(k_cache) || !ptr_ok(v_cache) || !ptr_ok(seqlens) || !ptr_ok(o) || !ptr_ok(workspace))
     return HILS_ERR_INVALID_ARGUMENT;
+  if (q_score != nullptr && !aligned16(q_score)) return HILS_ERR_INVALID_ARGUMENT;
   if ((ids_out != nullptr && !aligned16(ids_out)) || (scores_out != nullptr && !aligned16(scores_out)))
     return HILS_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < hils_decode_workspace_bytes(d)) return HILS_ERR_WORKSPACE_TOO_SMALL;
@@ -492,13 +509,13 @@ static int decode_entry(const hils_dims* d, const void* q, const void* k_cache, 
   if (d->dtype == HILS_BF16) {
     if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
     if (d->head_dim == 64)
-      return launch_decode<__nv_bfloat16, 64>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk);
-    return launch_decode<__nv_bfloat16, 128>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk);
+      return launch_decode<__nv_bfloat16, 64>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk, q_score);
+    return launch_decode<__nv_bfloat16, 128>(d, q, k_cache, v_cache, nullptr, nullptr, kprime_mma, seqlens, o, ids_out, scores_out, workspace, st, pk, q_score);
   }
   if (!ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
   if (d->head_dim == 64)
-    return launch_decode<float, 64>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk);
-  return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk);
+    return launch_decode<float, 64>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk, q_score);
+  return launch_decode<float, 128>(d, q, k_cache, v_cache, kprime, bprime, nullptr, seqlens, o, ids_out, scores_out, workspace, st, pk, q_score);
 }
 
 int hils_attn_decode(const hils_dims* d, const void* q, const void* k_cache, const void* v_cache,
@@ -516,6 +533,68 @@ int hils_attn_decode_paged(const hils_dims* d, const void* q, const void* k_page
   if (page_table == nullptr || n_pages < 1) return HILS_ERR_INVALID_ARGUMENT;
   return decode_entry(d, q, k_pages, v_pages, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out, workspace,
                       workspace_bytes, stream, PagedKv{page_table, n_pages});
+}
+
+int hils_attn_decode_qcal(const hils_dims* d, const void* q, const void* q_score, const void* k_cache,
+                          const void* v_cache, const int32_t* page_table, int64_t n_pages, const float* kprime,
+                          const float* bprime, const void* kprime_mma, const int32_t* seqlens, void* o,
+                          int32_t* ids_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                          hils_stream_t stream) {
+  if (q_score == nullptr) return HILS_ERR_INVALID_ARGUMENT;
+  if (page_table != nullptr && n_pages < 1) return HILS_ERR_INVALID_ARGUMENT;
+  return decode_entry(d, q, k_cache, v_cache, kprime, bprime, kprime_mma, seqlens, o, ids_out, scores_out, workspace,
+                      workspace_bytes, stream, PagedKv{page_table, page_table ? n_pages : 0}, q_score);
+}
+
+int hils_query_calibrate(const hils_dims* d, const void* q, int64_t n_pos, const void* w_down, const void* w_up,
+                         int32_t rank, void* q_hat, hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if (n_pos < 1 || rank < 8 || rank > kQcalMaxRank || rank % 8 != 0) return HILS_ERR_INVALID_ARGUMENT;
+  if (!ptr_ok(q) || !ptr_ok(w_down) || !ptr_ok(w_up) || !ptr_ok(q_hat)) return HILS_ERR_INVALID_ARGUMENT;
+  const int64_t rows = int64_t(d->batch) * d->heads_q * n_pos;
+  const size_t es = d->dtype == HILS_BF16 ? 2 : 4;
+  // q_hat may be q itself (in place) but must not overlap it otherwise
+  const uintptr_t a = reinterpret_cast<uintptr_t>(q), b = reinterpret_cast<uintptr_t>(q_hat);
+  const uintptr_t span = uintptr_t(rows) * d->head_dim * es;
+  if (a != b && a < b + span && b < a + span) return HILS_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t bhq = int64_t(d->batch) * d->heads_q;
+  if (d->dtype == HILS_BF16 && n_pos >= 64 && bhq <= 65535 && n_pos <= (int64_t(1) << 31) - 128) {
+    CUtensorMap tq, to;
+    if (!make_map_3d(&tq, q, d->head_dim, n_pos, bhq, 128) || !make_map_3d(&to, q_hat, d->head_dim, n_pos, bhq, 128))
+      return HILS_ERR_CUDA;
+    const dim3 grid(unsigned((n_pos + 127) / 128), unsigned(bhq));
+    const auto* wd = static_cast<const __nv_bfloat16*>(w_down);
+    const auto* wu = static_cast<const __nv_bfloat16*>(w_up);
+    if (d->head_dim == 64) {
+      constexpr auto fn = qcal_tc_kernel<64>;
+      if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
+      fn<<<grid, 128, QcalTc<64>::SMEM, st>>>(tq, to, wd, wu, rank, d->heads_q);
+    } else {
+      constexpr auto fn = qcal_tc_kernel<128>;
+      if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
+      fn<<<grid, 128, QcalTc<128>::SMEM, st>>>(tq, to, wd, wu, rank, d->heads_q);
+    }
+    return launched(1);
+  }
+  const unsigned blocks = unsigned((rows * 32 + 127) / 128);
+  if (d->dtype == HILS_BF16) {
+    const auto* qq = static_cast<const __nv_bfloat16*>(q);
+    const auto* wd = static_cast<const __nv_bfloat16*>(w_down);
+    const auto* wu = static_cast<const __nv_bfloat16*>(w_up);
+    auto* out = static_cast<__nv_bfloat16*>(q_hat);
+    if (d->head_dim == 64) qcal_simt_kernel<__nv_bfloat16, 64><<<blocks, 128, 0, st>>>(qq, wd, wu, rank, n_pos, d->heads_q, rows, out);
+    else qcal_simt_kernel<__nv_bfloat16, 128><<<blocks, 128, 0, st>>>(qq, wd, wu, rank, n_pos, d->heads_q, rows, out);
+  } else {
+    const auto* qq = static_cast<const float*>(q);
+    const auto* wd = static_cast<const float*>(w_down);
+    const auto* wu = static_cast<const float*>(w_up);
+    auto* out = static_cast<float*>(q_hat);
+    if (d->head_dim == 64) qcal_simt_kernel<float, 64><<<blocks, 128, 0, st>>>(qq, wd, wu, rank, n_pos, d->heads_q, rows, out);
+    else qcal_simt_kernel<float, 128><<<blocks, 128, 0, st>>>(qq, wd, wu, rank, n_pos, d->heads_q, rows, out);
+  }
+  return launched(1);
 }
 
 }  // extern "C"

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "HILS_OK", 1: "HILS_ERR_INVALID_ARGUMENT", 2: "HILS_ERR_UNSUP
 EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hils_prefill_workspace_bytes",
            "hils_attn_prefill",
            "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
-           "hils_landmark_summary_paged", "hils_attn_decode_paged",
+           "hils_landmark_summary_paged", "hils_attn_decode_paged", "hils_query_calibrate", "hils_attn_decode_qcal",
            "hils_get_status", "hils_selftest_bounded_wait", "hils_strerror", "hils_kernel_launches")
 DECODE_FIXED_SCRATCH_BYTES = 16 << 20
 
@@ -64,6 +64,8 @@ def lib():
         L.hils_attn_decode_fixed_scratch.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P]
         L.hils_landmark_summary_paged.argtypes = [D, P, P, I64, P, I64, I64, P, P, P, P]
         L.hils_attn_decode_paged.argtypes = [D, P, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_query_calibrate.argtypes = [D, P, I64, P, P, ctypes.c_int32, P, P]
+        L.hils_attn_decode_qcal.argtypes = [D, P, P, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
         L.hils_selftest_bounded_wait.argtypes = [ctypes.c_int32, P]
         L.hils_strerror.argtypes = [ctypes.c_int]
@@ -193,6 +195,22 @@ def hils_attn_decode_paged(dims, q, k_pages, v_pages, page_table, n_pages, kprim
                                         _stream(stream)))
 
 
+def hils_query_calibrate(dims, q, n_pos, w_down, w_up, rank, q_hat, stream=None):
+    _check("hils_query_calibrate",
+           lib().hils_query_calibrate(ctypes.byref(dims), _ptr(q), int(n_pos), _ptr(w_down), _ptr(w_up), int(rank),
+                                      _ptr(q_hat), _stream(stream)))
+
+
+def hils_attn_decode_qcal(dims, q, q_score, k_cache, v_cache, page_table, n_pages, kprime, bprime, kprime_mma,
+                          seqlens, o, ids_out, scores_out, workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("hils_attn_decode_qcal",
+           lib().hils_attn_decode_qcal(ctypes.byref(dims), _ptr(q), _ptr(q_score), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(page_table), int(n_pages), _ptr(kprime), _ptr(bprime), _ptr(kprime_mma),
+                                       _ptr(seqlens), _ptr(o), _ptr(ids_out), _ptr(scores_out), _ptr(workspace),
+                                       int(nbytes), _stream(stream)))
+
+
 def hils_get_status(stream=None) -> int:
     v = ctypes.c_int32(0)
     _check("hils_get_status", lib().hils_get_status(ctypes.byref(v), _stream(stream)))
@@ -255,6 +273,49 @@ def prefill(q, k, v, lq, topk, stream=None, return_all=False, window=0):
     if return_all:
         return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse)
     return o
+
+
+def query_calibrate(q, w_down, w_up, out=None, stream=None):
+    """Q-Cal: q^ = q + W_up (W_down q) per query head, for q [B,Hq,N,d] (a
+    prefill) or [B,Hq,d] (a decode step); w_down [Hq,r,d], w_up [Hq,d,r]."""
+    n_pos = q.shape[2] if q.dim() == 4 else 1
+    B, Hq, d = q.shape[0], q.shape[1], q.shape[-1]
+    Hq_w, r, _ = w_down.shape
+    dims = make_dims(B, Hq, Hq, d, CHUNK, 1, q.dtype)
+    out = torch.empty_like(q) if out is None else out
+    hils_query_calibrate(dims, q, n_pos, w_down, w_up, r, out, stream)
+    return out
+
+
+def prefill_qcal(q, k, v, lq, topk, w_down, w_up, stream=None, return_all=False, window=0):
+    """HiLS prefill with Q-Cal: summary -> calibrate -> select on q^ ->
+    sparse attention with q."""
+    dims = dims_for(q, k, topk, window)
+    summ = landmark_summary(k, lq, topk, stream=stream)
+    q_hat = query_calibrate(q, w_down, w_up, stream=stream)
+    ids, scores = select(q_hat, summ, k.shape[1], topk, stream, window)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, prefill_workspace(dims, q.device), stream=stream)
+    if return_all:
+        return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse, q_hat=q_hat)
+    return o
+
+
+def decode_step_qcal(q, q_score, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None,
+                     window=0):
+    """One decode step with a separate scoring query q_score [B,Hq,d]."""
+    B, Hq, d = q.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    dims = make_dims(B, Hq, Hkv, d, cap, topk, q.dtype, window=window)
+    if workspace is None:
+        workspace = torch.empty((hils_decode_workspace_bytes(dims),), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    ids = torch.empty((B, Hq, topk), dtype=torch.int32, device=q.device)
+    scores = torch.empty((B, Hq, topk), dtype=torch.float32, device=q.device)
+    hils_attn_decode_qcal(dims, q, q_score, k_cache, v_cache, None, 0, summ.kprime, summ.bprime, summ.kprime_mma,
+                          seqlens, o, ids, scores, workspace, stream=stream)
+    return o, ids, scores
 
 
 def decode_step(q, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None, window=0):

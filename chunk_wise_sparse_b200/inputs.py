@@ -258,3 +258,27 @@ def sample_rows(w: Workload, n: int | None = None) -> np.ndarray:
         return np.arange(total, dtype=np.int64)
     rng = np.random.default_rng(w.seed + 1000)
     return np.sort(rng.choice(total, size=n, replace=False)).astype(np.int64)
+
+
+@dataclasses.dataclass
+class QcalWeights:
+    """Random-init Q-Cal projections (no trained adapter exists here):
+    w_down [Hq, r, d] ~ N(0, 1/d), w_up [Hq, d, r] ~ N(0, 0.25/r), so that
+    W_down q has unit scale and the correction W_up W_down q about half the
+    scale of q.  ``*_f32`` hold the exact stored values; ``*_bits`` the bf16
+    patterns (bf16 only)."""
+    rank: int
+    w_down_f32: np.ndarray
+    w_up_f32: np.ndarray
+    w_down_bits: np.ndarray | None = None
+    w_up_bits: np.ndarray | None = None
+
+
+def qcal_weights(Hq: int, d: int, rank: int, seed: int, dtype: str = "bf16") -> QcalWeights:
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 17, rank]))
+    wd = (rng.standard_normal((Hq, rank, d), dtype=np.float32) / np.float32(np.sqrt(d))).astype(np.float32)
+    wu = (rng.standard_normal((Hq, d, rank), dtype=np.float32) * np.float32(0.5 / np.sqrt(rank))).astype(np.float32)
+    if dtype == "bf16":
+        bd, bu = round_bf16_bits(wd), round_bf16_bits(wu)
+        return QcalWeights(rank, bf16_bits_to_f32(bd), bf16_bits_to_f32(bu), bd, bu)
+    return QcalWeights(rank, wd, wu)

@@ -249,6 +249,43 @@ int hils_attn_decode_paged(const hils_dims* dims, const void* q, const void* k_p
                            hils_stream_t stream);
 
 /*
+ * Low-rank query calibration (Q-Cal) -- [AIT-Meth] and the glossary entry
+ * "저계수 쿼리 보정" of the same article: a light adapter maps each query to
+ *     q^ = q + W_up (W_down q)
+ * with per-query-head projections of rank r (read as residual, on the query).
+ * q^ is the scoring query: pass it to hils_select (prefill) or
+ * hils_attn_decode_qcal (decode) in place of q for the chunk scores; the
+ * attention inside chunks keeps q (hils_attn_prefill takes q and the scores
+ * that hils_select returned for q^).
+ *   q       [B, Hq, n_pos, d] dtype; n_pos = dims.seqlen for a prefill, 1 for
+ *           a decode step (dims.seqlen is otherwise not used here)
+ *   w_down  [Hq, r, d] dtype
+ *   w_up    [Hq, d, r] dtype
+ *   rank    r: a multiple of 8, 8 <= r <= 64
+ *   q_hat   [B, Hq, n_pos, d] dtype out; may be q itself (in place) but must
+ *           not overlap it otherwise
+ * bf16: products accumulate in fp32 on tensor cores, W_down q is rounded to
+ * bf16 before the up projection and q^ is rounded to bf16 (RNE).  fp32:
+ * fp32 arithmetic throughout.
+ */
+int hils_query_calibrate(const hils_dims* dims, const void* q, int64_t n_pos, const void* w_down,
+                         const void* w_up, int32_t rank, void* q_hat, hils_stream_t stream);
+
+/*
+ * Decode step whose chunk scores use a separate scoring query, e.g. the
+ * Q-Cal output of hils_query_calibrate: q_score [B, Hq, d] dtype scores and
+ * selects the chunks and gives the fusion weights; q attends.  page_table
+ * NULL: contiguous caches as in hils_attn_decode; otherwise chunk pages as in
+ * hils_attn_decode_paged (n_pages >= 1).  Other arguments, workspace and
+ * errors as in hils_attn_decode; q_score NULL is HILS_ERR_INVALID_ARGUMENT.
+ */
+int hils_attn_decode_qcal(const hils_dims* dims, const void* q, const void* q_score, const void* k_cache,
+                          const void* v_cache, const int32_t* page_table, int64_t n_pages,
+                          const float* kprime, const float* bprime, const void* kprime_mma,
+                          const int32_t* seqlens, void* o, int32_t* ids_out, float* scores_out,
+                          void* workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/*
  * Synchronises `stream`, copies the device status word of the current device
  * into *host_status (HILS_OK or a HILS_ERR_DEVICE_* code recorded by a kernel
  * since the last call) and clears it.  Returns HILS_ERR_CUDA if the

@@ -98,6 +98,21 @@ def test_window_sizes(lib):
     assert lib.hils_select(ctypes.byref(d16), None, None, None, None, None, None, None) == 1   # dims pass, q NULL
 
 
+def test_qcal_arguments_rejected_before_launch(lib):
+    d = dims()
+    p, q2 = ctypes.c_void_p(256), ctypes.c_void_p(512)
+    for rank in (0, 7, 12, 72):
+        assert lib.hils_query_calibrate(ctypes.byref(d), p, 64, p, p, rank, q2, None) == 1
+    assert lib.hils_query_calibrate(ctypes.byref(d), p, 0, p, p, 16, q2, None) == 1        # no positions
+    assert lib.hils_query_calibrate(ctypes.byref(d), p, 64, p, p, 16, ctypes.c_void_p(272), None) == 1  # overlap
+    assert lib.hils_query_calibrate(ctypes.byref(d), p, 64, None, p, 16, q2, None) == 1
+    big = hils.hils_decode_workspace_bytes(d)
+    assert lib.hils_attn_decode_qcal(ctypes.byref(d), p, None, p, p, None, 0, None, None, p, p, p, None, None, p,
+                                     big, None) == 1      # no scoring query
+    assert lib.hils_attn_decode_qcal(ctypes.byref(d), p, p, p, p, p, 0, None, None, p, p, p, None, None, p,
+                                     big, None) == 1      # a page table needs pages
+
+
 def test_strerror(lib):
     for code in range(7):
         assert len(hils.strerror(code)) >= 2
