@@ -128,8 +128,11 @@ def cpu_oracle_sample(w, inp, budget_s=15.0):
     """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
     the summaries of a head subset plus sampled prefill rows.  Returns
     (tokens/s, description, threads)."""
-    from oracle.oracle import Oracle, Rows, max_threads
+    from oracle.oracle import Oracle, Rows, max_threads, qcal
     o = Oracle.for_workload(w)
+    if w.qcal:
+        from chunk_wise_sparse_b200.inputs import qcal_weights
+        wt = qcal_weights(w.Hq, w.d, w.qcal, seed=w.seed, dtype=w.dtype)
     # summaries: all chunks of one (b, kv head)
     one = Oracle(1, w.G, 1, w.N, w.d, w.C, w.K, w.window)
     t0 = time.perf_counter()
@@ -148,8 +151,13 @@ def cpu_oracle_sample(w, inp, budget_s=15.0):
         rows = Rows(np.zeros(n), np.zeros(n), pos, inp.q_f32[0, 0, pos] if w.kind != "decode" else
                     np.repeat(inp.q_f32[:1, 0], n, axis=0))
         t0 = time.perf_counter()
-        ids, _, _ = o.select(kp, bp, rows)
-        o.attend(inp.k_f32, inp.v_f32, kp, bp, rows, ids)
+        if w.qcal:
+            qs = qcal(rows.q, rows.hq, wt.w_down_f32, wt.w_up_f32).astype(np.float32)
+            ids, _, _ = o.select(kp, bp, Rows(rows.b, rows.hq, rows.pos, qs))
+            o.attend(inp.k_f32, inp.v_f32, kp, bp, rows, ids, qscore=qs)
+        else:
+            ids, _, _ = o.select(kp, bp, rows)
+            o.attend(inp.k_f32, inp.v_f32, kp, bp, rows, ids)
         elapsed += time.perf_counter() - t0
         done += n
         n = min(2 * n, 4096)
@@ -214,7 +222,7 @@ def workload_config(w, n_gpus):
         "inputs smaller than L2: a 256 MB buffer is written before every step, outside the kernel events, " \
         "and ms_per_step is the sum of the kernel events"
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "C": w.C, "K": w.K,
-            "window": w.window, "needles": w.needles, "seed": w.seed,
+            "window": w.window, "qcal_rank": w.qcal, "needles": w.needles, "seed": w.seed,
             "parallelism": f"dp{n_gpus} (independent replicas)", "l2": l2}
 
 
@@ -252,27 +260,57 @@ def run_ours(args, w, rank, world, local_rank):
     sc_d = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     flush = None if inputs_exceed_l2(w) else torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    use_qcal = w.qcal > 0
+    if use_qcal:
+        # Q-Cal projections (random init, resident like model weights); the
+        # prefill scores with q^, the decode step with the calibrated last row
+        from chunk_wise_sparse_b200.inputs import qcal_weights
+        wt = qcal_weights(Hq, d, w.qcal, seed=w.seed, dtype=w.dtype)
+        if wt.w_down_bits is not None:
+            wd = torch.from_numpy(wt.w_down_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+            wu = torch.from_numpy(wt.w_up_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        else:
+            wd, wu = torch.from_numpy(wt.w_down_f32).to(dev), torch.from_numpy(wt.w_up_f32).to(dev)
+        q_hat, qd_hat = torch.empty_like(q), torch.empty_like(qd)
+        cdims = hils.make_dims(B, Hq, Hq, d, 64, 1, q.dtype)
+    names = ["summary"] + (["qcal"] if use_qcal else []) + ["select", "prefill", "decode"]
+    n_ev = len(names) + 1
 
     def step(ev=None):
+        e = [0]
+
+        def mark():
+            if ev: ev[e[0]].record(stream)
+            e[0] += 1
+
         if flush is not None:
             flush.fill_(1)
-        if ev: ev[0].record(stream)
+        mark()
         hils.hils_landmark_summary(dims, k, lq, 0, N // 64, summ.kprime, summ.bprime, summ.kprime_mma, stream)
-        if ev: ev[1].record(stream)
-        hils.hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
-        if ev: ev[2].record(stream)
+        mark()
+        if use_qcal:
+            hils.hils_query_calibrate(cdims, q, N, wd, wu, w.qcal, q_hat, stream)
+            hils.hils_query_calibrate(cdims, qd, 1, wd, wu, w.qcal, qd_hat, stream)
+            mark()
+        hils.hils_select(dims, q_hat if use_qcal else q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores,
+                         stream)
+        mark()
         hils.hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, pws, stream=stream)
-        if ev: ev[3].record(stream)
-        hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
-                              ws, stream=stream)
-        if ev: ev[4].record(stream)
+        mark()
+        if use_qcal:
+            hils.hils_attn_decode_qcal(ddims, qd, qd_hat, k, v, None, 0, summ.kprime, summ.bprime, summ.kprime_mma,
+                                       seq, od, ids_d, sc_d, ws, stream=stream)
+        else:
+            hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
+                                  ws, stream=stream)
+        mark()
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if hils.hils_get_status() != 0:
         raise RuntimeError("device status error during warm-up")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
     if world > 1:
         dist.barrier()
@@ -295,7 +333,7 @@ def run_ours(args, w, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # ms per kernel
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(n_ev - 1)] for e in evs])   # ms per kernel
     ms_step = total_ms / args.steps
     if flush is not None:
         ms_step = max_over_ranks(float(per.sum(axis=1).mean()), world, dev)
@@ -341,7 +379,6 @@ def run_ours(args, w, rank, world, local_rank):
 
     work = useful_work(w)
     peaks = load_peaks()
-    names = ["summary", "select", "prefill", "decode"]
     avg = per.mean(axis=0)
     kernels_ms = {n: float(a) for n, a in zip(names, avg)}
     dom = names[int(np.argmax(avg))]
@@ -375,6 +412,12 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clk,
         "e2e": e2e,
     }
+    if use_qcal:
+        eb = 2 if w.dtype == "bf16" else 4
+        qb = 2 * B * Hq * (N + 1) * d * eb     # q read and q^ written (prefill rows and the decode row)
+        line["qcal"] = {"rank": w.qcal, "ms": kernels_ms["qcal"], "bytes": qb,
+                        "gbs": qb / (kernels_ms["qcal"] / 1e3) / 1e9,
+                        "frac_of_hbm": qb / (kernels_ms["qcal"] / 1e3) / 1e9 / peaks["hbm_gbs"]}
     if not args.no_cpu_baseline and world == 1:
         v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}

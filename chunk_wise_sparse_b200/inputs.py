@@ -65,6 +65,7 @@ class Workload:
     sample_rows: int    # rows the oracle checks (0 = all rows)
     paged: bool = False  # decode: the KV cache in chunk pages (page_table)
     window: int = 0      # local window in tokens (0: the own chunk alone)
+    qcal: int = 0        # Q-Cal rank (0: no query calibration)
 
     @property
     def G(self) -> int:
@@ -95,6 +96,9 @@ WORKLOADS = {
                                        "bf16", 64, "random", "prefill", 4096),
     "prefill-512k-h16-d64": Workload("prefill-512k-h16-d64", 1, 16, 16, 64, 524288, 64, 16, 4,
                                      "bf16", 128, "random", "prefill+decode", 4096),
+    # the 512K workload with rank-16 Q-Cal: chunk scores from q^ = q + W_up W_down q
+    "prefill-512k-h16-d64-qcal16": Workload("prefill-512k-h16-d64-qcal16", 1, 16, 16, 64, 524288, 64, 16, 4,
+                                            "bf16", 128, "random", "prefill+decode", 4096, qcal=16),
     # the 512K workload's row lengths and kernels with two heads (about 0.3 GB
     # on the device): the case that profiler captures of the long-context
     # kernels run on
@@ -105,12 +109,13 @@ WORKLOAD_ORDER = list(WORKLOADS)
 
 
 def custom(name="custom", *, B=1, Hq=1, Hkv=1, d=64, N=1024, C=64, K=3, seed=0,
-           dtype="bf16", needles=0, needle_mode="none", kind="prefill", sample_rows=0, window=0) -> Workload:
+           dtype="bf16", needles=0, needle_mode="none", kind="prefill", sample_rows=0, window=0,
+           qcal=0) -> Workload:
     """A workload with arbitrary sizes (used for small parity cases)."""
     if needles == 0:
         needle_mode = "none"
     return Workload(name, B, Hq, Hkv, d, N, C, K, seed, dtype, needles, needle_mode, kind, sample_rows,
-                    window=window)
+                    window=window, qcal=qcal)
 
 
 def round_bf16_bits(x: np.ndarray) -> np.ndarray:
