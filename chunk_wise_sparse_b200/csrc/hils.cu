@@ -134,7 +134,7 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
   // reserved per CTA); the rest run one CTA per SM.  Two k' stages; the
   // candidate buffer takes what shared memory is left (it is compacted less
   // often the longer it is), at most 128 entries.
-  const uint32_t per_cta = D == 64 && KCAP == 16 ? 115712u : uint32_t(kMaxSmem);
+  const uint32_t per_cta = C::TWO_PER_SM ? 115712u : uint32_t(kMaxSmem);
   const int stages = 2;
   int cap = KCAP > 0 ? C::MIN_CAP : 0;
   if (KCAP > 0)

@@ -54,8 +54,17 @@ struct SelTc {
   // `cap` entries (K + 32 at least, host-chosen); KCAP == 0: a sorted
   // (score, chunk) list of K entries in shared memory.
   static constexpr int MIN_CAP = KCAP + 32;
-  // the staging area serves the shared-memory list path (K > 32) only
-  static constexpr uint32_t STG_BYTES = KCAP > 0 ? 0u : uint32_t(M) * STG_STRIDE * 4;
+  // d = 64 with K <= 16 runs two CTAs per SM; every other shape runs one
+  static constexpr bool TWO_PER_SM = D == 64 && KCAP == 16;
+  // STAGED: a row with passing scores in a 32-score group stages the group in
+  // shared memory and reads the passing ones back by column.  Otherwise they
+  // are picked out of the registers by a 5-level select (31 selects per
+  // append).  Staging wins where there is room for it next to two k' stages,
+  // i.e. with one CTA per SM; with two CTAs per SM it would cost a k' stage,
+  // which measured slower.
+  static constexpr bool STAGED = KCAP > 0 && !TWO_PER_SM;
+  // staging area (the shared-memory list path, K > 32, always uses it)
+  static constexpr uint32_t STG_BYTES = (KCAP == 0 || STAGED) ? uint32_t(M) * STG_STRIDE * 4 : 0u;
   static constexpr int THREADS = 192;
   // two CTAs per SM, two TMEM accumulators each (the MMA of tile j+1 runs
   // during the epilogue of tile j; three CTAs with one accumulator each
@@ -105,6 +114,13 @@ __device__ __forceinline__ void fma2_signs(float a0, float a1, uint64_t nt2, uin
       "mov.b64 {%0, %1}, vd;\n\t}"
       : "=r"(s0), "=r"(s1)
       : "f"(a0), "f"(a1), "l"(nt2), "l"(c2));
+}
+
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint64_t pack2(float x) {
@@ -335,6 +351,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = e < lim ? v[e] : -INFINITY;
       }
+      if (group == C::NT) {
+        // one maximum per tile: a tree of three-input maxima, 16 instructions
+        // for 32 scores plus the running maximum
+        float m[11];
+#pragma unroll
+        for (int t = 0; t < 10; ++t) m[t] = fmax3(v[3 * t], v[3 * t + 1], v[3 * t + 2]);
+        m[10] = fmaxf(v[30], v[31]);
+        const float a = fmax3(m[0], m[1], m[2]), bb = fmax3(m[3], m[4], m[5]), cc = fmax3(m[6], m[7], m[8]);
+        tmax = fmaxf(fmax3(a, bb, cc), fmax3(m[9], m[10], tmax));
+        return;
+      }
       // max tree: after the step of width w, v[t] (t < w) is the maximum of
       // the scores e = t (mod w) -- disjoint groups of 32 / w.
       // tau > 0 and rounding is monotone: tau * max = max of the scores.
@@ -357,8 +384,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return;
       }
       v[0] = fmaxf(v[0], v[1]);
-      if (group == 32) rv_insert(tau * v[0]);
-      else tmax = fmaxf(tmax, v[0]);
+      rv_insert(tau * v[0]);   // group == 32
     };
     // ---- scan, one 32-column group: test every score against thr, keep the
     // passing ones
@@ -389,26 +415,43 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // the buffer holds at least K + 32 entries and a compaction leaves at
         // most K, so one check per group makes room for all its scores
         if (__any_sync(0xffffffffu, count + __popc(bits) > p.cap)) keep_best(false, nullptr, nullptr);
-        // append the passing scores, one per lane and round; the score is
-        // picked out of the registers by a 5-level select on its column
-        while (__any_sync(0xffffffffu, bits != 0u)) {
-          const bool has = bits != 0u;
-          const int e = __clz(bits) & 31;
-          bits &= ~(0x80000000u >> e);
-          float w16[16], w8[8], w4[4], w2[2];
+        if constexpr (C::STAGED) {
+          // append the passing scores: a row with any stages its 32 scores,
+          // then reads each passing one back by its column
+          if (bits) {
 #pragma unroll
-          for (int t = 0; t < 16; ++t) w16[t] = (e & 16) ? v[t + 16] : v[t];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) w8[t] = (e & 8) ? w16[t + 8] : w16[t];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) w4[t] = (e & 4) ? w8[t + 4] : w8[t];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) w2[t] = (e & 2) ? w4[t + 2] : w4[t];
-          const float x = tau * ((e & 1) ? w2[1] : w2[0]);
-          if (has) {
-            tv[count * C::M] = x;
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(my_stg + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          }
+          while (bits) {
+            const int e = __clz(bits);
+            bits &= ~(0x80000000u >> e);
+            tv[count * C::M] = tau * my_stg[e];
             ti[count * C::M] = int32_t(cbase + e);
             ++count;
+          }
+        } else {
+          // append the passing scores, one per lane and round; the score is
+          // picked out of the registers by a 5-level select on its column
+          while (__any_sync(0xffffffffu, bits != 0u)) {
+            const bool has = bits != 0u;
+            const int e = __clz(bits) & 31;
+            bits &= ~(0x80000000u >> e);
+            float w16[16], w8[8], w4[4], w2[2];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) w16[t] = (e & 16) ? v[t + 16] : v[t];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) w8[t] = (e & 8) ? w16[t + 8] : w16[t];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) w4[t] = (e & 4) ? w8[t + 4] : w8[t];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) w2[t] = (e & 2) ? w4[t + 2] : w4[t];
+            const float x = tau * ((e & 1) ? w2[1] : w2[0]);
+            if (has) {
+              tv[count * C::M] = x;
+              ti[count * C::M] = int32_t(cbase + e);
+              ++count;
+            }
           }
         }
       } else {
