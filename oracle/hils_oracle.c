@@ -333,6 +333,182 @@ void hils_oracle_qcal(int64_t n_rows, int64_t d, int64_t r, const int32_t* rhq, 
   }
 }
 
+/*
+ * One branch of a row's fusion: keys [j0, j1) of one (b, kv head), their
+ * logits z_j = <q, k_j>/sqrt(d), the softmax p over them, the branch output
+ * o = sum p_j v_j and its log-sum-exp.
+ */
+typedef struct {
+  int64_t j0, j1;
+  double lse;
+  double u;        /* fusion score: s^ for a selected chunk, lse for the window */
+  int64_t chunk;   /* selected chunk id, -1 for the window branch */
+} branch_t;
+
+/*
+ * Backward of the forward pass for a fixed selection.  [AIT-Meth]: the chunk
+ * score s^ is part of the forward attention, so the gradient of the loss
+ * reaches the landmark queries (through k', b') and the Q-Cal adapter
+ * (through the scoring query); the top-K choice itself is not differentiated.
+ * Forward, per row i (query q, scoring query q^ = q unless dQs is given):
+ *   branch c (a selected chunk):  z_j = tau <q, k_j>, p = softmax(z),
+ *       o_c = sum p_j v_j,  u_c = tau <q^, k'_c> + b'_c
+ *   window branch w: the causal window keys, u_w = log sum_j exp(z_j)
+ *   a = softmax(u),  O = sum_c a_c o_c
+ * With g = dL/dO_i and Dg = <g, O>, per branch X_c = <g, o_c>:
+ *   du_c = a_c (X_c - Dg)
+ *   dz_j = a_c p_j (<g, v_j> - X_c)        (+ du_w p_j on the window branch,
+ *                                            since u_w = lse: together
+ *                                            a_w p_j (<g, v_j> - Dg))
+ *   dv_j += a_c p_j g,  dq += tau dz_j k_j,  dk_j += tau dz_j q
+ *   selected c: dq^ += tau du_c k'_c,  dk'_c += tau du_c q^,  db'_c += du_c
+ * Summary ([AIT-Meth], [AIT-Tech]), per chunk with zl_j = tau <lq, k_j>,
+ * pl = softmax(zl), k' = sum pl_j k_j, b' = lse(zl) - sum pl_j zl_j:
+ *   dzl_j = pl_j <dk', k_j - k'> - db' pl_j (zl_j - sum_k pl_k zl_k)
+ *   dlq += tau dzl_j k_j,  dk_j += tau dzl_j lq + pl_j dk'
+ * Inputs: Q [B,Hq,N,d], K, V [B,Hkv,N,d], LQ [B,Hkv,nc,d] (float, stored
+ * values), Qs (nullable; the scoring query, e.g. the Q-Cal output, else Q),
+ * ids [B,Hq,N,ids_stride] (-1 skipped), dO [B,Hq,N,d].  Outputs (double,
+ * overwritten): dQ, dQs (nullable: then the scoring-query gradient is added
+ * into dQ), dK, dV, dLQ.  Rows of different (b, kv head) touch disjoint
+ * gradients, so those run in parallel.
+ */
+void hils_oracle_backward(const hils_oracle_dims* D, const float* Q, const float* Qs, const float* Kt,
+                          const float* Vt, const float* LQ, const int32_t* ids, int64_t ids_stride,
+                          const float* dO, double* dQ, double* dQs, double* dK, double* dV, double* dLQ) {
+  const int64_t d = D->d, C = D->C, N = D->N, nc = N / C, G = D->Hq / D->Hkv;
+  const double tau = 1.0 / sqrt((double)d);
+  const int64_t nbh = D->B * D->Hkv;
+  double* kp = (double*)malloc(sizeof(double) * (size_t)(nbh * nc * d));
+  double* bp = (double*)malloc(sizeof(double) * (size_t)(nbh * nc));
+  double* dkp = (double*)calloc((size_t)(nbh * nc * d), sizeof(double));
+  double* dbp = (double*)calloc((size_t)(nbh * nc), sizeof(double));
+  hils_oracle_summary(D, Kt, LQ, 0, nc, kp, bp);
+  memset(dQ, 0, sizeof(double) * (size_t)(D->B * D->Hq * N * d));
+  if (dQs) memset(dQs, 0, sizeof(double) * (size_t)(D->B * D->Hq * N * d));
+  memset(dK, 0, sizeof(double) * (size_t)(nbh * N * d));
+  memset(dV, 0, sizeof(double) * (size_t)(nbh * N * d));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < nbh; ++bh) {
+    const int64_t b = bh / D->Hkv, h = bh % D->Hkv;
+    const float* Kbh = Kt + bh * N * d;
+    const float* Vbh = Vt + bh * N * d;
+    branch_t* br = (branch_t*)malloc(sizeof(branch_t) * (size_t)(ids_stride + 1));
+    double* z = (double*)malloc(sizeof(double) * (size_t)(C * window_chunks(D)));
+    double* o = (double*)malloc(sizeof(double) * (size_t)((ids_stride + 1) * d));
+    double* Orow = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t g = 0; g < G; ++g) {
+      const int64_t hq = h * G + g;
+      for (int64_t i = 0; i < N; ++i) {
+        const int64_t row = (b * D->Hq + hq) * N + i;
+        const float* q = Q + row * d;
+        const float* qs = Qs ? Qs + row * d : q;
+        const float* gr = dO + row * d;
+        double* dq = dQ + row * d;
+        double* dqs = dQs ? dQs + row * d : dq;
+        /* the row's branches: selected chunks, then the window */
+        int64_t nb = 0;
+        for (int64_t t = 0; t < ids_stride; ++t) {
+          const int64_t c = ids[row * ids_stride + t];
+          if (c < 0) continue;
+          br[nb].j0 = c * C;
+          br[nb].j1 = (c + 1) * C;
+          br[nb].chunk = c;
+          br[nb].u = tau * dot_fdd(qs, kp + (bh * nc + c) * d, d) + bp[bh * nc + c];
+          ++nb;
+        }
+        int64_t w0 = (i / C - (window_chunks(D) - 1)) * C;
+        if (w0 < 0) w0 = 0;
+        br[nb].j0 = w0;
+        br[nb].j1 = i + 1;
+        br[nb].chunk = -1;
+        ++nb;
+        for (int64_t c = 0; c < nb; ++c) {
+          br[c].lse = attend_keys(q, Kbh, Vbh, br[c].j0, br[c].j1, d, tau, z, o + c * d);
+          if (br[c].chunk < 0) br[c].u = br[c].lse;
+        }
+        double M = -INFINITY;
+        for (int64_t c = 0; c < nb; ++c) if (br[c].u > M) M = br[c].u;
+        double Zs = 0.0;
+        for (int64_t c = 0; c < nb; ++c) Zs += exp(br[c].u - M);
+        for (int64_t t = 0; t < d; ++t) Orow[t] = 0.0;
+        for (int64_t c = 0; c < nb; ++c) {
+          const double a = exp(br[c].u - M) / Zs;
+          for (int64_t t = 0; t < d; ++t) Orow[t] += a * o[c * d + t];
+        }
+        double Dg = 0.0;
+        for (int64_t t = 0; t < d; ++t) Dg += (double)gr[t] * Orow[t];
+        for (int64_t c = 0; c < nb; ++c) {
+          const double a = exp(br[c].u - M) / Zs;
+          double X = 0.0;
+          for (int64_t t = 0; t < d; ++t) X += (double)gr[t] * o[c * d + t];
+          const double du = a * (X - Dg);
+          for (int64_t j = br[c].j0; j < br[c].j1; ++j) {
+            const double zj = tau * dot_fd(q, Kbh + j * d, d);
+            const double pj = exp(zj - br[c].lse);
+            const double dP = dot_fd(gr, Vbh + j * d, d);
+            double dz = a * pj * (dP - X);
+            if (br[c].chunk < 0) dz += du * pj;
+            double* dkj = dK + (bh * N + j) * d;
+            double* dvj = dV + (bh * N + j) * d;
+            for (int64_t t = 0; t < d; ++t) {
+              dvj[t] += a * pj * (double)gr[t];
+              dq[t] += tau * dz * (double)Kbh[j * d + t];
+              dkj[t] += tau * dz * (double)q[t];
+            }
+          }
+          if (br[c].chunk >= 0) {
+            const int64_t cc = br[c].chunk;
+            for (int64_t t = 0; t < d; ++t) {
+              dqs[t] += tau * du * kp[(bh * nc + cc) * d + t];
+              dkp[(bh * nc + cc) * d + t] += tau * du * (double)qs[t];
+            }
+            dbp[bh * nc + cc] += du;
+          }
+        }
+      }
+    }
+    /* the landmark summaries of this (b, kv head) */
+    for (int64_t c = 0; c < nc; ++c) {
+      const float* lq = LQ + (bh * nc + c) * d;
+      const float* kc = Kbh + c * C * d;
+      const double* kpc = kp + (bh * nc + c) * d;
+      const double* dkpc = dkp + (bh * nc + c) * d;
+      const double dbpc = dbp[bh * nc + c];
+      double m = -INFINITY;
+      for (int64_t j = 0; j < C; ++j) {
+        z[j] = tau * dot_fd(lq, kc + j * d, d);
+        if (z[j] > m) m = z[j];
+      }
+      double Zl = 0.0;
+      for (int64_t j = 0; j < C; ++j) Zl += exp(z[j] - m);
+      double zbar = 0.0;
+      for (int64_t j = 0; j < C; ++j) zbar += exp(z[j] - m) / Zl * z[j];
+      double* dlq = dLQ + (bh * nc + c) * d;
+      for (int64_t t = 0; t < d; ++t) dlq[t] = 0.0;
+      for (int64_t j = 0; j < C; ++j) {
+        const double pj = exp(z[j] - m) / Zl;
+        double proj = 0.0;
+        for (int64_t t = 0; t < d; ++t) proj += dkpc[t] * ((double)kc[j * d + t] - kpc[t]);
+        const double dz = pj * proj - dbpc * pj * (z[j] - zbar);
+        double* dkj = dK + (bh * N + c * C + j) * d;
+        for (int64_t t = 0; t < d; ++t) {
+          dlq[t] += tau * dz * (double)kc[j * d + t];
+          dkj[t] += tau * dz * (double)lq[t] + pj * dkpc[t];
+        }
+      }
+    }
+    free(br);
+    free(z);
+    free(o);
+    free(Orow);
+  }
+  free(kp);
+  free(bp);
+  free(dkp);
+  free(dbp);
+}
+
 int hils_oracle_max_threads(void) {
 #ifdef _OPENMP
   extern int omp_get_max_threads(void);

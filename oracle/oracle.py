@@ -56,6 +56,7 @@ def _load():
         lib.hils_oracle_attend.argtypes = [P, P, P, P, P, ctypes.c_int64, P, P, P, P, P, P,
                                            ctypes.c_int64, ctypes.c_int, P, P]
         lib.hils_oracle_qcal.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P, P, P]
+        lib.hils_oracle_backward.argtypes = [P, P, P, P, P, P, P, ctypes.c_int64, P, P, P, P, P, P]
         lib.hils_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -180,6 +181,27 @@ class Oracle:
                                      _p(rows.b), _p(rows.hq), _p(rows.pos), _p(rows.q), _p(qscore), _p(ids),
                                      ids.shape[1], int(score_mode), _p(O), _p(lse))
         return O, lse
+
+    def backward(self, Q, Kt, Vt, LQ, ids, dO, Qs=None):
+        """Gradients of <dO, O> for a fixed selection ids [B,Hq,N,Kids]: dQ
+        (attention query, plus the scoring-query part unless Qs is given),
+        dQs (the scoring query's, when Qs is given), dK, dV, dLQ (double)."""
+        Q, Kt, Vt, LQ, dO = _f32(Q), _f32(Kt), _f32(Vt), _f32(LQ), _f32(dO)
+        B, Hq, Hkv, N, d, nc = self.B, self.Hq, self.Hkv, self.N, self.d, self.nc
+        assert Q.shape == (B, Hq, N, d) and dO.shape == Q.shape
+        assert Kt.shape == (B, Hkv, N, d) and Vt.shape == Kt.shape and LQ.shape == (B, Hkv, nc, d)
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        assert ids.shape[:3] == (B, Hq, N)
+        if Qs is not None:
+            Qs = _f32(Qs)
+            assert Qs.shape == Q.shape
+        dQ = np.empty((B, Hq, N, d))
+        dQs = np.empty((B, Hq, N, d)) if Qs is not None else None
+        dK, dV = np.empty((B, Hkv, N, d)), np.empty((B, Hkv, N, d))
+        dLQ = np.empty((B, Hkv, nc, d))
+        self._lib.hils_oracle_backward(ctypes.byref(self._d), _p(Q), _p(Qs), _p(Kt), _p(Vt), _p(LQ), _p(ids),
+                                       ids.shape[3], _p(dO), _p(dQ), _p(dQs), _p(dK), _p(dV), _p(dLQ))
+        return dict(dQ=dQ, dQs=dQs, dK=dK, dV=dV, dLQ=dLQ)
 
     def prefill_rows(self, Q, Kt, Vt, kp, bp, flat_rows):
         """Select + attend for the given flat rows of a prefill."""

@@ -42,12 +42,25 @@ MUTANTS = {
     "fusion_ignores_scoring_query": ("const float* qs = qscore ? qscore + r * d : q;", "const float* qs = q;"),
 }
 
+# mistakes in the backward pass, rejected by tests/test_oracle_backward.py
+BWD_MUTANTS = {
+    "bwd_no_compressed_key_gradient": ("dkp[(bh * nc + cc) * d + t] += tau * du * (double)qs[t];",
+                                       "dkp[(bh * nc + cc) * d + t] += 0.0;"),
+    "bwd_no_bias_gradient": ("dbp[bh * nc + cc] += du;", "dbp[bh * nc + cc] += 0.0;"),
+    "bwd_window_without_score_term": ("if (br[c].chunk < 0) dz += du * pj;", "(void)du;"),
+    "bwd_entropy_sign": ("const double dz = pj * proj - dbpc * pj * (z[j] - zbar);",
+                         "const double dz = pj * proj + dbpc * pj * (z[j] - zbar);"),
+    "bwd_summary_value_path": ("dkj[t] += tau * dz * (double)lq[t] + pj * dkpc[t];",
+                               "dkj[t] += tau * dz * (double)lq[t];"),
+    "bwd_score_uses_attention_query": ("dqs[t] += tau * du * kp[(bh * nc + cc) * d + t];",
+                                       "dqs[t] += tau * du * (double)Kbh[cc * C * d + t];"),
+    "bwd_value_weight_unfused": ("dvj[t] += a * pj * (double)gr[t];", "dvj[t] += pj * (double)gr[t];"),
+}
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name):
-    old, new = MUTANTS[name]
+
+def run_pins_on_mutant(old, new, pin_file):
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site of {name} not unique"
+    assert src.count(old) == 1, f"mutation site not unique: {old[:60]}"
     with tempfile.TemporaryDirectory() as tmp:
         cfile = os.path.join(tmp, "mutant.c")
         lib = os.path.join(tmp, "libmutant.so")
@@ -56,6 +69,18 @@ def test_pins_reject_mutant(name):
                                cfile, "-o", lib, "-lm"])
         env = dict(os.environ, HILS_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
         r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle.py")],
+                            os.path.join(ROOT, "tests", pin_file)],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-        assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+        return r
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name):
+    r = run_pins_on_mutant(*MUTANTS[name], "test_oracle.py")
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_pins_reject_mutant(name):
+    r = run_pins_on_mutant(*BWD_MUTANTS[name], "test_oracle_backward.py")
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
