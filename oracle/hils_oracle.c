@@ -475,22 +475,23 @@ void hils_oracle_backward(const hils_oracle_dims* D, const float* Q, const float
       const double* kpc = kp + (bh * nc + c) * d;
       const double* dkpc = dkp + (bh * nc + c) * d;
       const double dbpc = dbp[bh * nc + c];
+      double* zl = z;   /* the landmark logits of chunk c */
       double m = -INFINITY;
       for (int64_t j = 0; j < C; ++j) {
-        z[j] = tau * dot_fd(lq, kc + j * d, d);
-        if (z[j] > m) m = z[j];
+        zl[j] = tau * dot_fd(lq, kc + j * d, d);
+        if (zl[j] > m) m = zl[j];
       }
       double Zl = 0.0;
-      for (int64_t j = 0; j < C; ++j) Zl += exp(z[j] - m);
+      for (int64_t j = 0; j < C; ++j) Zl += exp(zl[j] - m);
       double zbar = 0.0;
-      for (int64_t j = 0; j < C; ++j) zbar += exp(z[j] - m) / Zl * z[j];
+      for (int64_t j = 0; j < C; ++j) zbar += exp(zl[j] - m) / Zl * zl[j];
       double* dlq = dLQ + (bh * nc + c) * d;
       for (int64_t t = 0; t < d; ++t) dlq[t] = 0.0;
       for (int64_t j = 0; j < C; ++j) {
-        const double pj = exp(z[j] - m) / Zl;
+        const double pj = exp(zl[j] - m) / Zl;
         double proj = 0.0;
         for (int64_t t = 0; t < d; ++t) proj += dkpc[t] * ((double)kc[j * d + t] - kpc[t]);
-        const double dz = pj * proj - dbpc * pj * (z[j] - zbar);
+        const double dz = pj * proj - dbpc * pj * (zl[j] - zbar);
         double* dkj = dK + (bh * N + c * C + j) * d;
         for (int64_t t = 0; t < d; ++t) {
           dlq[t] += tau * dz * (double)kc[j * d + t];

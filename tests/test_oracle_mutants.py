@@ -48,8 +48,8 @@ BWD_MUTANTS = {
                                        "dkp[(bh * nc + cc) * d + t] += 0.0;"),
     "bwd_no_bias_gradient": ("dbp[bh * nc + cc] += du;", "dbp[bh * nc + cc] += 0.0;"),
     "bwd_window_without_score_term": ("if (br[c].chunk < 0) dz += du * pj;", "(void)du;"),
-    "bwd_entropy_sign": ("const double dz = pj * proj - dbpc * pj * (z[j] - zbar);",
-                         "const double dz = pj * proj + dbpc * pj * (z[j] - zbar);"),
+    "bwd_entropy_sign": ("const double dz = pj * proj - dbpc * pj * (zl[j] - zbar);",
+                         "const double dz = pj * proj + dbpc * pj * (zl[j] - zbar);"),
     "bwd_summary_value_path": ("dkj[t] += tau * dz * (double)lq[t] + pj * dkpc[t];",
                                "dkj[t] += tau * dz * (double)lq[t];"),
     "bwd_score_uses_attention_query": ("dqs[t] += tau * du * kp[(bh * nc + cc) * d + t];",
