@@ -17,6 +17,7 @@
 #include "prefill_cc.cuh"
 #include "prefill_local.cuh"
 #include "qcal.cuh"
+#include "backward.cuh"
 
 using namespace hils;
 
@@ -180,24 +181,32 @@ bool cc_supported(const hils_dims* d) {
          rows * d->topk < (int64_t(1) << 31);
 }
 
-CcPlan cc_plan(const hils_dims* d) {
-  CcPlan P;
+// Sizes of the chunk-centric index over (kv head, window, chunk) keys.
+CcDims make_cc_dims(const hils_dims* d) {
+  CcDims c;
   const int64_t N = d->seqlen, D = d->head_dim, G = d->heads_q / d->heads_kv;
-  P.c.n_tok = N;
-  P.c.nc = N / kChunk;
-  P.c.Hq = d->heads_q;
-  P.c.Hkv = d->heads_kv;
-  P.c.G = int(G);
-  P.c.K = d->topk;
-  P.c.wm1 = window_wm1(d);
-  P.c.tau = 1.f / sqrtf(float(D));
+  c.n_tok = N;
+  c.nc = N / kChunk;
+  c.Hq = d->heads_q;
+  c.Hkv = d->heads_kv;
+  c.G = int(G);
+  c.K = d->topk;
+  c.wm1 = window_wm1(d);
+  c.tau = 1.f / sqrtf(float(D));
   // window: the fp32 accumulators and bf16 queries of one window of one kv head
   // (G x W positions) stay within 64 MiB of L2
   int shift = 6;
   while ((int64_t(1) << (shift + 1)) <= N && G * (int64_t(1) << (shift + 1)) * D * 6 <= (int64_t(64) << 20)) ++shift;
-  P.c.win_shift = shift;
-  P.c.n_win = int((N + (int64_t(1) << shift) - 1) >> shift);
-  P.c.n_keys = int64_t(d->batch) * d->heads_kv * P.c.n_win * P.c.nc;
+  c.win_shift = shift;
+  c.n_win = int((N + (int64_t(1) << shift) - 1) >> shift);
+  c.n_keys = int64_t(d->batch) * d->heads_kv * c.n_win * c.nc;
+  return c;
+}
+
+CcPlan cc_plan(const hils_dims* d) {
+  CcPlan P;
+  const int64_t N = d->seqlen, D = d->head_dim, G = d->heads_q / d->heads_kv;
+  P.c = make_cc_dims(d);
   P.rows = int64_t(d->batch) * d->heads_q * N;
   P.n_slots = P.rows * d->topk;
   P.P = int(128 / G);
@@ -314,6 +323,113 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   const int64_t n8 = P.rows * D / 8;
   cc_final_kernel<D><<<unsigned((n8 + 255) / 256), 256, 0, st>>>(oacc, static_cast<__nv_bfloat16*>(o), n8);
   return launched(9);
+}
+
+// ---------------------------------------------------------------- backward
+struct BwdPlan {
+  CcDims c;
+  int64_t rows, n_slots, max_items, n_scan_blocks, n_units;
+  size_t off_rowstat, off_dvec, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_erow,
+      off_efac, off_dkp, off_dbp, total;
+};
+
+BwdPlan bwd_plan(const hils_dims* d) {
+  BwdPlan P;
+  P.c = make_cc_dims(d);
+  const int64_t D = d->head_dim;
+  P.rows = int64_t(d->batch) * d->heads_q * d->seqlen;
+  P.n_slots = P.rows * d->topk;
+  P.n_units = int64_t(d->batch) * d->heads_kv * P.c.nc;
+  P.n_scan_blocks = (P.c.n_keys + kScanBlock - 1) / kScanBlock;
+  P.max_items = P.n_slots / kCcTileRows + P.c.n_keys + 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
+  P.off_rowstat = take(sizeof(float) * P.rows);
+  P.off_dvec = take(sizeof(float) * P.rows);
+  P.off_counts = take(sizeof(int32_t) * P.c.n_keys);
+  P.off_ranks = take(sizeof(int32_t) * P.n_slots);
+  P.off_offsets = take(sizeof(int64_t) * (P.c.n_keys + 1));
+  P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
+  P.off_items = take(sizeof(int4) * P.max_items);
+  P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
+  P.off_erow = take(sizeof(int32_t) * (P.n_slots + kCcTileRows));
+  P.off_efac = take(sizeof(float) * (P.n_slots + kCcTileRows));
+  P.off_dkp = take(sizeof(float) * P.n_units * D);
+  P.off_dbp = take(sizeof(float) * P.n_units);
+  P.total = off;
+  return P;
+}
+
+template <typename T, int D>
+int launch_backward(const hils_dims* d, const void* q, const void* q_score, const void* k, const void* v,
+                    const void* lq, const float* kprime, const int32_t* ids, const float* scores, const float* lse_w,
+                    const void* o, const void* d_o, float* dq, float* dq_score, float* dk, float* dv, float* dlq,
+                    void* ws, cudaStream_t st) {
+  using BT = BwdTiles<D>;
+  const BwdPlan P = bwd_plan(d);
+  char* base = static_cast<char*>(ws);
+  float* rowstat = reinterpret_cast<float*>(base + P.off_rowstat);
+  float* dvec = reinterpret_cast<float*>(base + P.off_dvec);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + P.off_counts);
+  int32_t* ranks = reinterpret_cast<int32_t*>(base + P.off_ranks);
+  int64_t* offsets = reinterpret_cast<int64_t*>(base + P.off_offsets);
+  int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
+  int4* items = reinterpret_cast<int4*>(base + P.off_items);
+  int64_t* sums = reinterpret_cast<int64_t*>(base + P.off_sums);
+  int32_t* e_row = reinterpret_cast<int32_t*>(base + P.off_erow);
+  float* e_fac = reinterpret_cast<float*>(base + P.off_efac);
+  float* dkp = reinterpret_cast<float*>(base + P.off_dkp);
+  float* dbp = reinterpret_cast<float*>(base + P.off_dbp);
+  const int64_t N = d->seqlen, kv_elems = int64_t(d->batch) * d->heads_kv * N * D;
+  const int G = d->heads_q / d->heads_kv;
+  const T* tq = static_cast<const T*>(q);
+  const T* tk = static_cast<const T*>(k);
+  const T* tv = static_cast<const T*>(v);
+  const T* tdo = static_cast<const T*>(d_o);
+  if (cudaMemsetAsync(dk, 0, sizeof(float) * kv_elems, st) != cudaSuccess ||
+      cudaMemsetAsync(dv, 0, sizeof(float) * kv_elems, st) != cudaSuccess ||
+      cudaMemsetAsync(dkp, 0, sizeof(float) * P.n_units * (D + 0), st) != cudaSuccess ||
+      cudaMemsetAsync(dbp, 0, sizeof(float) * P.n_units, st) != cudaSuccess ||
+      cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess ||
+      cudaMemsetAsync(base + P.off_erow + sizeof(int32_t) * P.n_slots, 0, sizeof(int32_t) * kCcTileRows, st) !=
+          cudaSuccess)
+    return HILS_ERR_CUDA;
+  if (dq_score && cudaMemsetAsync(dq_score, 0, sizeof(float) * P.rows * D, st) != cudaSuccess) return HILS_ERR_CUDA;
+  bwd_prep_kernel<T, D><<<unsigned((P.rows * 32 + 127) / 128), 128, 0, st>>>(
+      ids, scores, lse_w, static_cast<const T*>(o), tdo, N, d->topk, P.c.wm1, P.rows, rowstat, dvec);
+  // the forward's index: per (kv head, window, chunk) its (row, slot) pairs and s^ - M'
+  const size_t hist_bytes = sizeof(int32_t) * size_t(P.c.nc);
+  if (N % kCountRows == 0 && (int64_t(1) << P.c.win_shift) % kCountRows == 0 && hist_bytes <= 96 * 1024) {
+    constexpr auto cfn = cc_count_kernel;
+    if (hist_bytes > 48 * 1024 && set_smem_max<cfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    cfn<<<unsigned(P.rows / kCountRows), kCountThreads, hist_bytes, st>>>(ids, counts, ranks, P.c);
+  } else {
+    cc_count_direct_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, counts, ranks, P.c, P.n_slots);
+  }
+  const unsigned nsb = unsigned(P.n_scan_blocks);
+  cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
+  cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
+  cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
+  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_row, e_fac,
+                                                                     P.c, P.n_slots);
+  const float tau = 1.f / sqrtf(float(D));
+  const size_t smem_w = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(BT::SUB) * D * 4;
+  constexpr auto wfn = bwd_window_kernel<T, D>;
+  if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
+  wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
+      tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
+  const size_t smem_c = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(2 * D + 4) * 4;
+  constexpr auto cfn2 = bwd_chunk_kernel<T, D>;
+  if (set_smem_max<cfn2>() != cudaSuccess) return HILS_ERR_CUDA;
+  cfn2<<<unsigned(sm_count() * 2), BT::THREADS, smem_c, st>>>(
+      tq, static_cast<const T*>(q_score), tk, tv, tdo, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq,
+      dq_score ? dq_score : dq, dk, dv, dkp, dbp);
+  const size_t smem_s = size_t(4) * (kChunk * BT::KS + 3 * D) * 4;
+  constexpr auto sfn = bwd_summary_kernel<T, D>;
+  if (set_smem_max<sfn>() != cudaSuccess) return HILS_ERR_CUDA;
+  sfn<<<unsigned((P.n_units + 3) / 4), 128, smem_s, st>>>(tk, static_cast<const T*>(lq), kprime, dkp, dbp, N, P.c.nc,
+                                                          P.n_units, tau, dk, dlq);
+  return launched(10);
 }
 
 template <typename T, int D>
@@ -595,6 +711,43 @@ int hils_query_calibrate(const hils_dims* d, const void* q, int64_t n_pos, const
     else qcal_simt_kernel<float, 128><<<blocks, 128, 0, st>>>(qq, wd, wu, rank, n_pos, d->heads_q, rows, out);
   }
   return launched(1);
+}
+
+size_t hils_attn_backward_workspace_bytes(const hils_dims* d) {
+  if (check_dims(d) != HILS_OK) return 0;
+  return bwd_plan(d).total;
+}
+
+int hils_attn_backward(const hils_dims* d, const void* q, const void* q_score, const void* k, const void* v,
+                       const void* lq, const float* kprime, const int32_t* ids, const float* scores,
+                       const float* lse_own, const void* o, const void* d_o, float* dq, float* dq_score, float* dk,
+                       float* dv, float* dlq, void* workspace, size_t workspace_bytes, hils_stream_t stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(lq) || !ptr_ok(kprime) || !ptr_ok(ids) || !ptr_ok(scores) ||
+      !ptr_ok(lse_own) || !ptr_ok(o) || !ptr_ok(d_o) || !ptr_ok(dq) || !ptr_ok(dk) || !ptr_ok(dv) || !ptr_ok(dlq) ||
+      !ptr_ok(workspace))
+    return HILS_ERR_INVALID_ARGUMENT;
+  if ((q_score != nullptr && !aligned16(q_score)) || (dq_score != nullptr && !aligned16(dq_score)))
+    return HILS_ERR_INVALID_ARGUMENT;
+  const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
+  if (rows * d->topk >= (int64_t(1) << 31) || int64_t(d->batch) * d->heads_kv * d->seqlen >= (int64_t(1) << 31))
+    return HILS_ERR_UNSUPPORTED;
+  if (int64_t(d->batch) * d->heads_q > 65535) return HILS_ERR_UNSUPPORTED;
+  if (workspace_bytes < hils_attn_backward_workspace_bytes(d)) return HILS_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HILS_BF16) {
+    if (d->head_dim == 64)
+      return launch_backward<__nv_bfloat16, 64>(d, q, q_score, k, v, lq, kprime, ids, scores, lse_own, o, d_o, dq,
+                                                dq_score, dk, dv, dlq, workspace, st);
+    return launch_backward<__nv_bfloat16, 128>(d, q, q_score, k, v, lq, kprime, ids, scores, lse_own, o, d_o, dq,
+                                               dq_score, dk, dv, dlq, workspace, st);
+  }
+  if (d->head_dim == 64)
+    return launch_backward<float, 64>(d, q, q_score, k, v, lq, kprime, ids, scores, lse_own, o, d_o, dq, dq_score, dk,
+                                      dv, dlq, workspace, st);
+  return launch_backward<float, 128>(d, q, q_score, k, v, lq, kprime, ids, scores, lse_own, o, d_o, dq, dq_score, dk,
+                                     dv, dlq, workspace, st);
 }
 
 }  // extern "C"

@@ -23,6 +23,7 @@ EXPORTS = ("hils_landmark_summary", "hils_kprime_mma_bytes", "hils_select", "hil
            "hils_attn_prefill",
            "hils_decode_workspace_bytes", "hils_attn_decode", "hils_attn_decode_fixed_scratch",
            "hils_landmark_summary_paged", "hils_attn_decode_paged", "hils_query_calibrate", "hils_attn_decode_qcal",
+           "hils_attn_backward_workspace_bytes", "hils_attn_backward",
            "hils_get_status", "hils_selftest_bounded_wait", "hils_strerror", "hils_kernel_launches")
 DECODE_FIXED_SCRATCH_BYTES = 16 << 20
 
@@ -66,6 +67,9 @@ def lib():
         L.hils_attn_decode_paged.argtypes = [D, P, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_query_calibrate.argtypes = [D, P, I64, P, P, ctypes.c_int32, P, P]
         L.hils_attn_decode_qcal.argtypes = [D, P, P, P, P, P, I64, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_attn_backward_workspace_bytes.argtypes = [D]
+        L.hils_attn_backward_workspace_bytes.restype = SZ
+        L.hils_attn_backward.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
         L.hils_selftest_bounded_wait.argtypes = [ctypes.c_int32, P]
         L.hils_strerror.argtypes = [ctypes.c_int]
@@ -211,6 +215,20 @@ def hils_attn_decode_qcal(dims, q, q_score, k_cache, v_cache, page_table, n_page
                                        int(nbytes), _stream(stream)))
 
 
+def hils_attn_backward_workspace_bytes(dims) -> int:
+    return int(lib().hils_attn_backward_workspace_bytes(ctypes.byref(dims)))
+
+
+def hils_attn_backward(dims, q, q_score, k, v, lq, kprime, ids, scores, lse_own, o, d_o, dq, dq_score, dk, dv, dlq,
+                       workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("hils_attn_backward",
+           lib().hils_attn_backward(ctypes.byref(dims), _ptr(q), _ptr(q_score), _ptr(k), _ptr(v), _ptr(lq),
+                                    _ptr(kprime), _ptr(ids), _ptr(scores), _ptr(lse_own), _ptr(o), _ptr(d_o),
+                                    _ptr(dq), _ptr(dq_score), _ptr(dk), _ptr(dv), _ptr(dlq), _ptr(workspace),
+                                    int(nbytes), _stream(stream)))
+
+
 def hils_get_status(stream=None) -> int:
     v = ctypes.c_int32(0)
     _check("hils_get_status", lib().hils_get_status(ctypes.byref(v), _stream(stream)))
@@ -316,6 +334,22 @@ def decode_step_qcal(q, q_score, k_cache, v_cache, summ: Summary, seqlens, topk,
     hils_attn_decode_qcal(dims, q, q_score, k_cache, v_cache, None, 0, summ.kprime, summ.bprime, summ.kprime_mma,
                           seqlens, o, ids, scores, workspace, stream=stream)
     return o, ids, scores
+
+
+def backward(q, k, v, lq, aux, o, d_o, topk, q_score=None, window=0, stream=None):
+    """Gradients (fp32) of a prefill made by prefill()/prefill_qcal() with
+    return_all=True: returns dict(dq, dq_score (with q_score), dk, dv, dlq)."""
+    dims = dims_for(q, k, topk, window)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = dict(dq=torch.empty((B, Hq, N, d), **f32), dk=torch.empty((B, Hkv, N, d), **f32),
+             dv=torch.empty((B, Hkv, N, d), **f32), dlq=torch.empty((B, Hkv, N // CHUNK, d), **f32))
+    g["dq_score"] = torch.empty((B, Hq, N, d), **f32) if q_score is not None else None
+    ws = torch.empty((hils_attn_backward_workspace_bytes(dims),), dtype=torch.uint8, device=q.device)
+    hils_attn_backward(dims, q, q_score, k, v, lq, aux["summary"].kprime, aux["ids"], aux["scores"], aux["lse_own"], o,
+                       d_o, g["dq"], g["dq_score"], g["dk"], g["dv"], g["dlq"], ws, stream=stream)
+    return g
 
 
 def decode_step(q, k_cache, v_cache, summ: Summary, seqlens, topk, workspace=None, stream=None, window=0):

@@ -285,6 +285,44 @@ int hils_attn_decode_qcal(const hils_dims* dims, const void* q, const void* q_sc
                           const int32_t* seqlens, void* o, int32_t* ids_out, float* scores_out,
                           void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
+/* Device workspace bytes hils_attn_backward needs for these dims. */
+size_t hils_attn_backward_workspace_bytes(const hils_dims* dims);
+
+/*
+ * Backward pass of the prefill (hils_landmark_summary + the chunk scores of
+ * hils_select + hils_attn_prefill) for the selection the forward made --
+ * [AIT-Meth]: the chunk score is part of the forward attention, so the loss
+ * gradient reaches the landmark queries through k', b' and the scoring query
+ * (Q-Cal) through s^; the top-K choice itself is not differentiated.
+ * Given dO = dL/dO it returns the gradients of L with respect to q, k, v and
+ * lq.  Per row, with M' the fusion normaliser and a_c = exp(u_c - M'):
+ *   selected chunk c: dz_j = a_c p_j (<dO, v_j> - <dO, o_c>),
+ *                     du_c = a_c (<dO, o_c> - <dO, O>) -> q_score, k', b'
+ *   window:           dz_j = P_ij (<dO, v_j> - <dO, O>)
+ *   dq += tau dz_j k_j, dk_j += tau dz_j q, dv_j += a_c p_j dO, and the
+ *   landmark softmax passes dk', db' on to k and lq.
+ *   q, k, v, lq  the forward's inputs (dtype, layouts as in the forward)
+ *   q_score      the scoring query the selection used ([B,Hq,N,d] dtype, the
+ *                output of hils_query_calibrate), or NULL when it was q
+ *   kprime       fp32 [B,Hkv,nc,d] from hils_landmark_summary
+ *   ids, scores  [B,Hq,N,K] from hils_select
+ *   lse_own      [B,Hq,N] fp32 from hils_attn_prefill (required here)
+ *   o, d_o       [B,Hq,N,d] dtype: the forward output and dL/dO
+ *   dq           [B,Hq,N,d] fp32 out: through the attention, plus through
+ *                the chunk scores when dq_score is NULL
+ *   dq_score     [B,Hq,N,d] fp32 out (nullable): the scoring query's gradient
+ *   dk, dv       [B,Hkv,N,d] fp32 out;  dlq [B,Hkv,nc,d] fp32 out
+ * Outputs are overwritten.  fp32 arithmetic on CUDA cores; gradients are
+ * summed with fp32 atomics (the order of the sums is not fixed).  Any G;
+ * B * Hq <= 65535.  Ids outside a row's candidates are recorded as
+ * HILS_ERR_DEVICE_BOUNDS and skipped.
+ */
+int hils_attn_backward(const hils_dims* dims, const void* q, const void* q_score, const void* k, const void* v,
+                       const void* lq, const float* kprime, const int32_t* ids, const float* scores,
+                       const float* lse_own, const void* o, const void* d_o, float* dq, float* dq_score,
+                       float* dk, float* dv, float* dlq, void* workspace, size_t workspace_bytes,
+                       hils_stream_t stream);
+
 /*
  * Synchronises `stream`, copies the device status word of the current device
  * into *host_status (HILS_OK or a HILS_ERR_DEVICE_* code recorded by a kernel

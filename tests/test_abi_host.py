@@ -113,6 +113,19 @@ def test_qcal_arguments_rejected_before_launch(lib):
                                      big, None) == 1      # a page table needs pages
 
 
+def test_backward_arguments_rejected_before_launch(lib):
+    d = dims()
+    p = ctypes.c_void_p(256)
+    need = hils.hils_attn_backward_workspace_bytes(d)
+    assert need > 0
+    args = [p] * 11
+    # q_score and dq_score may be NULL; every other pointer is required
+    assert lib.hils_attn_backward(ctypes.byref(d), p, None, p, p, p, p, p, p, None, p, p, p, None, p, p, p, p,
+                                  need, None) == 1
+    assert lib.hils_attn_backward(ctypes.byref(d), p, None, p, p, p, p, p, p, p, p, p, p, None, p, p, p, p,
+                                  need - 1, None) == 4
+
+
 def test_strerror(lib):
     for code in range(7):
         assert len(hils.strerror(code)) >= 2
