@@ -439,6 +439,95 @@ def decode_selected_bytes(ids, w):
     return total
 
 
+def run_backward(args, w, rank, world, local_rank):
+    """One backward step (gradients of q, k, v, lq for the forward's
+    selection) per iteration, after one untimed forward."""
+    import torch
+    from chunk_wise_sparse_b200 import hils
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = generate(w)
+
+    def to_dev(name):
+        bits = getattr(inp, name + "_bits")
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(getattr(inp, name + "_f32")).to(dev)
+
+    q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
+    B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
+    o, aux = hils.prefill(q, k, v, lq, K, return_all=True, window=w.window)
+    d_o = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(w.seed)).to(q.dtype)
+    dims = hils.dims_for(q, k, K, w.window)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk = torch.empty((B, Hq, N, d), **f32), torch.empty((B, Hkv, N, d), **f32)
+    dv, dlq = torch.empty((B, Hkv, N, d), **f32), torch.empty((B, Hkv, N // 64, d), **f32)
+    ws = torch.empty((hils.hils_attn_backward_workspace_bytes(dims),), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = None if inputs_exceed_l2(w) else torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+
+    def step():
+        hils.hils_attn_backward(dims, q, None, k, v, lq, aux["summary"].kprime, aux["ids"], aux["scores"],
+                                aux["lse_own"], o, d_o, dq, None, dk, dv, dlq, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hils.hils_get_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = hils.hils_kernel_launches()
+    ms = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    launches = hils.hils_kernel_launches() - launches0
+    clk = clocks.stop()
+    if hils.hils_get_status() != 0:
+        raise RuntimeError("device status error during the timed steps")
+    if world > 1:
+        dist.barrier()
+    ms_step = max_over_ranks(float(np.mean(ms)), world, dev)
+    if rank != 0:
+        return
+    # algorithmic work: per attended key 10d flops (the logits and <dO, v_j>
+    # again, dq, dk, dv), per key of a summary 10d more
+    wc = max(1, w.window // w.C)
+    i = np.arange(N, dtype=np.int64)
+    n_cand = np.maximum(0, i // w.C - (wc - 1))
+    keys = np.minimum(K, n_cand) * w.C + (i - n_cand * w.C) + 1
+    flops = 10 * d * Hq * B * int(keys.sum()) + 10 * d * B * Hkv * N
+    props = torch.cuda.get_device_properties(dev)
+    max_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+    peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+    ach = flops / (ms_step / 1e3) / 1e12
+    line = {
+        "metric": "HiLS backward tokens/s (gradients of q, k, v, lq for a fixed selection)",
+        "value": job_throughput(world, B * N, ms_step), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (bf16 inputs)" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(w, world),
+        "roofline": {"kernel": "backward (whole call)", "bound": "alu", "achieved": ach, "peak": peak,
+                     "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                     "peak_source": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {max_mhz:.0f} MHz"},
+        "gpu_launches": int(launches), "clocks": clk, "e2e": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_decode(args, w, rank, world, local_rank):
     """One decode step per step for every sequence of the batch; the landmark
     summaries of the cache are built in the untimed setup.  L2 is flushed
@@ -547,6 +636,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
+    ap.add_argument("--backward", action="store_true", help="time the backward pass of a prefill workload")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -562,7 +652,9 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        if w.kind == "decode":
+        if args.backward:
+            run_backward(args, w, rank, world, local_rank)
+        elif w.kind == "decode":
             run_decode(args, w, rank, world, local_rank)
         else:
             run_ours(args, w, rank, world, local_rank)
