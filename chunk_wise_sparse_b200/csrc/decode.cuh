@@ -236,6 +236,99 @@ decode_topk_kernel(const float* __restrict__ ws_scores, const int32_t* __restric
   }
 }
 
+// D2 for rows of at most 256 * IT candidates: the same radix select and
+// stable compaction with each thread's contiguous segment of order keys held
+// in registers, so the scores are read once instead of once per pass.
+template <int IT>
+__global__ void __launch_bounds__(256)
+decode_topk_reg_kernel(const float* __restrict__ ws_scores, const int32_t* __restrict__ seqlens, int64_t cap,
+                       int64_t nc, int Hq, int K, int32_t* __restrict__ sel_ids, float* __restrict__ sel_scores,
+                       int wm1) {
+  __shared__ uint32_t hist[256];
+  __shared__ int warp_tot[8];
+  __shared__ uint32_t s_digit, s_above;
+  const int row = blockIdx.x, b = row / Hq, tid = threadIdx.x;
+  int64_t n = decode_own_chunk(seqlens, b, cap) - wm1;   // candidates
+  if (n < 0) n = 0;
+  const float* sc = ws_scores + int64_t(row) * nc;
+  int32_t* oid = sel_ids + int64_t(row) * K;
+  float* osc = sel_scores + int64_t(row) * K;
+  if (n <= K) {
+    for (int t = tid; t < K; t += 256) {
+      oid[t] = t < n ? t : -1;
+      osc[t] = t < n ? sc[t] : -INFINITY;
+    }
+    return;
+  }
+  const int seg = int((n + 255) / 256);   // <= IT
+  const int s0 = tid * seg;
+  const int cnt = s0 >= n ? 0 : (s0 + seg <= n ? seg : int(n - s0));
+  uint32_t key[IT];
+  float val[IT];
+#pragma unroll
+  for (int e = 0; e < IT; ++e) {
+    val[e] = e < cnt ? sc[s0 + e] : -INFINITY;
+    key[e] = order_key(val[e]);
+  }
+  uint32_t prefix = 0, mask = 0;
+  int krem = K;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    hist[tid] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < IT; ++e)
+      if (e < cnt && (key[e] & mask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1u);
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t loc[8], lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { loc[j] = hist[255 - 8 * tid - j]; lsum += loc[j]; }
+      uint32_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const uint32_t excl = incl - lsum;
+      if (excl < uint32_t(krem) && uint32_t(krem) <= incl) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + loc[j] >= uint32_t(krem)) { s_digit = 255 - 8 * tid - j; s_above = cum; break; }
+          cum += loc[j];
+        }
+      }
+    }
+    __syncthreads();
+    krem -= int(s_above);
+    prefix |= s_digit << shift;
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  // prefix = key of the K-th largest score; take every key above it and the
+  // krem lowest-id keys equal to it, in chunk order
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < IT; ++e) {
+    gt += e < cnt && key[e] > prefix;
+    eq += e < cnt && key[e] == prefix;
+  }
+  int tot;
+  const int eq_before = block_exclusive_scan256(eq, warp_tot, tot);
+  int take_eq = krem - eq_before;
+  take_eq = take_eq < 0 ? 0 : (take_eq > eq ? eq : take_eq);
+  int pos = block_exclusive_scan256(gt + take_eq, warp_tot, tot);
+  int eq_seen = 0;
+#pragma unroll
+  for (int e = 0; e < IT; ++e) {
+    if (e >= cnt) continue;
+    bool take = key[e] > prefix;
+    if (key[e] == prefix) take = eq_seen++ < take_eq;
+    if (take && pos < K) { oid[pos] = int32_t(s0 + e); osc[pos] = val[e]; ++pos; }
+  }
+}
+
 // D3, grouped by kv head: the G query heads of a kv head select overlapping
 // chunk sets, so each distinct chunk is read once and attended by all heads
 // that kept it.  One CTA per candidate slot (g, k) of the (b, kv head)'s
@@ -447,46 +540,60 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   }
 }
 
+// D4: one CTA of D threads per row, thread t owns output dim t; the slots'
+// partial rows are read 8 at a time with all loads in flight (the per-slot
+// work is one fused multiply-add, so the kernel is load-latency bound).
 template <typename T, int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(D)
 decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict__ part_o,
                       const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int K,
                       const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
                       T* __restrict__ o, int32_t* __restrict__ ids_out, float* __restrict__ scores_out,
                       int64_t n_rows, int wm1) {
-  constexpr int EL = D / 32;   // output elements per lane
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= n_rows) return;
+  __shared__ float s_w[kMaxTopK + 17];   // fusion weight of each slot
+  __shared__ float s_z;
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.x;
   const int b = int(row / Hq);
   const bool valid = decode_own_chunk(seqlens, b, cap) >= 0;
   const int PS = K + wm1 + 1;
-  float M = -INFINITY;
-  for (int s = 0; s < PS; ++s) M = fmaxf(M, part_u[row * PS + s]);
-  float Z = 0.f, acc[EL];
+  const float* pu = part_u + row * PS;
+  if (t < 32) {
+    float M = -INFINITY;
+    for (int s = t; s < PS; s += 32) M = fmaxf(M, pu[s]);
 #pragma unroll
-  for (int e = 0; e < EL; ++e) acc[e] = 0.f;
-  if (valid) {
-    for (int s = 0; s < PS; ++s) {
-      const float u = part_u[row * PS + s];
-      if (u == -INFINITY) continue;
-      const float w = expf(u - M);
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float Z = 0.f;
+    for (int s = t; s < PS; s += 32) {
+      const float u = pu[s];
+      const float w = (valid && u != -INFINITY) ? expf(u - M) : 0.f;
+      s_w[s] = w;
       Z += w;
-      const float* po = part_o + (row * PS + s) * D + lane * EL;
-#pragma unroll
-      for (int e = 0; e < EL; ++e) acc[e] += w * po[e];
     }
-  }
-  const float inv = Z > 0.f ? 1.f / Z : 0.f;
 #pragma unroll
-  for (int e = 0; e < EL; ++e) {
-    const float x = acc[e] * inv;
-    if constexpr (sizeof(T) == 2) o[row * D + lane * EL + e] = __float2bfloat16_rn(x);
-    else o[row * D + lane * EL + e] = x;
+    for (int off = 16; off; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+    if (t == 0) s_z = Z;
   }
-  for (int t = lane; t < K; t += 32) {
-    if (ids_out) ids_out[row * K + t] = valid ? sel_ids[row * K + t] : -1;
-    if (scores_out) scores_out[row * K + t] = valid ? sel_scores[row * K + t] : -INFINITY;
+  __syncthreads();
+  const float* po = part_o + row * PS * D + t;
+  float acc = 0.f;
+  int s = 0;
+  for (; s + 8 <= PS; s += 8) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = s_w[s + e] != 0.f ? po[int64_t(s + e) * D] : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc = fmaf(s_w[s + e], x[e], acc);
+  }
+  for (; s < PS; ++s)
+    if (s_w[s] != 0.f) acc = fmaf(s_w[s], po[int64_t(s) * D], acc);
+  const float Z = s_z;
+  const float y = Z > 0.f ? acc / Z : 0.f;
+  if constexpr (sizeof(T) == 2) o[row * D + t] = __float2bfloat16_rn(y);
+  else o[row * D + t] = y;
+  for (int k = t; k < K; k += D) {
+    if (ids_out) ids_out[row * K + k] = valid ? sel_ids[row * K + k] : -1;
+    if (scores_out) scores_out[row * K + k] = valid ? sel_scores[row * K + k] : -INFINITY;
   }
 }
 

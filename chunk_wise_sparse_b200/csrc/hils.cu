@@ -487,8 +487,12 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
   k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q_score ? q_score : q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores, wm1);
-  decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
-                                                      ws.sel_scores, wm1);
+  if (nc <= 256 * 16)
+    decode_topk_reg_kernel<16><<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
+                                                                ws.sel_ids, ws.sel_scores, wm1);
+  else
+    decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
+                                                        ws.sel_scores, wm1);
   const size_t smem3 = DecUnion<T, D>::smem(G, K);
   constexpr auto k3 = decode_partial_union_kernel<T, D>;
   if (smem3 > 48 * 1024 && set_smem_max<k3>() != cudaSuccess) return HILS_ERR_CUDA;
@@ -496,7 +500,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   k3<<<g3, 128, smem3, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
       d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, pk, wm1);
-  decode_combine_kernel<T, D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(
+  decode_combine_kernel<T, D><<<unsigned(rows), D, 0, st>>>(
       ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
       ids_out, scores_out, rows, wm1);
   return launched(4);
