@@ -18,6 +18,7 @@
 #include "prefill_local.cuh"
 #include "qcal.cuh"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 
 using namespace hils;
 
@@ -418,12 +419,28 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
   wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
       tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
-  const size_t smem_c = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(2 * D + 4) * 4;
-  constexpr auto cfn2 = bwd_chunk_kernel<T, D>;
-  if (set_smem_max<cfn2>() != cudaSuccess) return HILS_ERR_CUDA;
-  cfn2<<<unsigned(sm_count() * 2), BT::THREADS, smem_c, st>>>(
-      tq, static_cast<const T*>(q_score), tk, tv, tdo, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq,
-      dq_score ? dq_score : dq, dk, dv, dkp, dbp);
+  if (std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
+    // bf16 with the attention query as the scoring query: selected chunks on tensor cores
+    using CT = BwdTc<D>;
+    CUtensorMap mq, mg, mk, mv;
+    const uint64_t kv_rows = uint64_t(d->batch) * d->heads_kv * N;
+    if (!make_map_2d(&mq, q, D, uint64_t(P.rows), D * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mg, d_o, D, uint64_t(P.rows), D * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mk, k, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mv, v, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+      return HILS_ERR_CUDA;
+    constexpr auto tfn = bwd_chunk_tc_kernel<D>;
+    if (set_smem_max<tfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    tfn<<<unsigned(sm_count() * (D == 64 ? 2 : 1)), CT::THREADS, CT::SMEM, st>>>(
+        mq, mg, mk, mv, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq, dk, dv, dkp, dbp);
+  } else {
+    const size_t smem_c = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(2 * D + 4) * 4;
+    constexpr auto cfn2 = bwd_chunk_kernel<T, D>;
+    if (set_smem_max<cfn2>() != cudaSuccess) return HILS_ERR_CUDA;
+    cfn2<<<unsigned(sm_count() * 2), BT::THREADS, smem_c, st>>>(
+        tq, static_cast<const T*>(q_score), tk, tv, tdo, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq,
+        dq_score ? dq_score : dq, dk, dv, dkp, dbp);
+  }
   const size_t smem_s = size_t(4) * (kChunk * BT::KS + 3 * D) * 4;
   constexpr auto sfn = bwd_summary_kernel<T, D>;
   if (set_smem_max<sfn>() != cudaSuccess) return HILS_ERR_CUDA;
