@@ -458,6 +458,7 @@ def run_backward(args, w, rank, world, local_rank):
     q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
     B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
     o, aux = hils.prefill(q, k, v, lq, K, return_all=True, window=w.window)
+    torch.cuda.synchronize()
     d_o = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(w.seed)).to(q.dtype)
     dims = hils.dims_for(q, k, K, w.window)
     f32 = dict(dtype=torch.float32, device=dev)

@@ -419,8 +419,8 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
   wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
       tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
-  // The tensor-core kernel (bwd_chunk_tc_kernel) is not launched: a run of it
-  // stopped answering for minutes without a cause found yet.
+  // The tensor-core kernel (bwd_chunk_tc_kernel) is kept but not launched
+  // until a hang seen with it is explained.
   constexpr bool kUseTensorCoreBackward = false;
   if (kUseTensorCoreBackward && std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
     // bf16 with the attention query as the scoring query: selected chunks on tensor cores
