@@ -45,13 +45,17 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def kernels_sha256():
-    """Hash of the CUDA sources, to tell whether recorded counters still apply."""
+# The sources each recorded kernel is compiled from.
+KERNEL_SOURCES = {"select": ["select_tc.cuh", "sm100.cuh", "common.cuh"]}
+
+
+def kernels_sha256(kernel):
+    """Hash of a kernel's CUDA sources, to tell whether recorded counters still apply."""
     h = hashlib.sha256()
     src = os.path.join(ROOT, "chunk_wise_sparse_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(src, "*.cu")) + glob.glob(os.path.join(src, "*.cuh"))):
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(name.encode())
+        with open(os.path.join(src, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
@@ -65,7 +69,7 @@ def recorded_traffic(kernel, rows):
         return None
     with open(p) as f:
         j = json.load(f)
-    if j.get("kernels_sha256") != kernels_sha256() or kernel not in j.get("per_row_bytes", {}):
+    if kernel not in j.get("per_row_bytes", {}) or j.get("sources_sha256", {}).get(kernel) != kernels_sha256(kernel):
         return None
     return float(j["per_row_bytes"][kernel]) * rows
 
@@ -276,7 +280,7 @@ def run_ours(args, w, rank, world, local_rank):
     names = ["summary"] + (["qcal"] if use_qcal else []) + ["select", "prefill", "decode"]
     n_ev = len(names) + 1
 
-    def step(ev=None):
+    def step_on(q, k, v, lq, qd, ev=None):
         e = [0]
 
         def mark():
@@ -304,6 +308,9 @@ def run_ours(args, w, rank, world, local_rank):
             hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
                                   ws, stream=stream)
         mark()
+
+    def step(ev=None):
+        step_on(q, k, v, lq, qd, ev)
 
     for _ in range(args.warmup):
         step()
@@ -339,41 +346,66 @@ def run_ours(args, w, rank, world, local_rank):
         ms_step = max_over_ranks(float(per.sum(axis=1).mean()), world, dev)
     value = job_throughput(world, B * N, ms_step)
 
-    # end to end through the public API: pinned host inputs -> device -> path -> host result
+    # end to end through the public API: every step copies its inputs from
+    # pinned host memory and reads its outputs back.  Two device input sets:
+    # step i+1's inputs are copied (on a copy stream) while step i computes.
     e2e = None
     if not args.no_e2e:
         host = {n: getattr(inp, n + "_bits") if getattr(inp, n + "_bits") is not None else getattr(inp, n + "_f32")
                 for n in ("q", "k", "v", "lq")}
         pinned = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
                   for n, a in host.items()}
-        dev_t = {"q": q, "k": k, "v": v, "lq": lq}
+        sets = [{"q": q, "k": k, "v": v, "lq": lq, "qd": qd},
+                {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+                 "lq": torch.empty_like(lq), "qd": torch.empty_like(qd)}]
         o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         od_host = torch.empty(od.shape, dtype=od.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values())
         d2h = o_host.numel() * o_host.element_size() + od_host.numel() * od_host.element_size()
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for n, t in pinned.items():
-                dev_t[n].view(torch.int16 if dev_t[n].dtype == torch.bfloat16 else dev_t[n].dtype).copy_(
-                    t, non_blocking=True)
-            step()
-            o_host.copy_(o, non_blocking=True)
-            od_host.copy_(od, non_blocking=True)
+        def h2d_into(t):
+            for n, src in pinned.items():
+                t[n].view(torch.int16 if t[n].dtype == torch.bfloat16 else t[n].dtype).copy_(src, non_blocking=True)
 
-        e2e_step()
+        def run_e2e(n_steps):
+            for ev in done:
+                ev.record(stream)
+            copy_stream.wait_stream(stream)
+            with torch.cuda.stream(copy_stream):
+                h2d_into(sets[0])
+                copied[0].record(copy_stream)
+            for i in range(n_steps):
+                cur, nxt = i % 2, (i + 1) % 2
+                if i + 1 < n_steps:
+                    copy_stream.wait_event(done[nxt])   # the step that last read set nxt is done
+                    with torch.cuda.stream(copy_stream):
+                        h2d_into(sets[nxt])
+                        copied[nxt].record(copy_stream)
+                stream.wait_event(copied[cur])
+                t = sets[cur]
+                t["qd"].copy_(t["q"][:, :, -1, :])   # the decode query is the step's last prefill row
+                step_on(t["q"], t["k"], t["v"], t["lq"], t["qd"])
+                o_host.copy_(o, non_blocking=True)
+                od_host.copy_(od, non_blocking=True)
+                done[cur].record(stream)
+
+        run_e2e(2)
         torch.cuda.synchronize()
-        n_e2e = max(2, min(args.steps, 5))
+        n_e2e = max(2, min(args.steps, 8))
         if world > 1:
             dist.barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
+        run_e2e(n_e2e)
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a0.elapsed_time(a1) / n_e2e, world, dev)
         e2e = {"value": job_throughput(world, B * N, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "overlap": "step i+1's host-to-device copies run on a copy stream during step i"}
     if rank != 0:
         return
 
@@ -596,6 +628,9 @@ def run_decode(args, w, rank, world, local_rank):
     if hils.hils_get_status() != 0:
         raise RuntimeError("device status error during warm-up")
     times = []
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    clocks.start()
+    time.sleep(0.3)
     launches0 = hils.hils_kernel_launches()
     for _ in range(args.steps):
         flush.zero_()
@@ -606,10 +641,42 @@ def run_decode(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     launches = hils.hils_kernel_launches() - launches0
+    clk = clocks.stop()
     status = hils.hils_get_status()
     if status != 0:
         raise RuntimeError(f"device status {status} during the timed steps")
     us = 1e3 * max_over_ranks(float(np.median(times)), world, dev)
+    # end to end: every step copies the new queries and the sequence lengths in
+    # from pinned host memory and reads the outputs back (the KV cache and its
+    # summaries stay resident, as in a serving loop)
+    e2e = None
+    if not args.no_e2e:
+        q_host = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        q_host.copy_(q)
+        seq_host = torch.empty(seq.shape, dtype=seq.dtype).pin_memory()
+        seq_host.copy_(seq)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = q_host.numel() * q_host.element_size() + seq_host.numel() * seq_host.element_size()
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            q.copy_(q_host, non_blocking=True)
+            seq.copy_(seq_host, non_blocking=True)
+            step()
+            o_host.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(5, args.steps)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_us = 1e3 * max_over_ranks(a0.elapsed_time(a1) / n_e2e, world, dev)
+        e2e = {"value": e_us, "unit": "us/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "steps back to back, no L2 flush between them"}
     if rank != 0:
         return
     sel_bytes = decode_selected_bytes(ids.cpu().numpy(), w)
@@ -629,6 +696,8 @@ def run_decode(args, w, rank, world, local_rank):
                      "bytes": "selected-KV (union of kept chunks + local window chunks per (b, kv head))",
                      "selected_kv_bytes": sel_bytes, "all_bytes_gbs": all_gbs},
         "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
     }
     print(json.dumps(line), flush=True)
 
