@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(BwdTiles<D>::THREADS)
 bwd_chunk_kernel(const T* __restrict__ q, const T* __restrict__ q_score, const T* __restrict__ k,
                  const T* __restrict__ v, const T* __restrict__ d_o, const float* __restrict__ kprime,
                  const float* __restrict__ dvec, const int32_t* __restrict__ tile_start, const int4* __restrict__ items,
-                 const int32_t* __restrict__ e_row, const float* __restrict__ e_fac, const CcDims c,
+                 const int2* __restrict__ e_pair, const CcDims c,
                  float* dq, float* dqs, float* __restrict__ dk, float* __restrict__ dv,   // dqs may be dq
                  float* __restrict__ dkp, float* __restrict__ dbp) {
   using BT = BwdTiles<D>;
@@ -307,14 +307,15 @@ bwd_chunk_kernel(const T* __restrict__ q, const T* __restrict__ q_score, const T
       __syncthreads();
       for (int idx = tid; idx < ns * D; idx += BT::THREADS) {
         const int r = idx / D, t = idx % D;
-        const int64_t row = e_row[first + s0 + r];
+        const int64_t row = e_pair[first + s0 + r].x;
         qs[idx] = ldf(q + row * D + t);
         gs[idx] = ldf(d_o + row * D + t);
       }
       __syncthreads();
       for (int r = warp; r < ns; r += BT::THREADS / 32) {
-        const int64_t row = e_row[first + s0 + r];
-        const float a = expf(e_fac[first + s0 + r]);   // exp(s^ - M')
+        const int2 ep = e_pair[first + s0 + r];
+        const int64_t row = ep.x;
+        const float a = expf(__int_as_float(ep.y));   // exp(s^ - M')
         const float dg = dvec[row];
         float s0v, s1v, g0, g1;
         bwd_row_dots<D>(qs + r * D, ks, s0v, s1v);

@@ -67,7 +67,7 @@ bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float* __restrict__ kprime, const float* __restrict__ dvec,
                     const int32_t* __restrict__ tile_start, const int4* __restrict__ items,
-                    const int32_t* __restrict__ e_row, const float* __restrict__ e_fac, const CcDims c,
+                    const int2* __restrict__ e_pair, const CcDims c,
                     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dkp,
                     float* __restrict__ dbp) {
   using C = BwdTc<D>;
@@ -117,8 +117,9 @@ bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int n = rec.z;
     const int64_t bh = kvrow / c.n_tok, chunk = (kvrow % c.n_tok) / kChunk;
     // the tile's pair rows (entries are padded with valid rows past the end)
-    s_rows[tid] = e_row[first + tid];
-    s_fac[tid] = e_fac[first + tid];
+    const int2 ep = e_pair[first + tid];
+    s_rows[tid] = ep.x;
+    s_fac[tid] = __int_as_float(ep.y);
     for (int t = tid; t < D; t += C::THREADS) s_kp[t] = kprime[(bh * c.nc + chunk) * D + t];
     __syncthreads();
     if (tid == 0) {

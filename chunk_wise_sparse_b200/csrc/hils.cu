@@ -170,8 +170,7 @@ struct CcPlan {
   CcDims c;
   int64_t rows, n_slots, max_items, n_scan_blocks;
   int P, own_tiles;
-  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_erow, off_efac,
-      total;
+  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair, total;
 };
 
 bool cc_supported(const hils_dims* d) {
@@ -225,8 +224,7 @@ CcPlan cc_plan(const hils_dims* d) {
   P.off_items = take(sizeof(int4) * P.max_items);
   P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
   // entries are padded by one tile so that tile loads never run past the end
-  P.off_erow = take(sizeof(int32_t) * (P.n_slots + kCcTileRows));
-  P.off_efac = take(sizeof(float) * (P.n_slots + kCcTileRows));
+  P.off_epair = take(sizeof(int2) * (P.n_slots + kCcTileRows));
   P.total = off;
   return P;
 }
@@ -258,8 +256,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
   int4* items = reinterpret_cast<int4*>(base + P.off_items);
   int64_t* sums = reinterpret_cast<int64_t*>(base + P.off_sums);
-  int32_t* e_row = reinterpret_cast<int32_t*>(base + P.off_erow);
-  float* e_fac = reinterpret_cast<float*>(base + P.off_efac);
+  int2* e_pair = reinterpret_cast<int2*>(base + P.off_epair);
   const uint64_t kv_rows = uint64_t(d->batch) * d->heads_kv * d->seqlen;
   const uint32_t nk_own = P.P >= kChunk ? uint32_t(P.P) : uint32_t(kChunk);
   CUtensorMap tq_tile, tq_row, tk, tv, tk_own, tv_own;
@@ -272,7 +269,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
     return HILS_ERR_CUDA;
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess) return HILS_ERR_CUDA;
   // the padding after the last entry must hold valid row ids (row 0)
-  if (cudaMemsetAsync(base + P.off_erow + sizeof(int32_t) * P.n_slots, 0, sizeof(int32_t) * kCcTileRows, st) !=
+  if (cudaMemsetAsync(base + P.off_epair + sizeof(int2) * P.n_slots, 0, sizeof(int2) * kCcTileRows, st) !=
       cudaSuccess)
     return HILS_ERR_CUDA;
   CcOwnParams op;
@@ -309,7 +306,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
   cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
   cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_row, e_fac,
+  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
                                                                      P.c, P.n_slots);
   constexpr auto fn = cc_attend_kernel<D>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
@@ -317,8 +314,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   prm.c = P.c;
   prm.tile_start = tiles;
   prm.items = items;
-  prm.e_row = e_row;
-  prm.e_fac = e_fac;
+  prm.e_pair = e_pair;
   prm.oacc = oacc;
   fn<<<unsigned(sm_count() * C::MAX_CTAS), C::THREADS, C::SMEM, st>>>(tq_row, tk, tv, prm);
   const int64_t n8 = P.rows * D / 8;
@@ -330,8 +326,8 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
 struct BwdPlan {
   CcDims c;
   int64_t rows, n_slots, max_items, n_scan_blocks, n_units;
-  size_t off_rowstat, off_dvec, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_erow,
-      off_efac, off_dkp, off_dbp, total;
+  size_t off_rowstat, off_dvec, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair,
+      off_dkp, off_dbp, total;
 };
 
 BwdPlan bwd_plan(const hils_dims* d) {
@@ -353,8 +349,7 @@ BwdPlan bwd_plan(const hils_dims* d) {
   P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
   P.off_items = take(sizeof(int4) * P.max_items);
   P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
-  P.off_erow = take(sizeof(int32_t) * (P.n_slots + kCcTileRows));
-  P.off_efac = take(sizeof(float) * (P.n_slots + kCcTileRows));
+  P.off_epair = take(sizeof(int2) * (P.n_slots + kCcTileRows));
   P.off_dkp = take(sizeof(float) * P.n_units * D);
   P.off_dbp = take(sizeof(float) * P.n_units);
   P.total = off;
@@ -377,8 +372,7 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
   int4* items = reinterpret_cast<int4*>(base + P.off_items);
   int64_t* sums = reinterpret_cast<int64_t*>(base + P.off_sums);
-  int32_t* e_row = reinterpret_cast<int32_t*>(base + P.off_erow);
-  float* e_fac = reinterpret_cast<float*>(base + P.off_efac);
+  int2* e_pair = reinterpret_cast<int2*>(base + P.off_epair);
   float* dkp = reinterpret_cast<float*>(base + P.off_dkp);
   float* dbp = reinterpret_cast<float*>(base + P.off_dbp);
   const int64_t N = d->seqlen, kv_elems = int64_t(d->batch) * d->heads_kv * N * D;
@@ -392,7 +386,7 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
       cudaMemsetAsync(dkp, 0, sizeof(float) * P.n_units * (D + 0), st) != cudaSuccess ||
       cudaMemsetAsync(dbp, 0, sizeof(float) * P.n_units, st) != cudaSuccess ||
       cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess ||
-      cudaMemsetAsync(base + P.off_erow + sizeof(int32_t) * P.n_slots, 0, sizeof(int32_t) * kCcTileRows, st) !=
+      cudaMemsetAsync(base + P.off_epair + sizeof(int2) * P.n_slots, 0, sizeof(int2) * kCcTileRows, st) !=
           cudaSuccess)
     return HILS_ERR_CUDA;
   if (dq_score && cudaMemsetAsync(dq_score, 0, sizeof(float) * P.rows * D, st) != cudaSuccess) return HILS_ERR_CUDA;
@@ -411,7 +405,7 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
   cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
   cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_row, e_fac,
+  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
                                                                      P.c, P.n_slots);
   const float tau = 1.f / sqrtf(float(D));
   const size_t smem_w = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(BT::SUB) * D * 4;
@@ -435,13 +429,13 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
     constexpr auto tfn = bwd_chunk_tc_kernel<D>;
     if (set_smem_max<tfn>() != cudaSuccess) return HILS_ERR_CUDA;
     tfn<<<unsigned(sm_count() * (D == 64 ? 2 : 1)), CT::THREADS, CT::SMEM, st>>>(
-        mq, mg, mk, mv, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq, dk, dv, dkp, dbp);
+        mq, mg, mk, mv, kprime, dvec, tiles, items, e_pair, P.c, dq, dk, dv, dkp, dbp);
   } else {
     const size_t smem_c = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(2 * D + 4) * 4;
     constexpr auto cfn2 = bwd_chunk_kernel<T, D>;
     if (set_smem_max<cfn2>() != cudaSuccess) return HILS_ERR_CUDA;
     cfn2<<<unsigned(sm_count() * 2), BT::THREADS, smem_c, st>>>(
-        tq, static_cast<const T*>(q_score), tk, tv, tdo, kprime, dvec, tiles, items, e_row, e_fac, P.c, dq,
+        tq, static_cast<const T*>(q_score), tk, tv, tdo, kprime, dvec, tiles, items, e_pair, P.c, dq,
         dq_score ? dq_score : dq, dk, dv, dkp, dbp);
   }
   const size_t smem_s = size_t(4) * (kChunk * BT::KS + 3 * D) * 4;

@@ -522,8 +522,8 @@ cc_scan_apply_kernel(const int32_t* __restrict__ counts, const CcDims c, const i
 // and its fusion factor s^ - M'.
 __global__ void __launch_bounds__(256)
 cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const float* __restrict__ scores,
-               const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int32_t* __restrict__ e_row,
-               float* __restrict__ e_fac, const CcDims c, int64_t n_slots) {
+               const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int2* __restrict__ e_pair,
+               const CcDims c, int64_t n_slots) {
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n_slots) return;
   const int32_t ci = __ldg(ids + idx);
@@ -534,8 +534,8 @@ cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ rank
   const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
   const int64_t bh = b * c.Hkv + hq / c.G;
   const int64_t at = offsets[cc_key(c, bh, i, ci)] + __ldg(ranks + idx);
-  e_row[at] = int32_t(row);
-  e_fac[at] = __ldg(scores + idx) - __ldg(rowstat + row);
+  // one 8-byte record per pair: the row and its fusion factor
+  e_pair[at] = make_int2(int32_t(row), __float_as_int(__ldg(scores + idx) - __ldg(rowstat + row)));
 }
 
 // ---------------------------------------------------------------- accumulator -> output
@@ -607,8 +607,7 @@ struct CcTcParams {
   CcDims c;
   const int32_t* tile_start;   // [n_keys + 1]; the last entry is the number of tiles
   const int4* items;           // per tile: first entry, K/V row, pair count
-  const int32_t* e_row;        // per entry: global row id
-  const float* e_fac;          // per entry: s^ - M'
+  const int2* e_pair;          // per entry: global row id, s^ - M' (float bits)
   float* oacc;
 };
 
@@ -685,8 +684,9 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int base = r.x + 4 * lane;   // entries are padded past the last tile
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        row[t] = __ldg(p.e_row + base + t);
-        fac[t] = __ldg(p.e_fac + base + t);
+        const int2 e = __ldg(p.e_pair + base + t);
+        row[t] = e.x;
+        fac[t] = __int_as_float(e.y);
       }
     };
     int4 r0 = make_int4(0, 0, 0, 0), r1 = r0, r2 = r0;
