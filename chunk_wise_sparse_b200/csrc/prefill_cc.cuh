@@ -188,7 +188,29 @@ cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int64_t row = (b * c.Hq + h * G + g) * c.n_tok + pos;
   const int64_t own = pos / kChunk;
   float smax = -INFINITY;
-  if (live) {
+  // K <= 32 (a multiple of 4): the row's kept ids and scores are loaded once,
+  // all loads in flight, and kept in registers for both passes
+  const bool reg_k = c.K <= 32 && (c.K & 3) == 0;
+  int32_t kid[32];
+  float ksc[32];
+  if (live && reg_k) {
+    const int4* i4 = reinterpret_cast<const int4*>(p.ids + row * c.K);
+    const float4* s4 = reinterpret_cast<const float4*>(p.scores + row * c.K);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      int4 ci = make_int4(-1, -1, -1, -1);
+      float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < c.K / 4) {
+        ci = __ldg(i4 + t);
+        sc = __ldg(s4 + t);
+      }
+      kid[4 * t] = ci.x; kid[4 * t + 1] = ci.y; kid[4 * t + 2] = ci.z; kid[4 * t + 3] = ci.w;
+      ksc[4 * t] = sc.x; ksc[4 * t + 1] = sc.y; ksc[4 * t + 2] = sc.z; ksc[4 * t + 3] = sc.w;
+    }
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      if (kid[t] >= 0 && kid[t] < own) smax = fmaxf(smax, ksc[t]);
+  } else if (live) {
     if ((c.K & 3) == 0) {
       const int4* i4 = reinterpret_cast<const int4*>(p.ids + row * c.K);
       const float4* s4 = reinterpret_cast<const float4*>(p.scores + row * c.K);
@@ -258,9 +280,15 @@ cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (live) {
     const float Mx = fmaxf(smax, lse);
     float Z = expf(lse - Mx);
-    for (int t = 0; t < c.K; ++t) {
-      const int32_t ci = __ldg(p.ids + row * c.K + t);
-      if (ci >= 0 && ci < own) Z += expf(__ldg(p.scores + row * c.K + t) - Mx);
+    if (reg_k) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (kid[t] >= 0 && kid[t] < own) Z += expf(ksc[t] - Mx);
+    } else {
+      for (int t = 0; t < c.K; ++t) {
+        const int32_t ci = __ldg(p.ids + row * c.K + t);
+        if (ci >= 0 && ci < own) Z += expf(__ldg(p.scores + row * c.K + t) - Mx);
+      }
     }
     Mp = Mx + logf(Z);
     p.rowstat[row] = Mp;
