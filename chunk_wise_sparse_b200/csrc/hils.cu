@@ -306,8 +306,12 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
   cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
   cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
-                                                                     P.c, P.n_slots);
+  if (d->topk % 4 == 0)
+    cc_fill4_kernel<<<unsigned((P.n_slots / 4 + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets,
+                                                                            e_pair, P.c, P.n_slots / 4);
+  else
+    cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
+                                                                       P.c, P.n_slots);
   constexpr auto fn = cc_attend_kernel<D>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   CcTcParams prm;
@@ -405,8 +409,12 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
   cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
   cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
-                                                                     P.c, P.n_slots);
+  if (d->topk % 4 == 0)
+    cc_fill4_kernel<<<unsigned((P.n_slots / 4 + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets,
+                                                                            e_pair, P.c, P.n_slots / 4);
+  else
+    cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
+                                                                       P.c, P.n_slots);
   const float tau = 1.f / sqrtf(float(D));
   const size_t smem_w = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(BT::SUB) * D * 4;
   constexpr auto wfn = bwd_window_kernel<T, D>;

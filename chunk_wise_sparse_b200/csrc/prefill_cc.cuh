@@ -566,6 +566,37 @@ cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ rank
   e_pair[at] = make_int2(int32_t(row), __float_as_int(__ldg(scores + idx) - __ldg(rowstat + row)));
 }
 
+// The same scatter four slots of one row per thread (K a multiple of 4):
+// 16-byte loads of ids, ranks and scores, one row statistic, and the four
+// independent offset loads in flight together.
+__global__ void __launch_bounds__(256)
+cc_fill4_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const float* __restrict__ scores,
+                const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int2* __restrict__ e_pair,
+                const CcDims c, int64_t n_quads) {
+  const int64_t qd = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (qd >= n_quads) return;
+  const int64_t idx = qd * 4;
+  const int4 ci = __ldg(reinterpret_cast<const int4*>(ids) + qd);
+  const int4 rk = __ldg(reinterpret_cast<const int4*>(ranks) + qd);
+  const float4 sc = __ldg(reinterpret_cast<const float4*>(scores) + qd);
+  const int64_t row = idx / c.K;
+  const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
+  const int64_t n_cand = n_candidates(i, c.wm1);
+  const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
+  const int64_t bh = b * c.Hkv + hq / c.G;
+  const float ms = __ldg(rowstat + row);
+  const int32_t cv[4] = {ci.x, ci.y, ci.z, ci.w};
+  const int32_t rv[4] = {rk.x, rk.y, rk.z, rk.w};
+  const float sv[4] = {sc.x, sc.y, sc.z, sc.w};
+  int64_t at[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)   // out-of-range ids were recorded when counting
+    at[e] = (cv[e] >= 0 && cv[e] < n_cand) ? offsets[cc_key(c, bh, i, cv[e])] + rv[e] : -1;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (at[e] >= 0) e_pair[at[e]] = make_int2(int32_t(row), __float_as_int(sv[e] - ms));
+}
+
 // ---------------------------------------------------------------- accumulator -> output
 template <int D>
 __global__ void __launch_bounds__(256)
