@@ -384,6 +384,44 @@ cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, i
   const int64_t n = int64_t(kCountRows) * c.K;
   const int32_t* id0 = ids + row0 * c.K;
   int32_t* rk0 = ranks + row0 * c.K;
+  if ((c.K & 3) == 0) {
+    // four slots of one row per step, 16-byte loads and stores
+    const int64_t n4 = n / 4;
+    const int4* id4 = reinterpret_cast<const int4*>(id0);
+    int4* rk4 = reinterpret_cast<int4*>(rk0);
+#pragma unroll 4
+    for (int64_t t = threadIdx.x; t < n4; t += blockDim.x) {
+      const int4 ci = __ldg(id4 + t);
+      const int64_t nc_i = n_candidates(i0 + (4 * t) / c.K, c.wm1);
+      const int32_t cv[4] = {ci.x, ci.y, ci.z, ci.w};
+      int32_t r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        r[e] = 0;
+        if (cv[e] >= nc_i) record_error(HILS_ERR_DEVICE_BOUNDS);
+        if (cv[e] >= 0 && cv[e] < nc_i) r[e] = atomicAdd(hist + cv[e], 1);
+      }
+      rk4[t] = make_int4(r[0], r[1], r[2], r[3]);
+    }
+    __syncthreads();
+    for (int64_t t = threadIdx.x; t < nch; t += blockDim.x) {
+      const int32_t h = hist[t];
+      hist[t] = h > 0 ? atomicAdd(counts + key0 + t, h) : 0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int64_t t = threadIdx.x; t < n4; t += blockDim.x) {
+      const int4 ci = __ldg(id4 + t);
+      const int64_t nc_i = n_candidates(i0 + (4 * t) / c.K, c.wm1);
+      int4 r = rk4[t];
+      if (ci.x >= 0 && ci.x < nc_i) r.x += hist[ci.x];
+      if (ci.y >= 0 && ci.y < nc_i) r.y += hist[ci.y];
+      if (ci.z >= 0 && ci.z < nc_i) r.z += hist[ci.z];
+      if (ci.w >= 0 && ci.w < nc_i) r.w += hist[ci.w];
+      rk4[t] = r;
+    }
+    return;
+  }
   for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
     const int32_t ci = __ldg(id0 + t);
     if (ci < 0) continue;
