@@ -172,3 +172,29 @@ def test_decode_with_qcal(dtype, d, paged):
     err = np.abs(o.float().reshape(-1, w.d).cpu().numpy() - O_o)
     assert err.max() <= OUT_MAX[dtype], err.max()
     assert err.mean() <= OUT_MEAN[dtype], err.mean()
+
+
+def test_prefill_with_qcal_full_size():
+    """The bench's Q-Cal workload (512K, 16 heads, rank 16) on 4096 sampled rows."""
+    from chunk_wise_sparse_b200.inputs import WORKLOADS
+    w = WORKLOADS["prefill-512k-h16-d64-qcal16"]
+    inp = generate(w)
+    q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
+    wt = qcal_weights(w.Hq, w.d, w.qcal, seed=w.seed, dtype=w.dtype)
+    wd, wu = dev_weights(wt, w.dtype)
+    o, aux = hils.prefill_qcal(q, k, v, lq, w.K, wd, wu, return_all=True)
+    torch.cuda.synchronize()
+    assert hils.hils_get_status() == 0
+    oracle = Oracle.for_workload(w)
+    kp, bp = oracle.summary(inp.k_f32, inp.lq_f32)
+    flat = sample_rows(w)
+    rows = Rows.from_prefill(inp.q_f32, flat)
+    qs = scoring_query(qcal(rows.q, rows.hq, wt.w_down_f32, wt.w_up_f32), w.dtype)
+    srows = Rows(rows.b, rows.hq, rows.pos, qs)
+    ids_o, _, gap = oracle.select(kp, bp, srows)
+    ids_g = gather_rows(aux["ids"], flat).astype(np.int32)
+    check_selection(ids_g, ids_o, gap, oracle.scores(kp, bp, srows), SEL_GAP[w.dtype], SEL_GAP[w.dtype])
+    O_o, _ = oracle.attend(inp.k_f32, inp.v_f32, kp, bp, rows, ids_g, qscore=qs)
+    err = np.abs(gather_rows(o, flat) - O_o)
+    assert err.max() <= OUT_MAX[w.dtype], err.max()
+    assert err.mean() <= OUT_MEAN[w.dtype], err.mean()

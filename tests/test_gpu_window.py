@@ -93,3 +93,22 @@ def test_decode_window_agrees_with_prefill_last_row():
     assert hils.hils_get_status() == 0
     assert torch.equal(ids, aux["ids"][:, :, -1, :])
     assert torch.max(torch.abs(od - o[:, :, -1, :])).item() <= 1e-5
+
+
+def test_prefill_window_full_size():
+    """The bench's window workload (32K, window 512) on 4096 sampled rows."""
+    from chunk_wise_sparse_b200.inputs import WORKLOADS
+    run_prefill_case(WORKLOADS["prefill-32k-h16-d64-w512"])
+
+
+def test_decode_window_full_size():
+    """The bench's window decode workload (128K x 8, GQA 4, window 512)."""
+    from chunk_wise_sparse_b200.inputs import WORKLOADS
+    w = WORKLOADS["decode-128k-b8-gqa4-d128-w512"]
+    inp = generate(w)
+    q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
+    summ = hils.landmark_summary(k, lq, w.K)
+    oracle = Oracle.for_workload(w)
+    kp, bp = oracle.summary(inp.k_f32, inp.lq_f32)
+    check_summary(w, inp, summ, kp, bp)
+    run_decode_check(w, inp, q, k, v, summ, inp.seqlens, oracle, kp, bp, inp.q_f32)
