@@ -131,3 +131,27 @@ def test_backward_after_the_gpu_forward():
     assert hils.hils_get_status() == 0
     ref = oracle.backward(inp.q_f32, inp.k_f32, inp.v_f32, inp.lq_f32, ids_o.reshape(1, 2, w.N, w.K), dO)
     check(g, ref, "fp32", ["dq", "dk", "dv", "dlq"])
+
+
+def test_backward_full_size_identities():
+    """The bench's 32K workload after the GPU forward: at any size each row's
+    fusion weights sum to 1, so sum_j dV_j = sum over the kv head's query heads
+    of sum_i dO_i; and a common shift of all keys of a kv head leaves the output
+    unchanged, so sum_j dK_j = 0 (up to the bf16 rounding of O in <dO, O>)."""
+    from chunk_wise_sparse_b200.inputs import WORKLOADS
+    w = WORKLOADS["prefill-32k-h16-d64"]
+    inp = generate(w)
+    q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
+    o, aux = hils.prefill(q, k, v, lq, w.K, return_all=True)
+    d_o = torch.randn(q.shape, device="cuda", generator=torch.Generator(device="cuda").manual_seed(5)).to(q.dtype)
+    g = hils.backward(q, k, v, lq, aux, o, d_o, w.K)
+    torch.cuda.synchronize()
+    assert hils.hils_get_status() == 0
+    G = w.Hq // w.Hkv
+    dO = d_o.float().view(w.B, w.Hkv, G, w.N, w.d).sum(dim=(2, 3))
+    sv = g["dv"].sum(dim=2)
+    assert torch.max(torch.abs(sv - dO)).item() <= 1e-3 * max(1.0, torch.max(torch.abs(dO)).item())
+    sk = g["dk"].sum(dim=2)
+    scale = g["dk"].abs().sum(dim=2)
+    assert torch.all(torch.abs(sk) <= 1e-2 * scale + 1e-3), (torch.abs(sk) / scale).max().item()
+    assert all(torch.isfinite(g[n]).all() for n in ("dq", "dk", "dv", "dlq"))
