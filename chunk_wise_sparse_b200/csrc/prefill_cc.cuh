@@ -649,16 +649,21 @@ cc_final_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ o, i
 
 // ---------------------------------------------------------------- chunk tiles on tcgen05
 // Warp-specialised, two-stage pipeline per CTA over its tiles (item = blockIdx.x
-// + j * gridDim.x):
-//   warp 0       producer: the tile's entries (row ids, fusion factors) into
-//                shared memory (loaded one tile ahead), then one lane issues
-//                TMA loads of the chunk's K and V and 32*d/64 gather4 loads of
-//                the rows' queries (128B swizzle);
+// + j * gridDim.x), persistent with two CTAs per SM:
+//   warp 0       producer: tile records three tiles ahead and their entries
+//                (row id, fusion factor s^ - M') two tiles ahead, held in named
+//                registers; per tile the entries go to the stage's shared
+//                memory, one lane issues TMA loads of the chunk's K and V, and
+//                every lane issues the gather4 loads of its four query rows
+//                (128B swizzle);
 //   warp 1       one lane issues S = Q K^T into TMEM buffer b, and once the
-//                softmax warps have written P, O = P V into TMEM buffer b;
-//   warps 2-5    one thread per row: the fusion factor s^ - M' (two loads),
-//                softmax of its 64 scores into P (bf16, shared memory), then
-//                its row of O added to the accumulator (16-byte reductions).
+//                softmax warps have written P, O = P V into TMEM buffer b,
+//                then releases the stage;
+//   warps 2-5    one thread per row: softmax of its 64 scores into P (bf16,
+//                over the stage's Q tile); the softmax of tile j+1 runs before
+//                tile j's output rows are staged in a separate padded buffer
+//                and added to the accumulator (one bulk reduction per row at
+//                d = 64, coalesced 16-byte reductions per warp row at d = 128).
 // Stage / TMEM buffer b = j & 1, so loading tile j+1 and the MMAs of tile j+1
 // overlap the softmax and reductions of tile j.
 template <int D>
