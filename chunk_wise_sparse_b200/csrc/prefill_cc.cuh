@@ -11,19 +11,23 @@
 // (a 128-row block selects hundreds of distinct chunks), so that design would
 // spend most tensor-core work on rows that did not select the chunk.  Here the
 // work is regrouped by chunk instead:
-//   own    : per row, the causal own-chunk attention, the fusion normaliser
-//            M' = log(sum_c exp(s^_c) + exp(lse_own)), the own chunk's share
-//            exp(lse_own - M') o_own written to an fp32 accumulator, and a
-//            count of (row, slot) pairs per key (kv head, window, chunk).
+//   own    : per row, the causal own-chunk attention (or, with a local
+//            window of more than one chunk, the window branch of
+//            prefill_local.cuh), the fusion normaliser
+//            M' = log(sum_c exp(s^_c) + exp(lse_own)) and the own branch's
+//            share exp(lse_own - M') o_own written to an fp32 accumulator.
+//   count  : the number of (row, slot) pairs per key (kv head, window,
+//            chunk) and each pair's rank within its key.
 //   scan   : offsets of every key's pair list and of its 128-row tiles.
-//   fill   : the inverted index: each key's list of (row, slot) entries.
+//   fill   : the inverted index: per key its list of (row, s^ - M') records.
 //   attend : per tile of up to 128 pairs of one chunk: the chunk's K and V
-//            arrive by TMA, the rows' queries are gathered with cp.async into
-//            a 128B-swizzled tile, S = Q K^T on tcgen05 (fp32 in TMEM), one
+//            arrive by TMA, the rows' queries by TMA gather4 into a
+//            128B-swizzled tile, S = Q K^T on tcgen05 (fp32 in TMEM), one
 //            thread per row turns its 64 scores into
 //            P = exp(s - lse_c + s^_c - M'), P V on tcgen05, and the row's
-//            partial output is added to its accumulator with 16-byte vector
-//            reductions.  The weights are final, so partials simply add.
+//            partial output is added to its accumulator in L2 (bulk or
+//            16-byte vector reductions).  The weights are final, so partials
+//            simply add.
 //   final  : accumulator -> bf16 output.
 // Windows: a key's rows lie in one window of W positions; tiles are ordered
 // window by window, so the accumulators of the rows being updated stay
