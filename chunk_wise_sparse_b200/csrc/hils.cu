@@ -512,6 +512,9 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   if (nc <= 256 * 16)
     decode_topk_reg_kernel<16><<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
                                                                 ws.sel_ids, ws.sel_scores, wm1);
+  else if (nc <= 256 * 32)
+    decode_topk_reg_kernel<32><<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
+                                                                ws.sel_ids, ws.sel_scores, wm1);
   else
     decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
                                                         ws.sel_scores, wm1);
