@@ -89,6 +89,13 @@ __device__ __forceinline__ void tma_gather4(uint32_t smem_dst, const CUtensorMap
       : "memory");
 }
 
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3_f32(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -903,16 +910,22 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       uint8_t* prow = smem + s * C::STAGE + C::OFF_P + r * 128;
       if (live) {
-        float m = -INFINITY;
+        // short dependency chains: a tree of three-input maxima, four partial sums
+        float mx[22];
 #pragma unroll
-        for (int t = 0; t < 64; ++t) m = fmaxf(m, sc[t]);
+        for (int t = 0; t < 21; ++t) mx[t] = fmax3_f32(sc[3 * t], sc[3 * t + 1], sc[3 * t + 2]);
+        mx[21] = sc[63];
+#pragma unroll
+        for (int t = 0; t < 7; ++t) mx[t] = fmax3_f32(mx[3 * t], mx[3 * t + 1], mx[3 * t + 2]);
+        const float m = fmaxf(fmax3_f32(fmax3_f32(mx[0], mx[1], mx[2]), fmax3_f32(mx[3], mx[4], mx[5]), mx[6]), mx[21]);
         const float mb = m * k2;
-        float l = 0.f;
+        float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < 64; ++t) {
           sc[t] = ex2_approx(fmaf(sc[t], k2, -mb));
-          l += sc[t];
+          lp[t & 3] += sc[t];
         }
+        const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
         const float w = expf(fac) / l;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
