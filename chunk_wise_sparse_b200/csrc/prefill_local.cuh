@@ -207,7 +207,7 @@ cc_local_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // last valid key of window chunk cj for this row (-1: none)
     auto last_key = [&](int64_t cj) -> int { return (live && cj >= lo && cj <= own) ? (cj < own ? kChunk - 1 : jpos) : -1; };
     bool ok = true;
-    float m = -INFINITY;
+    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent chains
     for (int t = 0; t < KB; ++t) {
       const int sb = t & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag));
@@ -221,12 +221,13 @@ cc_local_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const int jmax = last_key(cw0 + t);
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        if (e <= jmax) m = fmaxf(m, sa[e]);
-        if (e + 32 <= jmax) m = fmaxf(m, sc[e]);
+        mp[e & 3] = fmaxf(mp[e & 3], e <= jmax ? sa[e] : -INFINITY);
+        mp[(e + 2) & 3] = fmaxf(mp[(e + 2) & 3], e + 32 <= jmax ? sc[e] : -INFINITY);
       }
     }
+    const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
     const float mb = (live ? m : 0.f) * k2;
-    float l = 0.f;
+    float lp[4] = {0.f, 0.f, 0.f, 0.f};
     for (int j = 0; ok && j < KB; ++j) {
       const int t = KB + j, sb = t & 1, pb = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag));
@@ -252,7 +253,7 @@ cc_local_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const float x1 = e0 + 1 < 32 ? sa[e0 + 1] : sc[e0 - 31];
           const float y0 = e0 <= jmax ? ex2_approx(fmaf(x0, k2, -mb)) : 0.f;
           const float y1 = e0 + 1 <= jmax ? ex2_approx(fmaf(x1, k2, -mb)) : 0.f;
-          l += y0 + y1;
+          lp[v2] += y0 + y1;
           __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
           wd[v2] = *reinterpret_cast<uint32_t*>(&h2);
         }
@@ -262,6 +263,7 @@ cc_local_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(&p_full[pb]);
     }
     // window log-sum-exp and the fusion normaliser over the kept chunks and the window
+    const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
     const float lse = (live ? m : 0.f) * c.tau + logf(l);
     float Mp = lse;
     if (live && ok) {
