@@ -79,6 +79,7 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
   constexpr int E = Vec16<KT>::E;                   // elements per 16-byte load
   constexpr int RS = MMA_OPERAND ? D + kExt : D;    // row stride of the k' rows
   extern __shared__ __align__(16) float sq[];       // [G][D]
+  pdl_trigger();
   const int bh = blockIdx.y;
   const int b = bh / Hkv, h = bh % Hkv;
   const int64_t own = decode_own_chunk(seqlens, b, cap);
@@ -161,6 +162,8 @@ decode_topk_kernel(const float* __restrict__ ws_scores, const int32_t* __restric
   __shared__ uint32_t hist[256];
   __shared__ int warp_tot[8];
   __shared__ uint32_t s_digit, s_above;
+  pdl_wait();      // the scores of the step's first kernel
+  pdl_trigger();
   const int row = blockIdx.x, b = row / Hq, tid = threadIdx.x;
   int64_t n = decode_own_chunk(seqlens, b, cap) - wm1;   // candidates
   if (n < 0) n = 0;
@@ -247,6 +250,8 @@ decode_topk_reg_kernel(const float* __restrict__ ws_scores, const int32_t* __res
   __shared__ uint32_t hist[256];
   __shared__ int warp_tot[8];
   __shared__ uint32_t s_digit, s_above;
+  pdl_wait();      // the scores of the step's first kernel
+  pdl_trigger();
   const int row = blockIdx.x, b = row / Hq, tid = threadIdx.x;
   int64_t n = decode_own_chunk(seqlens, b, cap) - wm1;   // candidates
   if (n < 0) n = 0;
@@ -398,6 +403,8 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   int* s_slot = sid + G * K;   // [32] per head: the chunk's slot in its list, -1 if not kept
   int& s_go = s_slot[32];
   int* s_off = s_slot + 34;   // [2] element offset of the chunk's rows, low and high words
+  pdl_wait();      // the top-K lists
+  pdl_trigger();
   const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t row0 = int64_t(b) * Hq + int64_t(h) * G;
@@ -552,6 +559,7 @@ decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict_
                       int64_t n_rows, int wm1) {
   __shared__ float s_w[kMaxTopK + 17];   // fusion weight of each slot
   __shared__ float s_z;
+  pdl_wait();      // the partial outputs
   const int t = threadIdx.x;
   const int64_t row = blockIdx.x;
   const int b = int(row / Hq);

@@ -48,6 +48,24 @@ int check_dims(const hils_dims* d) {
 // chunks of the local window before the own chunk
 inline int window_wm1(const hils_dims* d) { return d->window > kChunk ? d->window / kChunk - 1 : 0; }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// before the previous kernel in the stream completes and must call pdl_wait()
+// before it touches that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, static_cast<KArgs>(args)...);
+}
+
 inline int launched(int n) {
   g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
@@ -509,25 +527,34 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
   k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q_score ? q_score : q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores, wm1);
+  // the next three kernels start while their predecessor finishes and wait
+  // for it on the device (programmatic dependent launch)
+  const dim3 g2(static_cast<unsigned>(rows));
+  cudaError_t e;
   if (nc <= 256 * 16)
-    decode_topk_reg_kernel<16><<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
-                                                                ws.sel_ids, ws.sel_scores, wm1);
+    e = launch_pdl(decode_topk_reg_kernel<16>, g2, 256, 0, st, ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
+                   ws.sel_ids, ws.sel_scores, wm1);
   else if (nc <= 256 * 32)
-    decode_topk_reg_kernel<32><<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
-                                                                ws.sel_ids, ws.sel_scores, wm1);
+    e = launch_pdl(decode_topk_reg_kernel<32>, g2, 256, 0, st, ws.scores, seqlens, d->seqlen, nc, d->heads_q, K,
+                   ws.sel_ids, ws.sel_scores, wm1);
   else
-    decode_topk_kernel<<<unsigned(rows), 256, 0, st>>>(ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
-                                                        ws.sel_scores, wm1);
+    e = launch_pdl(decode_topk_kernel, g2, 256, 0, st, ws.scores, seqlens, d->seqlen, nc, d->heads_q, K, ws.sel_ids,
+                   ws.sel_scores, wm1);
+  if (e != cudaSuccess) return HILS_ERR_CUDA;
   const size_t smem3 = DecUnion<T, D>::smem(G, K);
   constexpr auto k3 = decode_partial_union_kernel<T, D>;
   if (smem3 > 48 * 1024 && set_smem_max<k3>() != cudaSuccess) return HILS_ERR_CUDA;
   const dim3 g3(unsigned(G * K + wm1 + 1), unsigned(d->batch * d->heads_kv));
-  k3<<<g3, 128, smem3, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), seqlens, d->seqlen,
-      d->heads_q, G, d->heads_kv, K, tau, ws.sel_ids, ws.sel_scores, ws.part_u, ws.part_o, pk, wm1);
-  decode_combine_kernel<T, D><<<unsigned(rows), D, 0, st>>>(
-      ws.part_u, ws.part_o, seqlens, d->seqlen, d->heads_q, K, ws.sel_ids, ws.sel_scores, static_cast<T*>(o),
-      ids_out, scores_out, rows, wm1);
+  e = launch_pdl(k3, g3, 128, smem3, st, static_cast<const T*>(q), static_cast<const T*>(kc),
+                 static_cast<const T*>(vc), seqlens, d->seqlen, d->heads_q, G, d->heads_kv, K, tau,
+                 static_cast<const int32_t*>(ws.sel_ids), static_cast<const float*>(ws.sel_scores), ws.part_u,
+                 ws.part_o, pk, wm1);
+  if (e != cudaSuccess) return HILS_ERR_CUDA;
+  e = launch_pdl(decode_combine_kernel<T, D>, dim3(unsigned(rows)), D, 0, st,
+                 static_cast<const float*>(ws.part_u), static_cast<const float*>(ws.part_o), seqlens, d->seqlen,
+                 d->heads_q, K, static_cast<const int32_t*>(ws.sel_ids), static_cast<const float*>(ws.sel_scores),
+                 static_cast<T*>(o), ids_out, scores_out, rows, wm1);
+  if (e != cudaSuccess) return HILS_ERR_CUDA;
   return launched(4);
 }
 
