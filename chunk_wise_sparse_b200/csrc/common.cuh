@@ -21,15 +21,6 @@ __device__ int32_t g_status;
 
 __device__ __forceinline__ void record_error(int32_t code) { atomicCAS(&g_status, 0, code); }
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
-// serialisation may start while the kernel before it in the stream is still
-// running; pdl_wait() returns once that kernel has completed and its memory
-// writes are visible (at once for a kernel launched without the attribute).
-// pdl_trigger() lets the next such kernel be scheduled as soon as every block
-// of this one has called it.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // Candidates of a query at position i: the chunks before its local window,
 // which spans the own chunk and the wm1 chunks before it (wm1 = 0: the own
 // chunk alone).

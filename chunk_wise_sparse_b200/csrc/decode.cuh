@@ -29,6 +29,15 @@
 
 namespace hils {
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it in the stream is still
+// running; pdl_wait() returns once that kernel has completed and its memory
+// writes are visible (at once for a kernel launched without the attribute).
+// pdl_trigger() lets the next such kernel be scheduled as soon as every block
+// of this one has called it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 struct DecodeWs {
   float* scores;      // [B*Hq, nc]
   int32_t* sel_ids;   // [B*Hq, K]
