@@ -46,7 +46,8 @@ def load_peaks():
 
 
 # The sources each recorded kernel is compiled from.
-KERNEL_SOURCES = {"select": ["select_tc.cuh", "sm100.cuh", "common.cuh"]}
+KERNEL_SOURCES = {"select": ["select_tc.cuh", "sm100.cuh", "common.cuh"],
+                  "decode": ["decode.cuh", "attend_simt.cuh", "common.cuh"]}
 
 
 def kernels_sha256(kernel):
@@ -72,6 +73,21 @@ def recorded_traffic(kernel, rows):
     if kernel not in j.get("per_row_bytes", {}) or j.get("sources_sha256", {}).get(kernel) != kernels_sha256(kernel):
         return None
     return float(j["per_row_bytes"][kernel]) * rows
+
+
+def recorded_step_traffic(kernel, workload):
+    """DRAM bytes per step of `kernel` (all its launches in one step) on
+    `workload` from the committed ncu record, or None when there is none or
+    the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    key = f"{kernel}:{workload}"
+    if key not in j.get("per_step_bytes", {}) or j.get("sources_sha256", {}).get(kernel) != kernels_sha256(kernel):
+        return None
+    return float(j["per_step_bytes"][key])
 
 
 def useful_work(w):
@@ -692,7 +708,8 @@ def run_decode(args, w, rank, world, local_rank):
         "data": f"synthetic: i.i.d. N(0,1), seed {w.seed}" + (", KV cache in chunk pages (random order)" if w.paged else ""),
         "config": dict(workload_config(w, world), l2="256 MiB buffer written between steps (L2 flush)"),
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": recorded_step_traffic("decode", w.name),
                      "bytes": "selected-KV (union of kept chunks + local window chunks per (b, kv head))",
                      "selected_kv_bytes": sel_bytes, "all_bytes_gbs": all_gbs},
         "gpu_launches": int(launches),
