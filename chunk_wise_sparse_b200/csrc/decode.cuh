@@ -26,6 +26,7 @@
 //   D4 combine  : softmax over the chunk scores fuses the partials.
 #pragma once
 #include "attend_simt.cuh"
+#include "sm100.cuh"
 
 namespace hils {
 
@@ -75,10 +76,21 @@ __device__ __forceinline__ int64_t decode_own_chunk(const int32_t* seqlens, int 
 
 constexpr int kDecChunksPerCta = 128;
 
-// One thread per candidate chunk: it reads the chunk's compressed-key row
-// once (16-byte loads) and scores it against the G query heads of the kv head
-// (query rows broadcast from shared memory), four heads per pass over the
-// row.  No cross-lane reductions.
+// Shared memory of decode_scores_kernel: the G query rows (fp32), then, for
+// the bf16 scoring operand, the CTA's operand rows and an mbarrier.
+template <int D, bool MMA_OPERAND>
+__host__ __device__ constexpr size_t decode_scores_smem(int G) {
+  return sizeof(float) * size_t(G) * D +
+         (MMA_OPERAND ? size_t(kDecChunksPerCta) * (D + kExt) * sizeof(__nv_bfloat16) + 16 : 0);
+}
+
+// One thread per candidate chunk scores the chunk's compressed key against
+// the G query heads of the kv head (query rows broadcast from shared memory),
+// four heads per pass over the row.  No cross-lane reductions.  The bf16
+// scoring operand rows of the CTA's chunks are contiguous in memory: one bulk
+// copy brings them into shared memory (whole lines from HBM instead of a
+// 16-byte piece of 32 rows per load instruction) and each thread reads its row
+// there; fp32 rows are read from global memory with 16-byte loads.
 template <typename T, int D, bool MMA_OPERAND>
 __global__ void __launch_bounds__(kDecChunksPerCta)
 decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, const float* __restrict__ bp,
@@ -88,6 +100,7 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
   constexpr int E = Vec16<KT>::E;                   // elements per 16-byte load
   constexpr int RS = MMA_OPERAND ? D + kExt : D;    // row stride of the k' rows
   extern __shared__ __align__(16) float sq[];       // [G][D]
+  __shared__ int s_abort;
   pdl_trigger();
   const int bh = blockIdx.y;
   const int b = bh / Hkv, h = bh % Hkv;
@@ -96,6 +109,28 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
     if (threadIdx.x == 0 && blockIdx.x == 0) record_error(HILS_ERR_DEVICE_BOUNDS);
     return;
   }
+  const int64_t c0 = int64_t(blockIdx.x) * kDecChunksPerCta;
+  const int64_t n_cand = own - wm1;
+  if (c0 >= n_cand) return;   // the whole CTA: no candidate chunk
+  __nv_bfloat16* srows = reinterpret_cast<__nv_bfloat16*>(sq + G * D);   // [rows][RS]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(srows + kDecChunksPerCta * RS);
+  if constexpr (MMA_OPERAND) {
+    if (threadIdx.x == 0) {
+      // rows c0 .. c0+nv-1: 16-byte aligned (the operand base is, and a row is
+      // (D + 16) x 2 bytes), a multiple of 16 bytes long
+      const int nv = n_cand - c0 < kDecChunksPerCta ? int(n_cand - c0) : kDecChunksPerCta;
+      const uint32_t bytes = uint32_t(nv) * RS * 2u;
+      s_abort = 0;
+      sm100::mbar_init(bar, 1);
+      sm100::fence_barrier_init();
+      sm100::mbar_arrive_expect_tx(bar, bytes);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              sm100::smem_u32(srows)),
+          "l"(kmma + (int64_t(bh) * nc + c0) * RS), "r"(bytes), "r"(sm100::smem_u32(bar))
+          : "memory");
+    }
+  }
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, t = idx % D;
     const T x = q[(int64_t(b) * Hq + h * G + g) * D + t];
@@ -103,13 +138,21 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
     else sq[idx] = x;
   }
   __syncthreads();
-  const int64_t c = int64_t(blockIdx.x) * kDecChunksPerCta + threadIdx.x;
-  if (c >= own - wm1) return;
-  const KT* row = (MMA_OPERAND ? reinterpret_cast<const KT*>(kmma) : reinterpret_cast<const KT*>(kp)) +
-                  (int64_t(bh) * nc + c) * RS;
+  if constexpr (MMA_OPERAND) {
+    if (!sm100::mbar_wait(bar, 0, &s_abort)) {
+      // the copy did not land within the time limit (recorded): let it land
+      // before the CTA's shared memory is released
+      if (threadIdx.x == 0) sm100::mbar_wait_drain(bar, 0);
+      return;
+    }
+  }
+  const int64_t c = c0 + threadIdx.x;
+  if (c >= n_cand) return;
+  const KT* row = MMA_OPERAND ? reinterpret_cast<const KT*>(srows + threadIdx.x * RS)
+                              : reinterpret_cast<const KT*>(kp) + (int64_t(bh) * nc + c) * RS;
   float bias;
   if constexpr (MMA_OPERAND) {
-    const __nv_bfloat16* ext = kmma + (int64_t(bh) * nc + c) * RS + D;
+    const __nv_bfloat16* ext = srows + threadIdx.x * RS + D;
     bias = __bfloat162float(ext[0]) + __bfloat162float(ext[1]);
   } else {
     bias = __ldg(bp + int64_t(bh) * nc + c);
@@ -120,7 +163,8 @@ decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kp, cons
 #pragma unroll 4
     for (int k0 = 0; k0 < D; k0 += E) {
       float kv[E];
-      Vec16<KT>::load(row + k0, kv);
+      if constexpr (MMA_OPERAND) Vec16<KT>::unpack(*reinterpret_cast<const uint4*>(row + k0), kv);
+      else Vec16<KT>::load(row + k0, kv);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (g0 + j < G) {

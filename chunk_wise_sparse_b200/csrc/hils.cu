@@ -521,7 +521,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   DecodeWs ws;
   const int wm1 = window_wm1(d);
   decode_ws_layout(rows, nc, K, wm1 + 1, D, static_cast<char*>(ws_ptr), &ws);
-  const size_t smem1 = sizeof(float) * size_t(G) * D;
+  const size_t smem1 = decode_scores_smem<D, BF>(G);
   constexpr auto k1 = decode_scores_kernel<T, D, BF>;
   if (smem1 > 48 * 1024 && set_smem_max<k1>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
