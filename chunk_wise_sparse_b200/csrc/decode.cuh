@@ -471,6 +471,29 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
     return;
   }
   const int64_t n_cand = own - wm1 > 0 ? own - wm1 : 0;
+  if (tid == 0) {
+    // send the chunk's key and value rows toward L2 now, while the slot
+    // bookkeeping below runs (a chunk another head's CTA takes is on its way
+    // for that CTA too); nothing is prefetched for an invalid chunk or page
+    int64_t c = -1;
+    if (pidx >= G * K) {
+      c = own - (pidx - G * K);
+    } else {
+      const int32_t ci = sel_ids[row0 * K + pidx];
+      if (ci >= 0 && ci < n_cand) c = ci;
+    }
+    int64_t off = -1;
+    if (c >= 0 && pk.table == nullptr) {
+      off = ((int64_t(b) * Hkv + h) * cap + c * kChunk) * D;
+    } else if (c >= 0) {
+      const int64_t page = __ldg(pk.table + int64_t(b) * (cap / kChunk) + c);
+      if (page >= 0 && page < pk.n_pages) off = (page * Hkv + h) * kChunk * D;
+    }
+    if (off >= 0) {
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kc + off), "r"(U::TILE) : "memory");
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vc + off), "r"(U::TILE) : "memory");
+    }
+  }
   for (int idx = tid; idx < G * K; idx += 128) sid[idx] = sel_ids[row0 * K + idx];
   __syncthreads();
   int64_t j0, j1;
