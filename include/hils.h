@@ -183,6 +183,11 @@ size_t hils_decode_workspace_bytes(const hils_dims* dims);
  *   scores_out   [B, Hq, K] fp32 out (nullable)
  *   workspace    device scratch of at least hils_decode_workspace_bytes(dims)
  * heads_q / heads_kv must be at most 32 (HILS_ERR_UNSUPPORTED otherwise).
+ * The step is four kernels on `stream`, ordered like any stream work.  The
+ * first is launched normally; the other three with programmatic stream
+ * serialisation, so each may be scheduled while the one before it finishes
+ * and waits for it on the device.  Only the library's own kernels overlap this
+ * way; work the caller enqueues before or after the call is not affected.
  */
 int hils_attn_decode(const hils_dims* dims, const void* q, const void* k_cache, const void* v_cache,
                      const float* kprime, const float* bprime, const void* kprime_mma,
