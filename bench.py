@@ -475,15 +475,16 @@ def run_ours(args, w, rank, world, local_rank):
 def decode_selected_bytes(ids, w):
     """Distinct K/V bytes a decode step must read at full length: per (b, kv
     head) the union of the G heads' kept chunks plus the local window's chunks,
-    64 keys x d x 2 bytes x (K, V)."""
+    64 keys x d elements x (K, V)."""
     B, Hq, K = ids.shape
     n_win = min(max(1, w.window // w.C), w.N // w.C)
+    elem = 2 if w.dtype == "bf16" else 4
     total = 0
     for b in range(B):
         for h in range(w.Hkv):
             sel = ids[b, h * w.G:(h + 1) * w.G].reshape(-1)
             n_union = len(np.unique(sel[sel >= 0])) + n_win
-            total += n_union * w.C * w.d * 2 * 2
+            total += n_union * w.C * w.d * elem * 2
     return total
 
 
