@@ -525,7 +525,7 @@ int launch_decode(const hils_dims* d, const void* q, const void* kc, const void*
   constexpr auto k1 = decode_scores_kernel<T, D, BF>;
   if (smem1 > 48 * 1024 && set_smem_max<k1>() != cudaSuccess) return HILS_ERR_CUDA;
   dim3 g1(unsigned((nc + kDecChunksPerCta - 1) / kDecChunksPerCta), unsigned(d->batch * d->heads_kv));
-  k1<<<g1, 128, smem1, st>>>(static_cast<const T*>(q_score ? q_score : q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
+  k1<<<g1, kDecChunksPerCta, smem1, st>>>(static_cast<const T*>(q_score ? q_score : q), kp, bp, static_cast<const __nv_bfloat16*>(kmma), seqlens,
                             d->seqlen, nc, d->heads_q, G, d->heads_kv, tau, ws.scores, wm1);
   // the next three kernels start while their predecessor finishes and wait
   // for it on the device (programmatic dependent launch)
