@@ -86,10 +86,17 @@ def strerror(status: int) -> str:
 
 
 def _ptr(t):
+    """Device address of a tensor argument (a raw int is passed as is).  Every
+    buffer the library reads or writes is device memory of the current GPU:
+    a host tensor, or one on another GPU, is refused here, before any call."""
     if t is None:
         return None
     if isinstance(t, int):
         return ctypes.c_void_p(t)
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device} but the current device is cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(t.data_ptr())
 
 

@@ -130,3 +130,18 @@ def test_strerror(lib):
     for code in range(7):
         assert len(hils.strerror(code)) >= 2
     assert hils.strerror(99) == "unknown status"
+
+
+def test_host_tensors_are_refused_by_the_binding(lib):
+    """Every buffer of the ABI is device memory: the binding refuses a host
+    tensor before the library is called (no launch, no host fallback)."""
+    import torch
+    d = dims()
+    q = torch.zeros((1, 2, 1024, 64), dtype=torch.bfloat16)
+    ids = torch.zeros((1, 2, 1024, 4), dtype=torch.int32)
+    before = hils.hils_kernel_launches()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        hils.hils_select(d, q, None, None, q, ids)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        hils.hils_landmark_summary(d, q, q, 0, 16, ids, ids)
+    assert hils.hils_kernel_launches() == before
