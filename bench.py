@@ -20,6 +20,7 @@ import glob
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -50,14 +51,22 @@ KERNEL_SOURCES = {"select": ["select_tc.cuh", "sm100.cuh", "common.cuh"],
                   "decode": ["decode.cuh", "attend_simt.cuh", "common.cuh"]}
 
 
+def code_only(text):
+    """C/CUDA source without its comments and blank space: what the compiler sees."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernels_sha256(kernel):
-    """Hash of a kernel's CUDA sources, to tell whether recorded counters still apply."""
+    """Hash of a kernel's CUDA sources (code only, comments ignored), to tell
+    whether recorded counters still apply."""
     h = hashlib.sha256()
     src = os.path.join(ROOT, "chunk_wise_sparse_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
         h.update(name.encode())
-        with open(os.path.join(src, name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(src, name), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()
 
 

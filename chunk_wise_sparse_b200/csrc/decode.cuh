@@ -9,10 +9,11 @@
 // candidates are the chunks before the window, c < o - wm1.
 //
 // Four short kernels, all HBM- or latency-bound:
-//   D1 scores   : s^ for every candidate chunk of every query head; one warp
-//                 streams 32 compressed-key rows and scores them against the
+//   D1 scores   : s^ for every candidate chunk of every query head; one
+//                 thread per chunk scores its compressed-key row against the
 //                 G query heads that share the kv head (one read of k' per
-//                 kv head).
+//                 kv head); the bf16 rows of a CTA arrive in shared memory by
+//                 one bulk copy.
 //   D2 top-K    : exact radix select (4 passes of 8 bits over an
 //                 order-preserving integer image of the score), then a
 //                 stable compaction in ascending chunk id; ties among equal
@@ -24,6 +25,9 @@
 //                 its exact log-sum-exp, so the window chunks' partials fuse
 //                 to the one window branch.
 //   D4 combine  : softmax over the chunk scores fuses the partials.
+// D2-D4 are launched with programmatic stream serialisation: each may start
+// while its predecessor finishes and waits for it (pdl_wait) before reading
+// its results.
 #pragma once
 #include "attend_simt.cuh"
 #include "sm100.cuh"

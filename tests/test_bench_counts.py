@@ -69,3 +69,10 @@ def test_recorded_traffic_needs_the_sources_it_was_taken_on(monkeypatch):
     assert bench.recorded_traffic("select", 10) is None
     assert bench.recorded_step_traffic("decode", "decode-128k-b8-gqa4-d128") is None
     monkeypatch.setattr(bench, "kernels_sha256", real)
+
+
+def test_source_hash_sees_code_not_comments():
+    a = "int x = 1;  // a note\n/* a block\n   comment */ int y = 2;\n"
+    b = "int x = 1;\nint y = 2;  // another note\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(a.replace("2", "3"))
