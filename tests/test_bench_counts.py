@@ -60,15 +60,24 @@ def test_decode_selected_bytes_is_the_union_per_kv_head():
         assert bench.decode_selected_bytes(ids, w) == want
 
 
-def test_recorded_traffic_needs_the_sources_it_was_taken_on(monkeypatch):
-    real = bench.kernels_sha256
-    assert bench.recorded_traffic("select", 10) == pytest.approx(10 * 160.0)
-    assert bench.recorded_step_traffic("decode", "decode-128k-b8-gqa4-d128") is not None
+def test_recorded_traffic_needs_the_sources_it_was_taken_on(monkeypatch, tmp_path):
+    """A record applies only while the hash of its kernel's code is the one it
+    was taken with (a temporary record, so the test does not depend on the
+    committed one)."""
+    import json
+    (tmp_path / "profiles").mkdir()
+    rec = {"per_row_bytes": {"select": 160.0},
+           "per_step_bytes": {"decode:decode-128k-b8-gqa4-d128": 3.0e8},
+           "sources_sha256": {"select": "h-select", "decode": "h-decode"}}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernels_sha256", lambda kernel: "h-" + kernel)
+    assert bench.recorded_traffic("select", 10) == pytest.approx(1600.0)
+    assert bench.recorded_step_traffic("decode", "decode-128k-b8-gqa4-d128") == pytest.approx(3.0e8)
     assert bench.recorded_step_traffic("decode", "some-other-workload") is None
-    monkeypatch.setattr(bench, "kernels_sha256", lambda kernel: "0" * 64)
+    monkeypatch.setattr(bench, "kernels_sha256", lambda kernel: "changed")
     assert bench.recorded_traffic("select", 10) is None
     assert bench.recorded_step_traffic("decode", "decode-128k-b8-gqa4-d128") is None
-    monkeypatch.setattr(bench, "kernels_sha256", real)
 
 
 def test_source_hash_sees_code_not_comments():
