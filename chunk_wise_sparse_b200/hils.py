@@ -87,8 +87,9 @@ def strerror(status: int) -> str:
 
 def _ptr(t):
     """Device address of a tensor argument (a raw int is passed as is).  Every
-    buffer the library reads or writes is device memory of the current GPU:
-    a host tensor, or one on another GPU, is refused here, before any call."""
+    buffer the library reads or writes is dense device memory of the current
+    GPU in the layout its header states: a host tensor, one on another GPU or
+    a strided view is refused here, before any call."""
     if t is None:
         return None
     if isinstance(t, int):
@@ -97,6 +98,8 @@ def _ptr(t):
         raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
     if t.device.index != torch.cuda.current_device():
         raise ValueError(f"tensor on {t.device} but the current device is cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {t.stride()} for shape {tuple(t.shape)}")
     return ctypes.c_void_p(t.data_ptr())
 
 
