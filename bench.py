@@ -100,7 +100,10 @@ def recorded_step_traffic(kernel, workload):
 
 
 def useful_work(w):
-    """Algorithmic work of one step (counts documented in the design doc)."""
+    """Algorithmic work of one step: 2d FLOPs per (row, candidate chunk) for
+    the scoring, 4d per (row, attended key) for the attention, and the bytes
+    the summary must move (keys, landmark queries in; k', b' and the scoring
+    operand out)."""
     B, Hq, Hkv, N, d, C, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.C, w.K
     nc = N // C
     wc = max(1, w.window // C)                      # chunks of the local window
