@@ -261,6 +261,29 @@ def test_selection_brute_force_with_ties():
     assert n_tie_rows >= 0
 
 
+def test_selection_ties_go_to_lower_ids():
+    """Reading of the selection rule: among equal scores the lower chunk ids
+    are kept.  With every chunk a copy of chunk 0 (keys and landmark query),
+    all surrogate scores of a row are exactly equal, so every row with more
+    than K candidates keeps chunks 0 .. K-1 and its K-th/(K+1)-th gap is 0."""
+    rng = np.random.default_rng(21)
+    B, H, N, d, C, K = 1, 1, 640, 16, 64, 3
+    nc = N // C
+    Kt = np.tile(rand(rng, 1, 1, C, d), (1, 1, nc, 1))
+    LQ = np.tile(rand(rng, 1, 1, 1, d), (1, 1, nc, 1))
+    o = Oracle(B, H, H, N, d, C, K)
+    kp, bp = o.summary(Kt, LQ)
+    Q = rand(rng, B, H, N, d)
+    rows = Rows.from_prefill(Q, np.arange(C * (K + 1), N, 7))
+    S = o.scores(kp, bp, rows)
+    ids, _, gap = o.select(kp, bp, rows)
+    for r in range(len(rows)):
+        own = rows.pos[r] // C
+        assert np.all(S[r, :own] == S[r, 0])
+        assert list(ids[r]) == list(range(K))
+        assert gap[r] == 0
+
+
 def test_rows_in_first_chunk_are_plain_causal_attention():
     """A query in chunk 0 has no candidate chunk: its output is causal softmax
     attention over keys 0..i; row 0 returns v_0."""

@@ -40,6 +40,10 @@ MUTANTS = {
                              "acc += (double)Wd[t * r + a] * (double)x[t];"),
     "qcal_one_head_for_all": ("const float* Wd = w_down + (int64_t)rhq[row] * r * d;", "const float* Wd = w_down;"),
     "fusion_ignores_scoring_query": ("const float* qs = qscore ? qscore + r * d : q;", "const float* qs = q;"),
+    "select_ties_to_higher_id": ("if (a->s < b->s) return 1;\n  return (a->c < b->c) ? -1 : (a->c > b->c);",
+                                 "if (a->s < b->s) return 1;\n  return (a->c > b->c) ? -1 : (a->c < b->c);"),
+    "summary_of_the_next_chunk": ("const float* kc = K + (bh * D->N + c * C) * d;",
+                                  "const float* kc = K + (bh * D->N + ((c + 1) % (D->N / C)) * C) * d;"),
 }
 
 # mistakes in the backward pass, rejected by tests/test_oracle_backward.py
