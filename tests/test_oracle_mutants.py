@@ -44,6 +44,13 @@ MUTANTS = {
                                  "if (a->s < b->s) return 1;\n  return (a->c > b->c) ? -1 : (a->c < b->c);"),
     "summary_of_the_next_chunk": ("const float* kc = K + (bh * D->N + c * C) * d;",
                                   "const float* kc = K + (bh * D->N + ((c + 1) % (D->N / C)) * C) * d;"),
+    "compressed_key_unnormalised": ("const double p = exp(z[j] - m) / Z;", "const double p = exp(z[j] - m);"),
+    "chunk_values_are_keys": ("attend_keys(q, Kbh, Vbh, c * C, (c + 1) * C, d, tau, s, oc + m_used * d);",
+                              "attend_keys(q, Kbh, Kbh, c * C, (c + 1) * C, d, tau, s, oc + m_used * d);"),
+    "chunk_attention_drops_first_key": ("attend_keys(q, Kbh, Vbh, c * C, (c + 1) * C, d, tau, s, oc + m_used * d);",
+                                        "attend_keys(q, Kbh, Vbh, c * C + 1, (c + 1) * C, d, tau, s, oc + m_used * d);"),
+    "attention_logits_unscaled": ("s[j - j0] = tau * dot_fd(q, Kbh + j * d, d);",
+                                  "s[j - j0] = dot_fd(q, Kbh + j * d, d);"),
 }
 
 # mistakes in the backward pass, rejected by tests/test_oracle_backward.py
@@ -59,6 +66,12 @@ BWD_MUTANTS = {
     "bwd_score_uses_attention_query": ("dqs[t] += tau * du * kp[(bh * nc + cc) * d + t];",
                                        "dqs[t] += tau * du * (double)Kbh[cc * C * d + t];"),
     "bwd_value_weight_unfused": ("dvj[t] += a * pj * (double)gr[t];", "dvj[t] += pj * (double)gr[t];"),
+    "bwd_softmax_without_row_term": ("double dz = a * pj * (dP - X);", "double dz = a * pj * dP;"),
+    "bwd_fusion_without_output_term": ("const double du = a * (X - Dg);", "const double du = a * X;"),
+    "bwd_query_gradient_unscaled": ("dq[t] += tau * dz * (double)Kbh[j * d + t];",
+                                    "dq[t] += dz * (double)Kbh[j * d + t];"),
+    "bwd_landmark_gradient_from_the_summary": ("dlq[t] += tau * dz * (double)kc[j * d + t];",
+                                               "dlq[t] += tau * dz * kpc[t];"),
 }
 
 
