@@ -201,6 +201,31 @@ def cpu_oracle_sample(w, inp, budget_s=15.0):
     return 1.0 / t_token, desc, max_threads()
 
 
+def cpu_oracle_decode(w, inp, budget_s=15.0):
+    """Time the fp64 oracle (as it stands) on the decode step of the workload.
+    The landmark summaries are setup, untimed, as on the GPU side; the timed
+    part is the decode step (scores, top-K, sparse attention) of one sequence
+    with all its query heads, repeated for about `budget_s` seconds and scaled
+    to the batch (the sequences are independent and equally long).  Returns
+    (us/step, description, threads)."""
+    from oracle.oracle import Oracle, max_threads
+    one = Oracle(1, w.Hq, w.Hkv, w.N, w.d, w.C, w.K, w.window)
+    kp, bp = one.summary(inp.k_f32[:1], inp.lq_f32[:1])
+    q, kc, vc = inp.q_f32[:1], np.ascontiguousarray(inp.k_f32[:1]), np.ascontiguousarray(inp.v_f32[:1])
+    seq = np.array([w.N], np.int32)
+    reps, elapsed = 0, 0.0
+    while reps == 0 or elapsed < budget_s:
+        t0 = time.perf_counter()
+        one.decode(q, kc, vc, kp, bp, seq)
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    us = elapsed / reps * w.B * 1e6
+    desc = (f"fp64 oracle: the decode step of 1 of {w.B} sequences (all {w.Hq} query heads, {w.N} cached "
+            f"tokens), {reps} repetitions in {elapsed:.1f} s, scaled to the batch; summaries built beforehand, "
+            f"untimed" + ("; contiguous cache (paging changes only the addresses)" if w.paged else ""))
+    return us, desc, max_threads()
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -729,6 +754,10 @@ def run_decode(args, w, rank, world, local_rank):
         "clocks": clk,
         "e2e": e2e,
     }
+    if not args.no_cpu_baseline and world == 1:
+        v_cpu, desc, threads = cpu_oracle_decode(w, inp, budget_s=args.ref_budget)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "us/step", "cores": threads, "kind": "oracle",
+                                "sample": desc}
     print(json.dumps(line), flush=True)
 
 

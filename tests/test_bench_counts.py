@@ -85,3 +85,12 @@ def test_source_hash_sees_code_not_comments():
     b = "int x = 1;\nint y = 2;  // another note\n"
     assert bench.code_only(a) == bench.code_only(b)
     assert bench.code_only(a) != bench.code_only(a.replace("2", "3"))
+
+
+def test_decode_cpu_baseline_times_the_oracle_decode_step():
+    from chunk_wise_sparse_b200.inputs import generate
+    for window in (0, 256):
+        w = custom("dec-cpu", B=3, Hq=4, Hkv=2, d=64, N=2048, K=4, window=window, kind="decode")
+        us, desc, threads = bench.cpu_oracle_decode(w, generate(w), budget_s=0.05)
+        assert us > 0 and threads >= 1
+        assert "1 of 3 sequences" in desc
