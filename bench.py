@@ -492,6 +492,7 @@ def run_ours(args, w, rank, world, local_rank):
         "decode_us_per_step": 1e3 * kernels_ms["decode"],
         "prefill_bc_tflops_useful": bc_flops / (bc_ms / 1e3) / 1e12,
         "prefill_bc_frac_of_bf16_peak": bc_flops / (bc_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "prefill_bc_frac_of_bf16_sustained": bc_flops / (bc_ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
         "roofline": roof,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -700,6 +701,19 @@ def run_decode(args, w, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status} during the timed steps")
     us = 1e3 * max_over_ranks(float(np.median(times)), world, dev)
+    # the median over 100 more flushed steps, after the timed ones
+    more = []
+    for _ in range(100):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        more.append(e0.elapsed_time(e1))
+    if hils.hils_get_status() != 0:
+        raise RuntimeError("device status error during the extra steps")
+    us_100 = 1e3 * max_over_ranks(float(np.median(more)), world, dev)
     # end to end: every step copies the new queries and the sequence lengths in
     # from pinned host memory and reads the outputs back (the KV cache and its
     # summaries stay resident, as in a serving loop)
@@ -753,6 +767,7 @@ def run_decode(args, w, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clk,
         "e2e": e2e,
+        "median_us_of_100_more_steps": us_100,
     }
     if not args.no_cpu_baseline and world == 1:
         v_cpu, desc, threads = cpu_oracle_decode(w, inp, budget_s=args.ref_budget)
