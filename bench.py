@@ -226,6 +226,32 @@ def cpu_oracle_decode(w, inp, budget_s=15.0):
     return us, desc, max_threads()
 
 
+def cpu_oracle_backward(w, inp):
+    """Time the fp64 oracle (as it stands) on the backward of one (b, kv head)
+    slab of the workload -- its G query heads, every row -- for the oracle's
+    own selection (setup, untimed) and a seeded output gradient, scaled to the
+    B x Hkv independent slabs.  Returns (tokens/s, description, threads)."""
+    from oracle.oracle import Oracle, Rows, max_threads
+    # a causal prefix of at most 32K tokens is a whole problem of its own;
+    # past the first chunks a row's cost does not grow with its position
+    n = min(w.N, 32768)
+    one = Oracle(1, w.G, 1, n, w.d, w.C, w.K, w.window)
+    Q, Kt, Vt, LQ = (np.ascontiguousarray(a[:1, :w.G, :rows] if name == "q" else a[:1, :1, :rows])
+                     for name, a, rows in (("q", inp.q_f32, n), ("k", inp.k_f32, n), ("v", inp.v_f32, n),
+                                           ("lq", inp.lq_f32, n // w.C)))
+    kp, bp = one.summary(Kt, LQ)
+    ids, _, _ = one.select(kp, bp, Rows.from_prefill(Q, np.arange(w.G * n)))
+    dO = np.random.default_rng(w.seed + 3000).standard_normal(Q.shape).astype(np.float32)
+    t0 = time.perf_counter()
+    one.backward(Q, Kt, Vt, LQ, ids.reshape(1, w.G, n, w.K), dO)
+    t_slab = time.perf_counter() - t0
+    tokens_per_s = n / (t_slab * w.Hkv)   # B*N tokens over B*Hkv slabs of N/n such prefixes each
+    desc = (f"fp64 oracle: backward of the first {n} tokens of 1 of {w.B * w.Hkv} (b, kv head) slabs "
+            f"({w.G} query heads) in {t_slab:.1f} s, scaled to the whole job; selection and summaries "
+            f"beforehand, untimed")
+    return tokens_per_s, desc, max_threads()
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -601,14 +627,10 @@ def run_backward(args, w, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     max_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
     ach = flops / (ms_step / 1e3) / 1e12
-    if w.dtype == "bf16":
-        # bf16: the selected chunks' contractions run on tcgen05
-        peaks = load_peaks()
-        bound, peak, psrc = "tensor", peaks["bf16_tflops"], peaks["source"] + " bf16 dense burst"
-    else:
-        bound = "alu"
-        peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
-        psrc = f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {max_mhz:.0f} MHz"
+    # every backward kernel runs on CUDA cores in fp32 (bf16 inputs are widened)
+    bound = "alu"
+    peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+    psrc = f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {max_mhz:.0f} MHz"
     line = {
         "metric": "HiLS backward tokens/s (gradients of q, k, v, lq for a fixed selection)",
         "value": job_throughput(world, B * N, ms_step), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -619,6 +641,10 @@ def run_backward(args, w, rank, world, local_rank):
                      "unit": "TFLOP/s", "frac": ach / peak, "traffic": None, "peak_source": psrc},
         "gpu_launches": int(launches), "clocks": clk, "e2e": None,
     }
+    if not args.no_cpu_baseline and world == 1:
+        v_cpu, desc, threads = cpu_oracle_backward(w, inp)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": desc}
     print(json.dumps(line), flush=True)
 
 

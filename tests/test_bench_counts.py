@@ -94,3 +94,12 @@ def test_decode_cpu_baseline_times_the_oracle_decode_step():
         us, desc, threads = bench.cpu_oracle_decode(w, generate(w), budget_s=0.05)
         assert us > 0 and threads >= 1
         assert "1 of 3 sequences" in desc
+
+
+def test_backward_cpu_baseline_times_one_slab_of_the_oracle_backward():
+    from chunk_wise_sparse_b200.inputs import generate
+    for window, Hq in ((0, 4), (192, 2)):
+        w = custom("bwd-cpu", B=2, Hq=Hq, Hkv=2, d=64, N=512, K=3, window=window, dtype="fp32")
+        v, desc, threads = bench.cpu_oracle_backward(w, generate(w))
+        assert v > 0 and threads >= 1
+        assert "1 of 4 (b, kv head) slabs" in desc
