@@ -130,13 +130,14 @@ def test_decode_full_size():
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_decode_ragged_seqlens(dtype):
-    w = custom(f"decode-ragged-{dtype}", B=3, Hq=8, Hkv=2, d=64, N=8192, K=8, seed=41, dtype=dtype, kind="decode")
+    # lengths 1 (no candidate chunk, one key) and 65 (one candidate) besides ragged long ones
+    w = custom(f"decode-ragged-{dtype}", B=5, Hq=8, Hkv=2, d=64, N=8192, K=8, seed=41, dtype=dtype, kind="decode")
     inp = generate(w)
     q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
     summ = hils.landmark_summary(k, lq, w.K)
     oracle = Oracle.for_workload(w)
     kp, bp = oracle.summary(inp.k_f32, inp.lq_f32)
-    seqlens = np.array([8192, 8192 - 37, 100], np.int32)
+    seqlens = np.array([8192, 8192 - 37, 100, 1, 65], np.int32)
     run_decode_check(w, inp, q, k, v, summ, seqlens, oracle, kp, bp, inp.q_f32)
 
 
