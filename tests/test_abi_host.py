@@ -145,3 +145,15 @@ def test_host_tensors_are_refused_by_the_binding(lib):
     with pytest.raises(ValueError, match="CUDA tensor"):
         hils.hils_landmark_summary(d, q, q, 0, 16, ids, ids)
     assert hils.hils_kernel_launches() == before
+
+
+def test_empty_summary_range_launches_nothing(lib):
+    """[c, c) is a valid range with no chunk: the call succeeds and launches
+    no kernel (the pointers, 16-byte aligned, are never touched)."""
+    d = dims()
+    fake = 1 << 20
+    before = hils.hils_kernel_launches()
+    hils.hils_landmark_summary(d, fake, fake, 5, 5, fake, fake, fake, stream=0)
+    assert hils.hils_kernel_launches() == before
+    with pytest.raises(hils.HilsError):
+        hils.hils_landmark_summary(d, fake, fake, 6, 5, fake, fake, fake, stream=0)
