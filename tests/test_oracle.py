@@ -258,7 +258,9 @@ def test_selection_brute_force_with_ties():
             assert gap[r] >= 0
             srt = np.sort(S[r, :own])[::-1]
             n_tie_rows += srt[K - 1] == srt[K]
-    assert n_tie_rows >= 0
+    # the planted copies tie at the K-th / (K+1)-th boundary on some rows, so
+    # the brute force above really decided ties there (20 of 256 rows here)
+    assert n_tie_rows > 0
 
 
 def test_selection_ties_go_to_lower_ids():

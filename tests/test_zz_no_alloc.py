@@ -5,8 +5,9 @@ that owns all device memory and hands out no workspace, or a decode loop that
 must not pay the device-wide synchronisation cudaMalloc implies.  For them the
 library keeps the decode scratch in a fixed device array of its own.  These
 tests check, through the C ABI, that two calls in a row give the results of
-hils_attn_decode with a caller-provided workspace, and that sizes beyond the
-array are refused before anything is launched.
+hils_attn_decode with a caller-provided workspace, that those calls take no
+device memory, and that sizes beyond the array are refused before anything
+is launched.
 """
 import ctypes
 
@@ -30,17 +31,29 @@ def test_fixed_scratch_decode_matches_workspace_decode(dtype):
     summ = hils.landmark_summary(k, lq, w.K)
     dims = hils.make_dims(w.B, w.Hq, w.Hkv, w.d, w.N, w.K, q.dtype)
     assert hils.hils_decode_workspace_bytes(dims) <= hils.DECODE_FIXED_SCRATCH_BYTES
-    # two calls in a row with different lengths: stale scratch from the first call must not leak
+    cases = []
     for seqlens in ([16384, 16384 - 100, 777], [9000, 64, 16384]):
         seq = torch.tensor(seqlens, dtype=torch.int32, device="cuda")
-        ref_o, ref_ids, ref_sc = hils.decode_step(q, k, v, summ, seq, w.K)
-        o = torch.full_like(q, float("nan"))
-        ids = torch.full((w.B, w.Hq, w.K), -7, dtype=torch.int32, device="cuda")
-        sc = torch.full((w.B, w.Hq, w.K), float("nan"), dtype=torch.float32, device="cuda")
+        ref = hils.decode_step(q, k, v, summ, seq, w.K)
+        out = (torch.full_like(q, float("nan")),
+               torch.full((w.B, w.Hq, w.K), -7, dtype=torch.int32, device="cuda"),
+               torch.full((w.B, w.Hq, w.K), float("nan"), dtype=torch.float32, device="cuda"))
+        cases.append((seq, ref, out))
+    # a first call loads the library's device code (and with it the array) on this GPU
+    warm = torch.empty_like(q)
+    hils.hils_attn_decode_fixed_scratch(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, cases[0][0], warm,
+                                        None, None)
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    # two calls in a row with different lengths: stale scratch from the first call must not leak
+    for seq, _, (o, ids, sc) in cases:
         hils.hils_attn_decode_fixed_scratch(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, o,
                                             ids, sc)
-        torch.cuda.synchronize()
-        assert hils.hils_get_status() == 0
+    torch.cuda.synchronize()
+    # nothing was allocated on the device by the two calls
+    assert torch.cuda.mem_get_info()[0] == free_before
+    assert hils.hils_get_status() == 0
+    for seq, (ref_o, ref_ids, ref_sc), (o, ids, sc) in cases:
         assert torch.equal(ids, ref_ids)
         err = (o.float() - ref_o.float()).abs()
         assert err.max().item() <= OUT_MAX[dtype] and err.mean().item() <= OUT_MEAN[dtype]
