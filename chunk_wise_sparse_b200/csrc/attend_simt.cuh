@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(128)
 prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                     const int32_t* __restrict__ ids, const float* __restrict__ scores, T* __restrict__ o,
                     float* __restrict__ lse_own, int64_t n_tok, int Hq, int G, int Hkv, int K, float tau,
-                    int64_t n_rows, int wm1) {
+                    int64_t n_rows, int wm1, const float* __restrict__ kp, const float* __restrict__ bp,
+                    const __nv_bfloat16* __restrict__ kmma) {
   using L = RowLayout<T, D>;
   constexpr int E = L::E, LPK = L::LPK;
   const int lane = threadIdx.x & 31;
@@ -114,7 +115,32 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
       if (lane == 0) record_error(HILS_ERR_DEVICE_BOUNDS);
       continue;
     }
-    const float u = __ldg(scores + row * K + t);
+    // the chunk score from select, or (scores NULL) recomputed as select
+    // computes it: fp32 tau <q, k'> + b', or from the bf16 scoring operand
+    float u;
+    if (scores != nullptr) {
+      u = __ldg(scores + row * K + t);
+    } else {
+      const int64_t cr = bh * (n_tok / kChunk) + c;
+      float part = 0.f;
+      if (kmma != nullptr) {   // bf16 rows (E = 8): one 16-byte piece of the bf16 k' row per lane
+        float kv[8];
+        Vec16<__nv_bfloat16>::load(kmma + cr * (D + kExt) + sub * 8, kv);
+#pragma unroll
+        for (int e = 0; e < E && e < 8; ++e) part = fmaf(qv[e], kv[e], part);
+        const float x = __bfloat162float(kmma[cr * (D + kExt) + D]) + __bfloat162float(kmma[cr * (D + kExt) + D + 1]);
+        u = tau * (group_sum<LPK>(part) + x);
+      } else {
+        float kv[4];
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+          Vec16<float>::load(kp + cr * D + sub * E + e, kv);
+#pragma unroll
+          for (int z = 0; z < 4; ++z) part = fmaf(qv[e + z], kv[z], part);
+        }
+        u = fmaf(tau, group_sum<LPK>(part), __ldg(bp + cr));
+      }
+    }
     attend_range<T, D>(qv, kbh, vbh, int64_t(c) * kChunk, int64_t(c + 1) * kChunk, tau, oc);
     f.add(u, oc);
   }

@@ -188,7 +188,8 @@ struct CcPlan {
   CcDims c;
   int64_t rows, n_slots, max_items, n_scan_blocks;
   int P, own_tiles;
-  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair, total;
+  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair,
+      off_rescore, total;
 };
 
 bool cc_supported(const hils_dims* d) {
@@ -243,6 +244,8 @@ CcPlan cc_plan(const hils_dims* d) {
   P.off_sums = take(sizeof(int64_t) * 2 * P.n_scan_blocks);
   // entries are padded by one tile so that tile loads never run past the end
   P.off_epair = take(sizeof(int2) * (P.n_slots + kCcTileRows));
+  // the recomputed chunk scores of a call without the selection's scores
+  P.off_rescore = take(sizeof(float) * P.n_slots);
   P.total = off;
   return P;
 }
@@ -260,8 +263,8 @@ int sm_count() {
 }
 
 template <int D>
-int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
-                      const float* scores, void* o, float* lse, void* ws, cudaStream_t st) {
+int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const void* v, const void* kmma,
+                      const int32_t* ids, const float* scores, void* o, float* lse, void* ws, cudaStream_t st) {
   using C = CcTc<D>;
   using CO = CcOwn<D>;
   const CcPlan P = cc_plan(d);
@@ -285,6 +288,15 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
       !make_map_2d(&tk_own, k, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tv_own, v, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B))
     return HILS_ERR_CUDA;
+  int n_launch = 9;
+  if (scores == nullptr) {
+    // no scores from the selection: recompute s^ of the kept ids
+    float* rescore = reinterpret_cast<float*>(base + P.off_rescore);
+    cc_rescore_kernel<D><<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kmma), ids, rescore, P.c, P.n_slots);
+    scores = rescore;
+    ++n_launch;
+  }
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * P.c.n_keys, st) != cudaSuccess) return HILS_ERR_CUDA;
   // the padding after the last entry must hold valid row ids (row 0)
   if (cudaMemsetAsync(base + P.off_epair + sizeof(int2) * P.n_slots, 0, sizeof(int2) * kCcTileRows, st) !=
@@ -341,7 +353,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   fn<<<unsigned(sm_count() * C::MAX_CTAS), C::THREADS, C::SMEM, st>>>(tq_row, tk, tv, prm);
   const int64_t n8 = P.rows * D / 8;
   cc_final_kernel<D><<<unsigned((n8 + 255) / 256), 256, 0, st>>>(oacc, static_cast<__nv_bfloat16*>(o), n8);
-  return launched(9);
+  return launched(n_launch);
 }
 
 // ---------------------------------------------------------------- backward
@@ -486,26 +498,28 @@ int launch_summary(const hils_dims* d, const void* k, const void* lq, int64_t c0
 
 template <typename T, int D, bool MMA>
 int launch_select_simt(const hils_dims* d, const void* q, const float* kp, const float* bp, const void* kmma,
-                       int32_t* ids, float* scores, cudaStream_t st) {
+                       const int64_t* row_pos, int64_t n_rows, int32_t* ids, float* scores, cudaStream_t st) {
   const size_t smem = select_simt_smem<D>(d->topk);
   constexpr auto fn = select_simt_kernel<T, D, MMA>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
-  dim3 grid(unsigned((d->seqlen + kSelRows - 1) / kSelRows), unsigned(d->batch * d->heads_q));
+  dim3 grid(unsigned((n_rows + kSelRows - 1) / kSelRows), unsigned(d->batch * d->heads_q));
   fn<<<grid, kSelRows, smem, st>>>(static_cast<const T*>(q), kp, bp, static_cast<const __nv_bfloat16*>(kmma),
                                   d->seqlen, d->seqlen / kChunk, d->heads_q, d->heads_q / d->heads_kv,
-                                  d->heads_kv, d->topk, 1.f / sqrtf(float(D)), ids, scores, window_wm1(d));
+                                  d->heads_kv, d->topk, 1.f / sqrtf(float(D)), ids, scores, window_wm1(d), row_pos,
+                                  n_rows);
   return launched(1);
 }
 
 template <typename T, int D>
-int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
-                        const float* scores, void* o, float* lse, cudaStream_t st) {
+int launch_prefill_simt(const hils_dims* d, const void* q, const void* k, const void* v, const float* kp,
+                        const float* bp, const void* kmma, const int32_t* ids, const float* scores, void* o,
+                        float* lse, cudaStream_t st) {
   const int64_t rows = int64_t(d->batch) * d->heads_q * d->seqlen;
   const int64_t blocks = (rows + 3) / 4;
   prefill_simt_kernel<T, D><<<dim3(unsigned(blocks)), 128, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), ids, scores,
       static_cast<T*>(o), lse, d->seqlen, d->heads_q, d->heads_q / d->heads_kv, d->heads_kv, d->topk,
-      1.f / sqrtf(float(D)), rows, window_wm1(d));
+      1.f / sqrtf(float(D)), rows, window_wm1(d), kp, bp, static_cast<const __nv_bfloat16*>(kmma));
   return launched(1);
 }
 
@@ -601,14 +615,20 @@ size_t hils_kprime_mma_bytes(const hils_dims* d) {
 }
 
 int hils_select(const hils_dims* d, const void* q, const float* kprime, const float* bprime, const void* kprime_mma,
-                int32_t* ids, float* scores, hils_stream_t stream) {
+                const int64_t* row_pos, int64_t n_rows, int32_t* ids, float* scores, hils_stream_t stream) {
   int rc = check_dims(d);
   if (rc) return rc;
   if (!ptr_ok(q) || !ptr_ok(ids) || (scores != nullptr && !aligned16(scores))) return HILS_ERR_INVALID_ARGUMENT;
+  // every position (row_pos NULL: n_rows 0 or seqlen) or a listed subset
+  if (row_pos == nullptr ? (n_rows != 0 && n_rows != d->seqlen) : (n_rows < 0 || !aligned16(row_pos)))
+    return HILS_ERR_INVALID_ARGUMENT;
+  if (row_pos == nullptr) n_rows = d->seqlen;
+  if (n_rows == 0) return HILS_OK;
+  if (int64_t(d->batch) * d->heads_q > 65535) return HILS_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d->dtype == HILS_BF16) {
     if (!ptr_ok(kprime_mma)) return HILS_ERR_INVALID_ARGUMENT;
-    if (select_tc_supported(d)) {
+    if (row_pos == nullptr && select_tc_supported(d)) {
       const int K = d->topk;
       if (d->head_dim == 64) {
         if (K <= 16) return launch_select_tc<64, 16>(d, q, kprime_mma, ids, scores, st);
@@ -620,12 +640,15 @@ int hils_select(const hils_dims* d, const void* q, const float* kprime, const fl
       return launch_select_tc<128, 0>(d, q, kprime_mma, ids, scores, st);
     }
     if (d->head_dim == 64)
-      return launch_select_simt<__nv_bfloat16, 64, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
-    return launch_select_simt<__nv_bfloat16, 128, true>(d, q, nullptr, nullptr, kprime_mma, ids, scores, st);
+      return launch_select_simt<__nv_bfloat16, 64, true>(d, q, nullptr, nullptr, kprime_mma, row_pos, n_rows, ids,
+                                                         scores, st);
+    return launch_select_simt<__nv_bfloat16, 128, true>(d, q, nullptr, nullptr, kprime_mma, row_pos, n_rows, ids,
+                                                        scores, st);
   }
   if (!ptr_ok(kprime) || !ptr_ok(bprime)) return HILS_ERR_INVALID_ARGUMENT;
-  if (d->head_dim == 64) return launch_select_simt<float, 64, false>(d, q, kprime, bprime, nullptr, ids, scores, st);
-  return launch_select_simt<float, 128, false>(d, q, kprime, bprime, nullptr, ids, scores, st);
+  if (d->head_dim == 64)
+    return launch_select_simt<float, 64, false>(d, q, kprime, bprime, nullptr, row_pos, n_rows, ids, scores, st);
+  return launch_select_simt<float, 128, false>(d, q, kprime, bprime, nullptr, row_pos, n_rows, ids, scores, st);
 }
 
 size_t hils_prefill_workspace_bytes(const hils_dims* d) {
@@ -634,28 +657,36 @@ size_t hils_prefill_workspace_bytes(const hils_dims* d) {
   return cc_plan(d).total;
 }
 
-int hils_attn_prefill(const hils_dims* d, const void* q, const void* k, const void* v, const int32_t* ids,
-                      const float* scores, void* o, float* lse_own, void* workspace, size_t workspace_bytes,
-                      hils_stream_t stream) {
+int hils_attn_prefill(const hils_dims* d, const void* q, const void* k, const void* v, const float* kprime,
+                      const float* bprime, const void* kprime_mma, const int32_t* ids, const float* scores, void* o,
+                      float* lse_own, void* workspace, size_t workspace_bytes, hils_stream_t stream) {
   int rc = check_dims(d);
   if (rc) return rc;
-  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(ids) || !ptr_ok(scores) || !ptr_ok(o))
-    return HILS_ERR_INVALID_ARGUMENT;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(ids) || !ptr_ok(o)) return HILS_ERR_INVALID_ARGUMENT;
+  if (scores != nullptr && !aligned16(scores)) return HILS_ERR_INVALID_ARGUMENT;
   if (lse_own != nullptr && !aligned16(lse_own)) return HILS_ERR_INVALID_ARGUMENT;
+  // without scores the chunk scores are recomputed: bf16 from the scoring
+  // operand, fp32 from k' and b'
+  if (scores == nullptr && (d->dtype == HILS_BF16 ? !ptr_ok(kprime_mma) : (!ptr_ok(kprime) || !ptr_ok(bprime))))
+    return HILS_ERR_INVALID_ARGUMENT;
   const size_t need = hils_prefill_workspace_bytes(d);
   if (workspace_bytes < need) return HILS_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && !ptr_ok(workspace)) return HILS_ERR_INVALID_ARGUMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const void* kmma = scores == nullptr ? kprime_mma : nullptr;
+  const float* kp = scores == nullptr ? kprime : nullptr;
+  const float* bp = scores == nullptr ? bprime : nullptr;
   if (d->dtype == HILS_BF16 && need > 0) {
-    if (d->head_dim == 64) return launch_prefill_cc<64>(d, q, k, v, ids, scores, o, lse_own, workspace, st);
-    return launch_prefill_cc<128>(d, q, k, v, ids, scores, o, lse_own, workspace, st);
+    if (d->head_dim == 64) return launch_prefill_cc<64>(d, q, k, v, kmma, ids, scores, o, lse_own, workspace, st);
+    return launch_prefill_cc<128>(d, q, k, v, kmma, ids, scores, o, lse_own, workspace, st);
   }
   if (d->dtype == HILS_BF16) {
-    if (d->head_dim == 64) return launch_prefill_simt<__nv_bfloat16, 64>(d, q, k, v, ids, scores, o, lse_own, st);
-    return launch_prefill_simt<__nv_bfloat16, 128>(d, q, k, v, ids, scores, o, lse_own, st);
+    if (d->head_dim == 64)
+      return launch_prefill_simt<__nv_bfloat16, 64>(d, q, k, v, nullptr, nullptr, kmma, ids, scores, o, lse_own, st);
+    return launch_prefill_simt<__nv_bfloat16, 128>(d, q, k, v, nullptr, nullptr, kmma, ids, scores, o, lse_own, st);
   }
-  if (d->head_dim == 64) return launch_prefill_simt<float, 64>(d, q, k, v, ids, scores, o, lse_own, st);
-  return launch_prefill_simt<float, 128>(d, q, k, v, ids, scores, o, lse_own, st);
+  if (d->head_dim == 64) return launch_prefill_simt<float, 64>(d, q, k, v, kp, bp, nullptr, ids, scores, o, lse_own, st);
+  return launch_prefill_simt<float, 128>(d, q, k, v, kp, bp, nullptr, ids, scores, o, lse_own, st);
 }
 
 size_t hils_decode_workspace_bytes(const hils_dims* d) {
@@ -814,17 +845,13 @@ namespace {
 // every call, kept until the process exits.
 __device__ __align__(256) unsigned char g_decode_scratch[HILS_DECODE_FIXED_SCRATCH_BYTES];
 
-// Device address of g_decode_scratch on the current device (looked up once per
-// device; host code cannot use the symbol itself as a device pointer).
+// Device address of g_decode_scratch on the current device.  Host code cannot
+// use the symbol itself as a device pointer, so it is looked up on every call
+// (a host-side table lookup once the module is loaded): a cached address would
+// go stale if the caller reset the device and the module came back elsewhere.
 void* decode_scratch_address() {
-  static std::atomic<void*> addr[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  void* p = addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    addr[dev].store(p, std::memory_order_release);
-  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return nullptr;
   return p;
 }
 

@@ -646,6 +646,45 @@ cc_fill4_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ran
     if (at[e] >= 0) e_pair[at[e]] = make_int2(int32_t(row), __float_as_int(sv[e] - ms));
 }
 
+// ---------------------------------------------------------------- chunk scores, recomputed
+// For a prefill called without the scores hils_select returned: s^ of every
+// kept (row, slot) from the query row and the bf16 scoring operand, with the
+// tensor-core selection's arithmetic (aitrends.kr article, section "방법론":
+// s^ = tau <q, k'> + b'; here tau * (<q, k'_bf16> + x_hi + x_lo), products
+// exact and summed in fp32, so only the order of the sums differs).  One
+// thread per slot; the K threads of a row read the same query row.  Padding
+// (-1) and ids outside the row's candidates (recorded when the pairs are
+// counted) get -inf.
+template <int D>
+__global__ void __launch_bounds__(256)
+cc_rescore_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kmma,
+                  const int32_t* __restrict__ ids, float* __restrict__ scores, const CcDims c, int64_t n_slots) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n_slots) return;
+  const int32_t ci = __ldg(ids + idx);
+  const int64_t row = idx / c.K;
+  const int64_t bhq = row / c.n_tok, i = row % c.n_tok;
+  if (ci < 0 || ci >= n_candidates(i, c.wm1)) {
+    scores[idx] = -INFINITY;
+    return;
+  }
+  const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
+  const int64_t bh = b * c.Hkv + hq / c.G;
+  const __nv_bfloat16* kr = kmma + (bh * c.nc + ci) * (D + kExt);
+  const __nv_bfloat16* qr = q + row * D;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int t = 0; t < D; t += 8) {
+    float qv[8], kv[8];
+    Vec16<__nv_bfloat16>::load(qr + t, qv);
+    Vec16<__nv_bfloat16>::load(kr + t, kv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e & 3] = fmaf(qv[e], kv[e], acc[e & 3]);
+  }
+  const float x = __bfloat162float(kr[D]) + __bfloat162float(kr[D + 1]);
+  scores[idx] = c.tau * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + x);
+}
+
 // ---------------------------------------------------------------- accumulator -> output
 template <int D>
 __global__ void __launch_bounds__(256)

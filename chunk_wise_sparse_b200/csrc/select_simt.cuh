@@ -5,8 +5,10 @@
 //   K largest.
 //
 // This is the fp32 path (fp32 has no tensor-core MMA that meets a 1e-5
-// tolerance).  One CTA scores 128 consecutive rows of one (b, hq) against
-// tiles of 32 compressed keys staged in shared memory.  q is stored
+// tolerance), and the path for a listed subset of query positions (row_pos,
+// any order).  One CTA scores 128 rows of one (b, hq) -- consecutive
+// positions, or 128 consecutive entries of row_pos -- against tiles of 32
+// compressed keys staged in shared memory.  q is stored
 // transposed ([d][128]) so each thread reads its own row conflict-free; k'
 // is transposed ([d][32]) so a float4 read broadcasts four chunks.  Each
 // thread keeps its row's running top-K (sorted, ties to the lower id, which
@@ -32,7 +34,8 @@ template <typename T, int D, bool MMA_OPERAND>
 __global__ void __launch_bounds__(kSelRows)
 select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const float* __restrict__ bp,
                    const __nv_bfloat16* __restrict__ kmma, int64_t n_tok, int64_t nc, int Hq, int G,
-                   int Hkv, int K, float tau, int32_t* __restrict__ ids, float* __restrict__ scores, int wm1) {
+                   int Hkv, int K, float tau, int32_t* __restrict__ ids, float* __restrict__ scores, int wm1,
+                   const int64_t* __restrict__ row_pos, int64_t n_rows) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* qT = reinterpret_cast<float*>(smem_raw);          // [D][128]
   float* kT = qT + D * kSelRows;                           // [D][32]
@@ -44,26 +47,38 @@ select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const 
   const int64_t bhq = blockIdx.y;
   const int b = int(bhq / Hq), hq = int(bhq % Hq);
   const int64_t bh = int64_t(b) * Hkv + hq / G;
-  const int64_t i0 = int64_t(blockIdx.x) * kSelRows;
-  const int64_t i = i0 + tid;
-  const bool valid = i < n_tok;
+  __shared__ int64_t pos_s[kSelRows];
+  __shared__ int c_end_s;
+  // this thread's output row r (0 .. n_rows-1) and its query position
+  const int64_t r = int64_t(blockIdx.x) * kSelRows + tid;
+  const bool in_rows = r < n_rows;
+  int64_t i = in_rows ? (row_pos ? __ldg(row_pos + r) : r) : -1;
+  if (in_rows && (i < 0 || i >= n_tok)) {
+    record_error(HILS_ERR_DEVICE_BOUNDS);   // listed position outside the sequence: ids -1
+    i = -1;
+  }
+  const bool valid = i >= 0;
   const int64_t n_cand = valid ? n_candidates(i, wm1) : 0;
+  pos_s[tid] = i;
+  if (tid == 0) c_end_s = 0;
+  __syncthreads();
+  if (n_cand > 0) atomicMax(&c_end_s, int(n_cand));   // candidates of the tile's longest row
 
   // stage q (transposed)
   for (int idx = tid; idx < kSelRows * D; idx += kSelRows) {
-    const int r = idx / D, t = idx % D;
-    const int64_t ii = i0 + r;
+    const int rr = idx / D, t = idx % D;
+    const int64_t ii = pos_s[rr];
     float x = 0.f;
-    if (ii < n_tok) {
+    if (ii >= 0) {
       if constexpr (sizeof(T) == 2) x = __bfloat162float(q[(bhq * n_tok + ii) * D + t]);
       else x = q[(bhq * n_tok + ii) * D + t];
     }
-    qT[t * kSelRows + r] = x;
+    qT[t * kSelRows + rr] = x;
   }
   int count = 0;
   float thr = -INFINITY;
-  const int64_t i_last = (i0 + kSelRows - 1 < n_tok - 1) ? i0 + kSelRows - 1 : n_tok - 1;
-  const int64_t c_end = n_candidates(i_last, wm1);  // candidates of the last row of the tile
+  __syncthreads();
+  const int64_t c_end = c_end_s;
 
   for (int64_t c0 = 0; c0 < c_end; c0 += kSelTile) {
     __syncthreads();
@@ -123,7 +138,7 @@ select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const 
       }
     }
   }
-  if (!valid) return;
+  if (!in_rows) return;
   // ascending chunk id order
   for (int a = 1; a < count; ++a) {
     const int32_t ci = topi[a * kSelRows + tid];
@@ -137,7 +152,7 @@ select_simt_kernel(const T* __restrict__ q, const float* __restrict__ kp, const 
     topi[j * kSelRows + tid] = ci;
     topv[j * kSelRows + tid] = cv;
   }
-  const int64_t row = bhq * n_tok + i;
+  const int64_t row = bhq * n_rows + r;
   for (int t = 0; t < K; ++t) {
     ids[row * K + t] = t < count ? topi[t * kSelRows + tid] : -1;
     if (scores) scores[row * K + t] = t < count ? topv[t * kSelRows + tid] : -INFINITY;

@@ -55,10 +55,10 @@ def lib():
         L.hils_landmark_summary.argtypes = [D, P, P, I64, I64, P, P, P, P]
         L.hils_kprime_mma_bytes.argtypes = [D]
         L.hils_kprime_mma_bytes.restype = SZ
-        L.hils_select.argtypes = [D, P, P, P, P, P, P, P]
+        L.hils_select.argtypes = [D, P, P, P, P, P, I64, P, P, P]
         L.hils_prefill_workspace_bytes.argtypes = [D]
         L.hils_prefill_workspace_bytes.restype = SZ
-        L.hils_attn_prefill.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_attn_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_workspace_bytes.argtypes = [D]
         L.hils_decode_workspace_bytes.restype = SZ
         L.hils_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -141,21 +141,27 @@ def hils_kprime_mma_bytes(dims) -> int:
     return int(lib().hils_kprime_mma_bytes(ctypes.byref(dims)))
 
 
-def hils_select(dims, q, kprime, bprime, kprime_mma, ids, scores=None, stream=None):
+def hils_select(dims, q, kprime, bprime, kprime_mma, row_pos, n_rows, ids, scores=None, stream=None):
+    """row_pos None (n_rows 0): every position; else a device int64 tensor of
+    n_rows query positions, ids / scores [B, Hq, n_rows, K]."""
     _check("hils_select", lib().hils_select(ctypes.byref(dims), _ptr(q), _ptr(kprime), _ptr(bprime),
-                                            _ptr(kprime_mma), _ptr(ids), _ptr(scores), _stream(stream)))
+                                            _ptr(kprime_mma), _ptr(row_pos), int(n_rows), _ptr(ids), _ptr(scores),
+                                            _stream(stream)))
 
 
 def hils_prefill_workspace_bytes(dims) -> int:
     return int(lib().hils_prefill_workspace_bytes(ctypes.byref(dims)))
 
 
-def hils_attn_prefill(dims, q, k, v, ids, scores, o, lse_own=None, workspace=None, workspace_bytes=None,
-                      stream=None):
+def hils_attn_prefill(dims, q, k, v, kprime, bprime, kprime_mma, ids, scores, o, lse_own=None, workspace=None,
+                      workspace_bytes=None, stream=None):
+    """scores None: the chunk scores of the kept ids are recomputed from q and
+    the summaries (kprime_mma for bf16, kprime and bprime for fp32)."""
     if workspace_bytes is None:
         workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check("hils_attn_prefill", lib().hils_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(ids),
-                                                        _ptr(scores), _ptr(o), _ptr(lse_own), _ptr(workspace),
+    _check("hils_attn_prefill", lib().hils_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(kprime),
+                                                        _ptr(bprime), _ptr(kprime_mma), _ptr(ids), _ptr(scores),
+                                                        _ptr(o), _ptr(lse_own), _ptr(workspace),
                                                         int(workspace_bytes), _stream(stream)))
 
 
@@ -279,25 +285,31 @@ def landmark_summary(k, lq, topk=1, chunk_begin=0, chunk_end=None, out: Summary 
     return out
 
 
-def select(q, summ: Summary, heads_kv, topk, stream=None, window=0):
+def select(q, summ: Summary, heads_kv, topk, stream=None, window=0, row_pos=None, with_scores=True):
+    """ids (and scores, or None) of every position, or of the positions in
+    row_pos (a device int64 tensor): [B, Hq, rows, K]."""
     B, Hq, N, d = q.shape
     dims = make_dims(B, Hq, heads_kv, d, N, topk, q.dtype, window=window)
-    ids = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device)
-    scores = torch.empty((B, Hq, N, topk), dtype=torch.float32, device=q.device)
-    hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, stream)
+    n_rows = N if row_pos is None else row_pos.numel()
+    ids = torch.empty((B, Hq, n_rows, topk), dtype=torch.int32, device=q.device)
+    scores = torch.empty((B, Hq, n_rows, topk), dtype=torch.float32, device=q.device) if with_scores else None
+    hils_select(dims, q, summ.kprime, summ.bprime, summ.kprime_mma, row_pos, 0 if row_pos is None else n_rows, ids,
+                scores, stream)
     return ids, scores
 
 
-def prefill(q, k, v, lq, topk, stream=None, return_all=False, window=0):
+def prefill(q, k, v, lq, topk, stream=None, return_all=False, window=0, scores_buffer=True):
     """Full HiLS prefill: summary -> select -> sparse attention.  Returns O
     (and, with return_all, the summary, ids, scores and the local branch's
-    log-sum-exp)."""
+    log-sum-exp).  scores_buffer False: the selection writes no scores and
+    the attention recomputes them."""
     dims = dims_for(q, k, topk, window)
     summ = landmark_summary(k, lq, topk, stream=stream)
-    ids, scores = select(q, summ, k.shape[1], topk, stream, window)
+    ids, scores = select(q, summ, k.shape[1], topk, stream, window, with_scores=scores_buffer)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, prefill_workspace(dims, q.device), stream=stream)
+    hils_attn_prefill(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, o, lse,
+                      prefill_workspace(dims, q.device), stream=stream)
     if return_all:
         return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse)
     return o
@@ -324,7 +336,8 @@ def prefill_qcal(q, k, v, lq, topk, w_down, w_up, stream=None, return_all=False,
     ids, scores = select(q_hat, summ, k.shape[1], topk, stream, window)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, prefill_workspace(dims, q.device), stream=stream)
+    hils_attn_prefill(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores, o, lse,
+                      prefill_workspace(dims, q.device), stream=stream)
     if return_all:
         return o, dict(summary=summ, ids=ids, scores=scores, lse_own=lse, q_hat=q_hat)
     return o

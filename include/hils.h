@@ -113,29 +113,42 @@ int hils_landmark_summary(const hils_dims* dims, const void* k, const void* lq,
 size_t hils_kprime_mma_bytes(const hils_dims* dims);
 
 /*
- * Chunk scoring and top-K selection for every query row of a prefill --
+ * Chunk scoring and top-K selection for the query rows of a prefill --
  * [AIT-Meth]: s^_{i,c} = tau*<q_i, k'_c> + b'_c over the candidates
  * c < floor(i/C) - W + 1 (W = window chunks); keep the K largest.  Ties go to
  * the lower chunk id.
- *   q          [B, Hq, seqlen, d] dtype
+ *   q          [B, Hq, seqlen, d] dtype (every position, also when a subset
+ *              of rows is selected)
  *   kprime     fp32 [B,Hkv,nc,d]  (fp32 path; may be NULL for bf16)
  *   bprime     fp32 [B,Hkv,nc]    (fp32 path; may be NULL for bf16)
  *   kprime_mma bf16 scoring operand (required for bf16, ignored for fp32);
- *              the bf16 path scores on tensor cores with bf16 k'.
- *   ids        [B, Hq, seqlen, K] int32 out: the kept chunk ids in ascending
- *              order; rows with fewer than K candidates are padded with -1.
- *   scores     [B, Hq, seqlen, K] fp32 out (nullable): s^ of each id, -inf
- *              for padding.  hils_attn_prefill consumes it.
+ *              the bf16 path scores with bf16 k' and fp32 accumulation.
+ *   row_pos    NULL: every position 0 .. seqlen-1 (n_rows 0 or seqlen), on
+ *              tensor cores where the shape allows.  Otherwise a device
+ *              int64 array of n_rows query positions (any order, repeats
+ *              allowed, 16-byte aligned), selected on CUDA cores: row r of
+ *              every (b, hq) is position row_pos[r].  A position outside
+ *              [0, seqlen) is recorded as HILS_ERR_DEVICE_BOUNDS and its ids
+ *              are all -1.  This serves checks on a sample of rows and
+ *              queries that need only some positions' selection.
+ *   n_rows     number of listed positions (>= 0; 0 with a list: no work)
+ *   ids        [B, Hq, n_rows, K] int32 out: the kept chunk ids in
+ *              ascending order; rows with fewer than K candidates are padded
+ *              with -1.
+ *   scores     [B, Hq, n_rows, K] fp32 out (nullable): s^ of each id, -inf
+ *              for padding.  hils_attn_prefill can take it or recompute it.
  */
 int hils_select(const hils_dims* dims, const void* q, const float* kprime, const float* bprime,
-                const void* kprime_mma, int32_t* ids, float* scores, hils_stream_t stream);
+                const void* kprime_mma, const int64_t* row_pos, int64_t n_rows, int32_t* ids, float* scores,
+                hils_stream_t stream);
 
 /*
  * Device workspace bytes hils_attn_prefill needs for these dims (0 when the
  * call needs none: the fp32 path).  For bf16 it holds an fp32 output
- * accumulator (rows x d), the fusion normaliser of every row, and the
- * inverted index of (row, slot) pairs per (kv head, window, chunk): about
- * rows x (4d + 4 + 4K) bytes.
+ * accumulator (rows x d), the fusion normaliser of every row, the inverted
+ * index of (row, slot) pairs per (kv head, window, chunk) and room for the
+ * recomputed chunk scores of a call without scores: about
+ * rows x (4d + 4 + 16K) bytes.
  */
 size_t hils_prefill_workspace_bytes(const hils_dims* dims);
 
@@ -148,19 +161,35 @@ size_t hils_prefill_workspace_bytes(const hils_dims* dims);
  * weights are a softmax over {s^_c : c kept} U {lse_own}:
  *     O_i = sum_c w_c o_c + w_own o_own.
  *   q, k, v   [B,Hq,N,d] / [B,Hkv,N,d] / [B,Hkv,N,d] dtype
+ *   kprime, bprime, kprime_mma
+ *             the summaries of hils_landmark_summary; read only when scores
+ *             is NULL (bf16: kprime_mma required, the others may be NULL;
+ *             fp32: kprime and bprime required)
  *   ids       [B,Hq,N,K] int32 from hils_select (-1 entries are skipped; an id
  *             outside the candidates [0, floor(i/C)-W+1) is recorded as
  *             HILS_ERR_DEVICE_BOUNDS and skipped)
- *   scores    [B,Hq,N,K] fp32 from hils_select (required)
+ *   scores    [B,Hq,N,K] fp32 from hils_select, or NULL: then s^ of every
+ *             kept id is recomputed from q and the summaries as hils_select
+ *             computes it ([AIT-Meth]; bf16: tau (<q, k'_bf16> + x_hi + x_lo)
+ *             with fp32 sums in another order, so within rounding of the
+ *             selection's values), and the caller needs no [B,Hq,N,K] scores
+ *             buffer.  Pass the scores when the selection scored another
+ *             query than q (Q-Cal's q^).
  *   o         [B,Hq,N,d] dtype out
  *   lse_own   [B,Hq,N] fp32 out (nullable): log-sum-exp of the local window
  *   workspace device scratch of at least hils_prefill_workspace_bytes(dims)
  *             (may be NULL when that is 0); HILS_ERR_WORKSPACE_TOO_SMALL
  *             otherwise
+ * bf16 outputs: the chunk outputs are summed in fp32 by reductions whose
+ * order is not fixed, so two runs on the same inputs may differ by one bf16
+ * ulp in an output element (the fp32 sums differ only in their last bits,
+ * and rounding to bf16 can then land on the neighbouring value), or by about
+ * 1e-6 for an output that is almost zero (its sum cancels); ids and lse_own
+ * are reproducible.
  */
-int hils_attn_prefill(const hils_dims* dims, const void* q, const void* k, const void* v,
-                      const int32_t* ids, const float* scores, void* o, float* lse_own,
-                      void* workspace, size_t workspace_bytes, hils_stream_t stream);
+int hils_attn_prefill(const hils_dims* dims, const void* q, const void* k, const void* v, const float* kprime,
+                      const float* bprime, const void* kprime_mma, const int32_t* ids, const float* scores, void* o,
+                      float* lse_own, void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
 /* Device workspace bytes hils_attn_decode needs for these dims. */
 size_t hils_decode_workspace_bytes(const hils_dims* dims);
@@ -207,9 +236,13 @@ int hils_attn_decode(const hils_dims* dims, const void* q, const void* k_cache, 
  * GPU that loads the library keeps until the process exits.
  * - Sizes whose hils_decode_workspace_bytes() exceeds that maximum are
  *   rejected with HILS_ERR_WORKSPACE_TOO_SMALL before anything is launched.
- * - The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ * - The 16 MiB are taken on a device when the library's device code is loaded
+ *   there.  Under CUDA's lazy module loading (the default) that happens at the
+ *   first library call or symbol lookup on the device, so that call may
+ *   allocate and synchronise inside the driver: make the first call on each
+ *   device during set-up, before any stream capture.
+ * - Each call looks up the array's device address (cudaGetSymbolAddress,
+ *   with the call's device current), so a device reset in between is safe.
  * - Every call uses the same array and it keeps the previous call's
  *   contents.  Each byte a call reads is written earlier in that same call,
  *   so nothing has to start at zero.  Calls whose executions overlap on the

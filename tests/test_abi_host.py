@@ -53,18 +53,18 @@ def test_sizes(lib):
 def test_bad_dims_rejected_before_launch(lib, kw, code):
     d = dims(**kw)
     p = ctypes.c_void_p(256)     # never dereferenced: validation fails first
-    rc = lib.hils_select(ctypes.byref(d), p, p, p, p, p, None, None)
+    rc = lib.hils_select(ctypes.byref(d), p, p, p, p, None, 0, p, None, None)
     assert rc == code
-    rc = lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, None, 0, None)
+    rc = lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, p, p, p, None, None, 0, None)
     assert rc == code
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
     d = dims()
     p, bad = ctypes.c_void_p(256), ctypes.c_void_p(258)
-    assert lib.hils_select(ctypes.byref(d), None, p, p, p, p, None, None) == 1
-    assert lib.hils_select(ctypes.byref(d), bad, p, p, p, p, None, None) == 1
-    assert lib.hils_select(ctypes.byref(d), p, p, p, None, p, None, None) == 1   # bf16 needs the MMA operand
+    assert lib.hils_select(ctypes.byref(d), None, p, p, p, None, 0, p, None, None) == 1
+    assert lib.hils_select(ctypes.byref(d), bad, p, p, p, None, 0, p, None, None) == 1
+    assert lib.hils_select(ctypes.byref(d), p, p, p, None, None, 0, p, None, None) == 1   # bf16 needs the MMA operand
     assert lib.hils_landmark_summary(ctypes.byref(d), p, p, 0, 17, p, p, None, None) == 1   # range past nc
     assert lib.hils_landmark_summary(ctypes.byref(d), p, p, 3, 3, p, p, None, None) == 0    # empty range
     small = hils.hils_decode_workspace_bytes(d) - 1
@@ -75,8 +75,37 @@ def test_null_and_misaligned_pointers_rejected(lib):
     # bf16 prefill needs its workspace
     need = hils.hils_prefill_workspace_bytes(d)
     assert need > 0
-    assert lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, None, p, need - 1, None) == 4
+    assert lib.hils_attn_prefill(ctypes.byref(d), p, p, p, None, None, None, p, p, p, None, p, need - 1, None) == 4
     assert hils.hils_prefill_workspace_bytes(dims(dtype=hils.FP32)) == 0
+
+
+def test_select_row_subset_arguments(lib):
+    """A listed row subset (row_pos) needs a 16-byte aligned list; without a
+    list n_rows must be 0 or seqlen; an empty list launches nothing."""
+    d = dims()
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(264)
+    assert lib.hils_select(ctypes.byref(d), p, p, p, p, None, 7, p, None, None) == 1          # n_rows without a list
+    assert lib.hils_select(ctypes.byref(d), p, p, p, p, None, d.seqlen + 64, p, None, None) == 1
+    assert lib.hils_select(ctypes.byref(d), p, p, p, p, p, -1, p, None, None) == 1            # negative count
+    assert lib.hils_select(ctypes.byref(d), p, p, p, p, bad, 4, p, None, None) == 1           # misaligned list
+    before = hils.hils_kernel_launches()
+    assert lib.hils_select(ctypes.byref(d), p, p, p, p, p, 0, p, None, None) == 0             # empty list: no work
+    assert hils.hils_kernel_launches() == before
+
+
+def test_prefill_without_scores_needs_the_summaries(lib):
+    """scores NULL makes the prefill recompute the chunk scores: bf16 then needs
+    the scoring operand, fp32 needs k' and b' (refused before any launch)."""
+    p = ctypes.c_void_p(256)
+    d = dims()
+    need = hils.hils_prefill_workspace_bytes(d)
+    assert lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, None, p, None, p, None, p, need, None) == 1
+    d32 = dims(dtype=hils.FP32)
+    assert lib.hils_attn_prefill(ctypes.byref(d32), p, p, p, None, p, p, p, None, p, None, None, 0, None) == 1
+    assert lib.hils_attn_prefill(ctypes.byref(d32), p, p, p, p, None, p, p, None, p, None, None, 0, None) == 1
+    # misaligned scores are refused too
+    assert lib.hils_attn_prefill(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.c_void_p(260), p, None, p, need,
+                                 None) == 1
 
 
 def test_decode_rejects_more_than_32_query_heads_per_kv_head(lib):
@@ -95,7 +124,7 @@ def test_window_sizes(lib):
     d0, d8 = dims(window=0), dims(window=512)
     assert hils.hils_decode_workspace_bytes(d8) > hils.hils_decode_workspace_bytes(d0)
     d16 = dims(window=1024)
-    assert lib.hils_select(ctypes.byref(d16), None, None, None, None, None, None, None) == 1   # dims pass, q NULL
+    assert lib.hils_select(ctypes.byref(d16), None, None, None, None, None, 0, None, None, None) == 1   # dims pass, q NULL
 
 
 def test_qcal_arguments_rejected_before_launch(lib):
@@ -141,7 +170,7 @@ def test_host_tensors_are_refused_by_the_binding(lib):
     ids = torch.zeros((1, 2, 1024, 4), dtype=torch.int32)
     before = hils.hils_kernel_launches()
     with pytest.raises(ValueError, match="CUDA tensor"):
-        hils.hils_select(d, q, None, None, q, ids)
+        hils.hils_select(d, q, None, None, q, None, 0, ids)
     with pytest.raises(ValueError, match="CUDA tensor"):
         hils.hils_landmark_summary(d, q, q, 0, 16, ids, ids)
     assert hils.hils_kernel_launches() == before

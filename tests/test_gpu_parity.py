@@ -163,7 +163,9 @@ def test_out_of_range_id_is_recorded_and_skipped():
     ids[0, 0, 300, 0] = 7       # row 300 is in chunk 4: chunk 7 is not a candidate
     o2 = torch.empty_like(o)
     dims = hils.dims_for(q, k, w.K)
-    hils.hils_attn_prefill(dims, q, k, v, ids, aux["scores"], o2, None, hils.prefill_workspace(dims, q.device))
+    summ = aux["summary"]
+    hils.hils_attn_prefill(dims, q, k, v, summ.kprime, summ.bprime, summ.kprime_mma, ids, aux["scores"], o2, None,
+                           hils.prefill_workspace(dims, q.device))
     assert hils.hils_get_status() == 6
     assert hils.hils_get_status() == 0
     others = torch.ones(w.N, dtype=torch.bool)

@@ -8,8 +8,11 @@ the selection must equal the oracle's element for element: the K largest
 scores, equal scores ordered by lower chunk id (HiLS paper, aitrends.kr
 article, section "방법론"; tie rule as read in the design notes), ids in
 ascending order, -1 padding.  Rows are sampled across every row length at
-which the kernel changes how it bounds the K-th score (no bound, groups of
-8, 16, 32 and 128 chunks) and both rows of each boundary.
+which a kernel changes how it bounds the K-th score (no bound, groups of 8,
+16, 32, 64 and 128 chunks) and both rows of each boundary.  At d = 64 and
+K <= 16 the selection runs with two threads per row, whose halves exchange
+their bounds and merge their lists: the ties cases check that merge against
+the lower-id rule.
 """
 import numpy as np
 import pytest
@@ -34,9 +37,9 @@ def _operand(kp):
 
 def _rows(N, K, Hq, rng):
     """Sampled positions: random ones plus both sides of every length at
-    which the bound changes (n = 8K, 16K, 32K, 128K candidates)."""
+    which a bound changes (n = 8K, 16K, 32K, 64K, 128K candidates)."""
     pos = set(rng.integers(0, N, 192).tolist()) | {0, 1, C - 1, C, 2 * C, N - 1}
-    for mult in (8, 16, 32, 128):
+    for mult in (8, 16, 32, 64, 128):
         for n in (mult * K - 1, mult * K, mult * K + 1):
             for off in (0, C - 1):
                 p = n * C + off
@@ -73,7 +76,7 @@ def test_select_exact_on_representable_scores(kind, K):
     ids = torch.empty((B, Hq, N, K), dtype=torch.int32, device="cuda")
     sc = torch.empty((B, Hq, N, K), dtype=torch.float32, device="cuda")
     dummy = torch.zeros((1,), dtype=torch.float32, device="cuda")
-    hils.hils_select(dims, q_dev, dummy, dummy, op, ids, sc)
+    hils.hils_select(dims, q_dev, dummy, dummy, op, None, 0, ids, sc)
     torch.cuda.synchronize()
     assert hils.hils_get_status() == 0
 
