@@ -5,9 +5,13 @@
 One step = one pass of the whole path over one batch of synthetic input
 already resident in HBM: landmark summary (a) -> chunk scoring + top-K (b) ->
 sparse prefill attention with fusion (c) -> one decode step at full length
-(d).  Prints ONE JSON line (rank 0).  For N > 1 (torchrun) every rank runs
-the same independent workload (weak scaling, no collective on the data path);
-the time is the max over ranks.
+(d).  Prints ONE JSON line (rank 0).  The default run also times, in the same
+process, the batch-8 GQA decode step and the 7B-shaped GQA prefill (the line's
+"extra").  For N > 1 (torchrun) the ranks split one problem: rank r takes a
+contiguous range of (batch, kv head) groups of a prefill, or of the sequences
+of a decode batch (chunk_wise_sparse_b200/partition.py), and runs the same C
+ABI calls on its slice; no collective runs on the data path (strong scaling:
+the job is the whole workload, its time the max over ranks).
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
 method: there is no other implementation to run) on a bounded sample of the
@@ -156,10 +160,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_sample(w, inp, budget_s=15.0):
+def cpu_oracle_sample(w, inp, budget_s=15.0, info=None):
     """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
     the summaries of a head subset plus sampled prefill rows.  Returns
-    (tokens/s, description, threads)."""
+    (tokens/s, description, threads); `info` (a dict) gets the rows and the
+    seconds the sample took."""
     from oracle.oracle import Oracle, Rows, max_threads, qcal
     o = Oracle.for_workload(w)
     if w.qcal:
@@ -195,6 +200,8 @@ def cpu_oracle_sample(w, inp, budget_s=15.0):
         n = min(2 * n, 4096)
     t_per_row = elapsed / done
     t_token = t_summary / w.N + t_per_row * w.Hq * w.B
+    if info is not None:
+        info.update(rows=done, row_seconds=elapsed, summary_seconds=t_sum_head)
     desc = (f"fp64 oracle: summaries of 1 of {w.B * w.Hkv} (b, kv head) slabs ({t_sum_head:.2f} s, scaled), "
             f"select+attend of {done} sampled rows of head 0 ({elapsed:.1f} s); tokens/s = 1 / (summary "
             f"time per token + row time x {w.B * w.Hq} rows per token)")
@@ -253,20 +260,36 @@ def cpu_oracle_backward(w, inp):
 
 
 def run_reference(args, w, rank):
+    """The reference arm: the fp64 oracle as it stands, on the host cores, each
+    step a bounded sample of the workload (about --ref-budget seconds of rows),
+    extrapolated to the whole workload for `value`.  steps / ms_per_step are
+    the sample steps actually run and their wall time."""
     if rank != 0:
         return
     inp = generate(w)
-    vals = []
     for _ in range(args.warmup):
         cpu_oracle_sample(w, inp, budget_s=2.0)
+    vals, walls, infos = [], [], []
     for _ in range(args.steps):
-        v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget)
+        info = {}
+        t0 = time.perf_counter()
+        v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget, info=info)
+        walls.append(time.perf_counter() - t0)
         vals.append(v)
+        infos.append(info)
     value = float(np.mean(vals))
+    ms_step = 1e3 * float(np.mean(walls))
+    full_ms = 1e3 * w.B * w.N / value          # the whole workload at the sampled rate
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.B * w.N / value,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, args.gpus),
+            "extrapolated": True,
+            "extrapolation": {"sampled_rows_per_step": int(np.mean([i["rows"] for i in infos])),
+                              "sampled_row_seconds_per_step": float(np.mean([i["row_seconds"] for i in infos])),
+                              "workload_ms_at_sampled_rate": full_ms, "scale_factor": full_ms / ms_step,
+                              "note": "each step times a bounded sample; value is the sampled rate applied to "
+                                      "the whole workload"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -306,10 +329,134 @@ def workload_config(w, n_gpus):
         "and ms_per_step is the sum of the kernel events"
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "C": w.C, "K": w.K,
             "window": w.window, "qcal_rank": w.qcal, "needles": w.needles, "seed": w.seed,
-            "parallelism": f"dp{n_gpus} (independent replicas)", "l2": l2}
+            "parallelism": ("1 GPU" if n_gpus == 1 else
+                            f"{n_gpus} GPUs, one problem split by " +
+                            ("sequence" if w.kind == "decode" else "(batch, kv head) group") +
+                            ", no collective on the data path"), "l2": l2}
+
+
+def rank_slices(w, world, rank):
+    """The sub-problems rank runs: its (b, kv head) groups of a prefill as
+    runs of consecutive kv heads (each one independent problem of batch 1),
+    or its sequences of a decode batch.  One rank: the whole workload."""
+    from chunk_wise_sparse_b200.partition import decode_slice, prefill_slices
+    if world == 1:
+        return [None]
+    if w.kind == "decode":
+        b_lo, b_hi = decode_slice(w.B, world, rank)
+        return [("b", b_lo, b_hi)] if b_hi > b_lo else []
+    return [("h", s.b, s.h_lo, s.h_hi) for s in prefill_slices(w.B, w.Hkv, world, rank)]
+
+
+def slice_inputs(w, inp, sl):
+    """(workload, inputs) of one sub-problem of rank_slices: views of the host
+    arrays of the groups or sequences it covers (no arithmetic)."""
+    import dataclasses
+    from chunk_wise_sparse_b200.inputs import Inputs
+    if sl is None:
+        return w, inp
+    if sl[0] == "b":
+        _, b0, b1 = sl
+        cut = {n: lambda a, b0=b0, b1=b1: None if a is None else a[b0:b1] for n in ("q", "k", "v", "lq")}
+        ws = dataclasses.replace(w, B=b1 - b0)
+    else:
+        _, b, h0, h1 = sl
+        G = w.G
+        cut = {"q": lambda a: None if a is None else a[b:b + 1, h0 * G:h1 * G]}
+        for n in ("k", "v", "lq"):
+            cut[n] = lambda a: None if a is None else a[b:b + 1, h0:h1]
+        ws = dataclasses.replace(w, B=1, Hq=(h1 - h0) * G, Hkv=h1 - h0)
+    kw = {}
+    for n in ("q", "k", "v", "lq"):
+        kw[n + "_f32"] = np.ascontiguousarray(cut[n](getattr(inp, n + "_f32")))
+        bits = getattr(inp, n + "_bits")
+        kw[n + "_bits"] = None if bits is None else np.ascontiguousarray(cut[n](bits))
+    return ws, Inputs(ws, kw["q_f32"], kw["k_f32"], kw["v_f32"], kw["lq_f32"], inp.needle_chunks, inp.needle_blocks,
+                      kw["q_bits"], kw["k_bits"], kw["v_bits"], kw["lq_bits"])
+
+
+class PrefillSlice:
+    """Device buffers and C ABI calls of one prefill sub-problem (the whole
+    workload on one rank, or a rank's run of (b, kv head) groups)."""
+
+    def __init__(self, w, inp, dev, hils):
+        import torch
+        self.w, self.inp, self.dev, self.h = w, inp, dev, hils
+        self.q, self.k, self.v, self.lq = (self.to_dev(n) for n in ("q", "k", "v", "lq"))
+        B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
+        self.dims = hils.dims_for(self.q, self.k, K, w.window)
+        self.summ = hils.Summary(self.dims, dev)
+        self.ids = torch.empty((B, Hq, N, K), dtype=torch.int32, device=dev)
+        self.scores = torch.empty((B, Hq, N, K), dtype=torch.float32, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        self.qd = self.q[:, :, -1, :].contiguous()
+        self.seq = torch.full((B,), N, dtype=torch.int32, device=dev)
+        self.ddims = hils.make_dims(B, Hq, Hkv, d, N, K, self.q.dtype, window=w.window)
+        self.ws = torch.empty((hils.hils_decode_workspace_bytes(self.ddims),), dtype=torch.uint8, device=dev)
+        self.pws = hils.prefill_workspace(self.dims, dev)
+        self.od = torch.empty_like(self.qd)
+        self.ids_d = torch.empty((B, Hq, K), dtype=torch.int32, device=dev)
+        self.sc_d = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
+        self.use_qcal = w.qcal > 0
+        if self.use_qcal:
+            # Q-Cal projections (random init, resident like model weights); the
+            # prefill scores with q^, the decode step with the calibrated last row
+            from chunk_wise_sparse_b200.inputs import qcal_weights
+            wt = qcal_weights(Hq, d, w.qcal, seed=w.seed, dtype=w.dtype)
+            if wt.w_down_bits is not None:
+                self.wd = torch.from_numpy(wt.w_down_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+                self.wu = torch.from_numpy(wt.w_up_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+            else:
+                self.wd, self.wu = torch.from_numpy(wt.w_down_f32).to(dev), torch.from_numpy(wt.w_up_f32).to(dev)
+            self.q_hat, self.qd_hat = torch.empty_like(self.q), torch.empty_like(self.qd)
+            self.cdims = hils.make_dims(B, Hq, Hq, d, 64, 1, self.q.dtype)
+        self.cur = {"q": self.q, "k": self.k, "v": self.v, "lq": self.lq, "qd": self.qd}
+
+    def to_dev(self, name):
+        import torch
+        bits = getattr(self.inp, name + "_bits")
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).to(self.dev).view(torch.bfloat16)
+        return torch.from_numpy(getattr(self.inp, name + "_f32")).to(self.dev)
+
+    # the phases of one step, each one C ABI call (two for Q-Cal)
+    def summary(self, st):
+        t = self.cur
+        self.h.hils_landmark_summary(self.dims, t["k"], t["lq"], 0, self.w.N // 64, self.summ.kprime,
+                                     self.summ.bprime, self.summ.kprime_mma, st)
+
+    def qcal(self, st):
+        t = self.cur
+        self.h.hils_query_calibrate(self.cdims, t["q"], self.w.N, self.wd, self.wu, self.w.qcal, self.q_hat, st)
+        self.h.hils_query_calibrate(self.cdims, t["qd"], 1, self.wd, self.wu, self.w.qcal, self.qd_hat, st)
+
+    def select(self, st):
+        t, s = self.cur, self.summ
+        self.h.hils_select(self.dims, self.q_hat if self.use_qcal else t["q"], s.kprime, s.bprime, s.kprime_mma,
+                           None, 0, self.ids, self.scores, st)
+
+    def prefill(self, st):
+        t, s = self.cur, self.summ
+        self.h.hils_attn_prefill(self.dims, t["q"], t["k"], t["v"], s.kprime, s.bprime, s.kprime_mma, self.ids,
+                                 self.scores, self.o, self.lse, self.pws, stream=st)
+
+    def decode(self, st):
+        t, s = self.cur, self.summ
+        if self.use_qcal:
+            self.h.hils_attn_decode_qcal(self.ddims, t["qd"], self.qd_hat, t["k"], t["v"], None, 0, s.kprime,
+                                         s.bprime, s.kprime_mma, self.seq, self.od, self.ids_d, self.sc_d, self.ws,
+                                         stream=st)
+        else:
+            self.h.hils_attn_decode(self.ddims, t["qd"], t["k"], t["v"], s.kprime, s.bprime, s.kprime_mma, self.seq,
+                                    self.od, self.ids_d, self.sc_d, self.ws, stream=st)
 
 
 def run_ours(args, w, rank, world, local_rank):
+    """One prefill step (summary, [Q-Cal,] select, prefill, one decode step at
+    full length) per iteration.  With N ranks, rank r runs the step on its own
+    (b, kv head) groups only (partition.prefill_slices); the job is the whole
+    workload, its time the max over ranks.  Returns the JSON line (rank 0)."""
     import torch
     import torch.distributed as dist
     from chunk_wise_sparse_b200 import hils
@@ -318,78 +465,22 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.set_device(dev)
     hils.lib()
     inp = generate(w)
-
-    def to_dev(name):
-        bits = getattr(inp, name + "_bits")
-        if bits is not None:
-            return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(getattr(inp, name + "_f32")).to(dev)
-
-    q, k, v, lq = (to_dev(n) for n in ("q", "k", "v", "lq"))
+    parts = [PrefillSlice(*slice_inputs(w, inp, sl), dev, hils) for sl in rank_slices(w, world, rank)]
     B, Hq, Hkv, N, d, K = w.B, w.Hq, w.Hkv, w.N, w.d, w.K
-    dims = hils.dims_for(q, k, K, w.window)
-    summ = hils.Summary(dims, dev)
-    ids = torch.empty((B, Hq, N, K), dtype=torch.int32, device=dev)
-    scores = torch.empty((B, Hq, N, K), dtype=torch.float32, device=dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
-    qd = q[:, :, -1, :].contiguous()
-    seq = torch.full((B,), N, dtype=torch.int32, device=dev)
-    ddims = hils.make_dims(B, Hq, Hkv, d, N, K, q.dtype, window=w.window)
-    ws = torch.empty((hils.hils_decode_workspace_bytes(ddims),), dtype=torch.uint8, device=dev)
-    pws = hils.prefill_workspace(dims, dev)
-    od = torch.empty_like(qd)
-    ids_d = torch.empty((B, Hq, K), dtype=torch.int32, device=dev)
-    sc_d = torch.empty((B, Hq, K), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     flush = None if inputs_exceed_l2(w) else torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
     use_qcal = w.qcal > 0
-    if use_qcal:
-        # Q-Cal projections (random init, resident like model weights); the
-        # prefill scores with q^, the decode step with the calibrated last row
-        from chunk_wise_sparse_b200.inputs import qcal_weights
-        wt = qcal_weights(Hq, d, w.qcal, seed=w.seed, dtype=w.dtype)
-        if wt.w_down_bits is not None:
-            wd = torch.from_numpy(wt.w_down_bits.view(np.int16)).to(dev).view(torch.bfloat16)
-            wu = torch.from_numpy(wt.w_up_bits.view(np.int16)).to(dev).view(torch.bfloat16)
-        else:
-            wd, wu = torch.from_numpy(wt.w_down_f32).to(dev), torch.from_numpy(wt.w_up_f32).to(dev)
-        q_hat, qd_hat = torch.empty_like(q), torch.empty_like(qd)
-        cdims = hils.make_dims(B, Hq, Hq, d, 64, 1, q.dtype)
     names = ["summary"] + (["qcal"] if use_qcal else []) + ["select", "prefill", "decode"]
     n_ev = len(names) + 1
 
-    def step_on(q, k, v, lq, qd, ev=None):
-        e = [0]
-
-        def mark():
-            if ev: ev[e[0]].record(stream)
-            e[0] += 1
-
+    def step(ev=None):
         if flush is not None:
             flush.fill_(1)
-        mark()
-        hils.hils_landmark_summary(dims, k, lq, 0, N // 64, summ.kprime, summ.bprime, summ.kprime_mma, stream)
-        mark()
-        if use_qcal:
-            hils.hils_query_calibrate(cdims, q, N, wd, wu, w.qcal, q_hat, stream)
-            hils.hils_query_calibrate(cdims, qd, 1, wd, wu, w.qcal, qd_hat, stream)
-            mark()
-        hils.hils_select(dims, q_hat if use_qcal else q, summ.kprime, summ.bprime, summ.kprime_mma, ids, scores,
-                         stream)
-        mark()
-        hils.hils_attn_prefill(dims, q, k, v, ids, scores, o, lse, pws, stream=stream)
-        mark()
-        if use_qcal:
-            hils.hils_attn_decode_qcal(ddims, qd, qd_hat, k, v, None, 0, summ.kprime, summ.bprime, summ.kprime_mma,
-                                       seq, od, ids_d, sc_d, ws, stream=stream)
-        else:
-            hils.hils_attn_decode(ddims, qd, k, v, summ.kprime, summ.bprime, summ.kprime_mma, seq, od, ids_d, sc_d,
-                                  ws, stream=stream)
-        mark()
-
-    def step(ev=None):
-        step_on(q, k, v, lq, qd, ev)
+        if ev: ev[0].record(stream)
+        for j, name in enumerate(names):
+            for pt in parts:
+                getattr(pt, name)(stream)
+            if ev: ev[j + 1].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -423,53 +514,61 @@ def run_ours(args, w, rank, world, local_rank):
     ms_step = total_ms / args.steps
     if flush is not None:
         ms_step = max_over_ranks(float(per.sum(axis=1).mean()), world, dev)
-    value = job_throughput(world, B * N, ms_step)
+    value = B * N / (ms_step / 1e3)    # the whole job's tokens, all ranks together
 
     # end to end through the public API: every step copies its inputs from
     # pinned host memory and reads its outputs back.  Two device input sets:
     # step i+1's inputs are copied (on a copy stream) while step i computes.
     e2e = None
     if not args.no_e2e:
-        host = {n: getattr(inp, n + "_bits") if getattr(inp, n + "_bits") is not None else getattr(inp, n + "_f32")
-                for n in ("q", "k", "v", "lq")}
-        pinned = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
-                  for n, a in host.items()}
-        sets = [{"q": q, "k": k, "v": v, "lq": lq, "qd": qd},
-                {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
-                 "lq": torch.empty_like(lq), "qd": torch.empty_like(qd)}]
-        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        od_host = torch.empty(od.shape, dtype=od.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-        d2h = o_host.numel() * o_host.element_size() + od_host.numel() * od_host.element_size()
         copy_stream = torch.cuda.Stream(device=dev)
         copied = [torch.cuda.Event() for _ in range(2)]
         done = [torch.cuda.Event() for _ in range(2)]
+        h2d = d2h = 0
+        for pt in parts:
+            host = {n: getattr(pt.inp, n + "_bits") if getattr(pt.inp, n + "_bits") is not None else
+                    getattr(pt.inp, n + "_f32") for n in ("q", "k", "v", "lq")}
+            pt.pinned = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
+                         for n, a in host.items()}
+            pt.sets = [{"q": pt.q, "k": pt.k, "v": pt.v, "lq": pt.lq, "qd": pt.qd},
+                       {"q": torch.empty_like(pt.q), "k": torch.empty_like(pt.k), "v": torch.empty_like(pt.v),
+                        "lq": torch.empty_like(pt.lq), "qd": torch.empty_like(pt.qd)}]
+            pt.o_host = torch.empty(pt.o.shape, dtype=pt.o.dtype).pin_memory()
+            pt.od_host = torch.empty(pt.od.shape, dtype=pt.od.dtype).pin_memory()
+            h2d += sum(t.numel() * t.element_size() for t in pt.pinned.values())
+            d2h += pt.o_host.numel() * pt.o_host.element_size() + pt.od_host.numel() * pt.od_host.element_size()
 
-        def h2d_into(t):
-            for n, src in pinned.items():
-                t[n].view(torch.int16 if t[n].dtype == torch.bfloat16 else t[n].dtype).copy_(src, non_blocking=True)
+        def h2d_into(k):
+            for pt in parts:
+                for n, src in pt.pinned.items():
+                    t = pt.sets[k][n]
+                    t.view(torch.int16 if t.dtype == torch.bfloat16 else t.dtype).copy_(src, non_blocking=True)
 
         def run_e2e(n_steps):
             for ev in done:
                 ev.record(stream)
             copy_stream.wait_stream(stream)
             with torch.cuda.stream(copy_stream):
-                h2d_into(sets[0])
+                h2d_into(0)
                 copied[0].record(copy_stream)
             for i in range(n_steps):
                 cur, nxt = i % 2, (i + 1) % 2
                 if i + 1 < n_steps:
                     copy_stream.wait_event(done[nxt])   # the step that last read set nxt is done
                     with torch.cuda.stream(copy_stream):
-                        h2d_into(sets[nxt])
+                        h2d_into(nxt)
                         copied[nxt].record(copy_stream)
                 stream.wait_event(copied[cur])
-                t = sets[cur]
-                t["qd"].copy_(t["q"][:, :, -1, :])   # the decode query is the step's last prefill row
-                step_on(t["q"], t["k"], t["v"], t["lq"], t["qd"])
-                o_host.copy_(o, non_blocking=True)
-                od_host.copy_(od, non_blocking=True)
+                for pt in parts:
+                    pt.cur = pt.sets[cur]
+                    pt.cur["qd"].copy_(pt.cur["q"][:, :, -1, :])   # the decode query is the step's last prefill row
+                step()
+                for pt in parts:
+                    pt.o_host.copy_(pt.o, non_blocking=True)
+                    pt.od_host.copy_(pt.od, non_blocking=True)
                 done[cur].record(stream)
+            for pt in parts:
+                pt.cur = pt.sets[0]
 
         run_e2e(2)
         torch.cuda.synchronize()
@@ -482,23 +581,30 @@ def run_ours(args, w, rank, world, local_rank):
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a0.elapsed_time(a1) / n_e2e, world, dev)
-        e2e = {"value": job_throughput(world, B * N, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": B * N / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
                "overlap": "step i+1's host-to-device copies run on a copy stream during step i"}
+        if world > 1:
+            e2e["bytes_note"] = "h2d / d2h bytes of rank 0's slice"
     if rank != 0:
-        return
+        return None
 
-    work = useful_work(w)
+    # the work and the kernel fractions are those of rank 0's share of the job
+    w0 = parts[0].w if len(parts) == 1 else w
+    work = useful_work(w0)
+    if len(parts) > 1:
+        work = {key: sum(useful_work(pt.w)[key] for pt in parts) for key in work}
     peaks = load_peaks()
     avg = per.mean(axis=0)
     kernels_ms = {n: float(a) for n, a in zip(names, avg)}
     dom = names[int(np.argmax(avg))]
+    rows0 = sum(pt.w.B * pt.w.Hq * N for pt in parts)
     if dom in ("select", "prefill"):
         fl = work["flops_score"] if dom == "select" else work["flops_attn"]
         ach = fl / (kernels_ms[dom] / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                "traffic": recorded_traffic(dom, B * w.Hq * N),
+                "traffic": recorded_traffic(dom, rows0),
                 "peak_source": peaks["source"] + " bf16 dense burst"}
     else:
         by = work["bytes_summary"]
@@ -509,7 +615,7 @@ def run_ours(args, w, rank, world, local_rank):
     bc_ms = kernels_ms["select"] + kernels_ms["prefill"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
         "data": f"synthetic: i.i.d. N(0,1) Q/K/V/landmark queries, {w.needles} planted needle chunks, seed {w.seed}",
         "config": workload_config(w, world),
@@ -524,16 +630,19 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clk,
         "e2e": e2e,
     }
+    if world > 1:
+        line["rank0_share"] = {"slices": [list(sl) for sl in rank_slices(w, world, 0)],
+                               "note": "kernels_ms, roofline and the (b)+(c) fraction are rank 0's share"}
     if use_qcal:
         eb = 2 if w.dtype == "bf16" else 4
-        qb = 2 * B * Hq * (N + 1) * d * eb     # q read and q^ written (prefill rows and the decode row)
+        qb = sum(2 * pt.w.B * pt.w.Hq * (N + 1) * d * eb for pt in parts)   # q read and q^ written
         line["qcal"] = {"rank": w.qcal, "ms": kernels_ms["qcal"], "bytes": qb,
                         "gbs": qb / (kernels_ms["qcal"] / 1e3) / 1e9,
                         "frac_of_hbm": qb / (kernels_ms["qcal"] / 1e3) / 1e9 / peaks["hbm_gbs"]}
     if not args.no_cpu_baseline and world == 1:
         v, desc, threads = cpu_oracle_sample(w, inp, budget_s=args.ref_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def decode_selected_bytes(ids, w):
@@ -658,7 +767,11 @@ def run_decode(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     hils.lib()
-    inp = generate(w)
+    w_job = w
+    sl = rank_slices(w, world, rank)
+    if not sl:
+        raise RuntimeError(f"rank {rank}: no sequence of the batch of {w.B} to decode")
+    w, inp = slice_inputs(w_job, generate(w_job), sl[0])   # this rank's sequences
 
     def to_dev(name):
         bits = getattr(inp, name + "_bits")
@@ -772,7 +885,7 @@ def run_decode(args, w, rank, world, local_rank):
         e2e = {"value": e_us, "unit": "us/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "steps back to back, no L2 flush between them"}
     if rank != 0:
-        return
+        return None
     sel_bytes = decode_selected_bytes(ids.cpu().numpy(), w)
     kp_bytes = B * Hkv * w.nc * (d + 16) * 2
     peaks = load_peaks()
@@ -781,10 +894,10 @@ def run_decode(args, w, rank, world, local_rank):
     line = {
         "metric": "HiLS decode us/step (one new token per sequence: scoring, top-K, sparse attention)",
         "value": us, "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "fp32",
         "data": f"synthetic: i.i.d. N(0,1), seed {w.seed}" + (", KV cache in chunk pages (random order)" if w.paged else ""),
-        "config": dict(workload_config(w, world), l2="256 MiB buffer written between steps (L2 flush)"),
+        "config": dict(workload_config(w_job, world), l2="256 MiB buffer written between steps (L2 flush)"),
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "traffic": recorded_step_traffic("decode", w.name),
@@ -795,11 +908,39 @@ def run_decode(args, w, rank, world, local_rank):
         "e2e": e2e,
         "median_us_of_100_more_steps": us_100,
     }
+    if world > 1:
+        line["rank0_share"] = {"sequences": list(sl[0][1:]),
+                               "note": "the roofline bytes and the e2e copies are rank 0's sequences"}
     if not args.no_cpu_baseline and world == 1:
         v_cpu, desc, threads = cpu_oracle_decode(w, inp, budget_s=args.ref_budget)
         line["cpu_baseline"] = {"value": v_cpu, "unit": "us/step", "cores": threads, "kind": "oracle",
                                 "sample": desc}
-    print(json.dumps(line), flush=True)
+    return line
+
+
+# Workloads the default run also times, each in the same process after the
+# headline workload, reported under "extra": the batch-8 GQA decode step and
+# the 7B-shaped GQA prefill.
+EXTRA_WORKLOADS = ("decode-128k-b8-gqa4-d128", "prefill-128k-gqa4-d128")
+EXTRA_KEYS = ("value", "unit", "steps", "warmup", "ms_per_step", "higher_is_better", "kernels_ms",
+              "decode_us_per_step", "prefill_bc_tflops_useful", "prefill_bc_frac_of_bf16_peak", "roofline",
+              "gpu_launches", "clocks", "e2e", "median_us_of_100_more_steps", "config", "rank0_share")
+
+
+def run_extra(args, name, rank, world, local_rank):
+    import copy
+    import torch
+    w = WORKLOADS[name]
+    a = copy.copy(args)
+    a.no_cpu_baseline = True
+    if w.kind == "decode":
+        a.steps, a.warmup = max(args.steps, 50), max(args.warmup, 5)
+        line = run_decode(a, w, rank, world, local_rank)
+    else:
+        a.no_e2e = True
+        line = run_ours(a, w, rank, world, local_rank)
+    torch.cuda.empty_cache()
+    return None if line is None else {k: line[k] for k in EXTRA_KEYS if k in line}
 
 
 def main():
@@ -807,14 +948,17 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=list(WORKLOADS),
+                    help=f"default {DEFAULT_WORKLOAD}, plus the extra workloads {', '.join(EXTRA_WORKLOADS)}")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="time the headline workload only")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--backward", action="store_true", help="time the backward pass of a prefill workload")
     args = ap.parse_args()
-    w = WORKLOADS[args.workload]
+    extras = args.workload is None and not args.no_extras and not args.backward
+    w = WORKLOADS[args.workload or DEFAULT_WORKLOAD]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -830,10 +974,14 @@ def main():
     try:
         if args.backward:
             run_backward(args, w, rank, world, local_rank)
-        elif w.kind == "decode":
-            run_decode(args, w, rank, world, local_rank)
-        else:
-            run_ours(args, w, rank, world, local_rank)
+            return
+        line = (run_decode if w.kind == "decode" else run_ours)(args, w, rank, world, local_rank)
+        if extras:
+            ex = {name: run_extra(args, name, rank, world, local_rank) for name in EXTRA_WORKLOADS}
+            if line is not None:
+                line["extra"] = ex
+        if line is not None:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist
