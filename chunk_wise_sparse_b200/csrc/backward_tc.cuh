@@ -55,6 +55,10 @@ struct BwdTc {
   // TMEM columns: [0, 64) S then dK^T, [64, 128) dP then dV^T, [128, 128 + d) dQ
   static constexpr uint32_t T_S = 0, T_P = 64, T_Q = 128;
   static constexpr uint32_t TMEM_COLS = 256;
+  // more CTAs than 512 / TMEM_COLS per SM (228 KB of shared memory, 1 KB
+  // reserved per CTA) could make a tcgen05.alloc wait for columns that a
+  // co-resident CTA never frees
+  static_assert((512 / TMEM_COLS + 1) * (SMEM + 1024) > 233472u, "TMEM never oversubscribed");
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16(M, kChunk);
   static constexpr uint32_t IDESC_Q = sm100::idesc_bf16(M, D) | (1u << 16);                  // B MN-major
   static constexpr uint32_t IDESC_T = sm100::idesc_bf16(M, kChunk) | (1u << 15) | (1u << 16);   // A, B MN-major

@@ -161,6 +161,9 @@ int launch_select_tc(const hils_dims* d, const void* q, const void* kmma, int32_
     while (cap + 8 <= 128 && C::layout(d->topk, stages, cap + 8).total <= per_cta) cap += 8;
   const uint32_t smem = C::layout(d->topk, stages, cap).total;
   if (smem > uint32_t(kMaxSmem)) return HILS_ERR_UNSUPPORTED;
+  // no more CTAs per SM than 512 TMEM columns hold (a tcgen05.alloc would
+  // otherwise wait for columns a co-resident persistent CTA never frees)
+  if ((512u / C::TMEM_COLS + 1u) * (smem + 1024u) <= 233472u) return HILS_ERR_UNSUPPORTED;
   constexpr auto fn = select_tc_kernel<D, KCAP>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   SelTcParams p;

@@ -124,6 +124,10 @@ struct CcOwn {
   static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
   // S (NK <= 128 columns) is read out before P V overwrites its first D columns
   static constexpr uint32_t TMEM_COLS = 128;
+  // more CTAs than 512 / TMEM_COLS per SM (228 KB of shared memory, 1 KB
+  // reserved per CTA) could make a tcgen05.alloc wait for columns that a
+  // co-resident CTA never frees
+  static_assert((512 / TMEM_COLS + 1) * (SMEM + 1024) > 233472u, "TMEM never oversubscribed");
 };
 
 struct CcOwnParams {
@@ -747,6 +751,7 @@ struct CcTc {
   // columns that a co-resident persistent CTA never frees
   static constexpr uint32_t SMEM_FLOOR = 233472u / (MAX_CTAS + 1) + 1024u;
   static constexpr uint32_t SMEM = SMEM_MIN > SMEM_FLOOR ? SMEM_MIN : SMEM_FLOOR;
+  static_assert((512 / TMEM_COLS + 1) * (SMEM + 1024) > 233472u, "TMEM never oversubscribed");
   static constexpr uint32_t TX_BYTES = M * D * 2 + 2 * K_BYTES;
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16(M, kChunk);
   // P (K-major) x V (MN-major: d contiguous in each key row)

@@ -57,6 +57,10 @@ struct CcLocal {
   // S[2] x 64 columns, then O (D columns).  Shared memory holds at most two
   // CTAs per SM (d = 64) or one (d = 128), so 256 columns each always fit.
   static constexpr uint32_t TMEM_COLS = 256;
+  // more CTAs than 512 / TMEM_COLS per SM (228 KB of shared memory, 1 KB
+  // reserved per CTA) could make a tcgen05.alloc wait for columns that a
+  // co-resident CTA never frees
+  static_assert((512 / TMEM_COLS + 1) * (SMEM + 1024) > 233472u, "TMEM never oversubscribed");
   static constexpr uint32_t T_O = 2 * kChunk;
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16(M, kChunk);
   static constexpr uint32_t IDESC_O = sm100::idesc_bf16(M, D) | (1u << 16);   // V is MN-major
