@@ -400,10 +400,13 @@ decode_topk_reg_kernel(const float* __restrict__ ws_scores, const int32_t* __res
 // lists, one lane per head), brings the chunk's 64 key and value rows into
 // shared memory with all copies in flight at once (cp.async, 16 bytes per
 // copy; keys with the 16-byte blocks of row r rotated by r mod 8 so that the
-// key-per-lane reads hit distinct banks), then, four heads at a time,
-// computes the scores (lanes own keys), the softmax (warp reductions) and
-// P V (lanes own dims, weights broadcast by shuffle).  Each head's partial
-// goes to its own slot; invalid slots get score -inf.
+// key-per-lane reads hit distinct banks), then, one head that kept it at a
+// time, the four warps split the 64 keys: each scores its 16 keys (two lanes
+// per key, half of the dimensions each), takes their maximum and sum, and
+// accumulates their weighted values (lanes own dims, weights broadcast by
+// shuffle); the four partial results merge through shared memory.  A chunk
+// is usually kept by one head only, so this keeps all four warps busy.
+// Each head's partial goes to its own slot; invalid slots get score -inf.
 template <typename T, int D>
 struct DecUnion {
   static constexpr int RB = D * int(sizeof(T));   // bytes per key / value row
@@ -412,9 +415,11 @@ struct DecUnion {
   // keys, values, queries, kept ids, then per-head slots and a flag (all dynamic:
   // the kernel may be given the largest dynamic size, which leaves no room
   // for static shared memory)
+  // per warp: its keys' maximum, sum and partial output row (D + 4 floats)
+  static constexpr int RED = D + 4;
   static size_t smem(int G, int K) {
     return 2 * size_t(TILE) + sizeof(float) * size_t(G) * D + sizeof(int32_t) * size_t(G) * K +
-           sizeof(int32_t) * 36 + 16;
+           sizeof(int32_t) * 36 + 16 + sizeof(float) * 4 * RED + 16;
   }
 };
 
@@ -460,6 +465,8 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   int* s_slot = sid + G * K;   // [32] per head: the chunk's slot in its list, -1 if not kept
   int& s_go = s_slot[32];
   int* s_off = s_slot + 34;   // [2] element offset of the chunk's rows, low and high words
+  // [4][RED] per-warp softmax statistics and partial outputs, 16-byte aligned
+  float* s_red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_slot + 36) + 15) & ~uintptr_t(15));
   pdl_wait();      // the top-K lists
   pdl_trigger();
   const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
@@ -573,57 +580,83 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   }
   cp_async_wait_all();
   __syncthreads();
-  const int ra = lane, rb = lane + 32;
-  const bool va = j0 + ra < j1, vb = j0 + rb < j1;
-  for (int g = warp; g < G; g += 4) {
+  // The heads that kept the chunk are taken one at a time by all four warps:
+  // warp w scores and weighs the chunk's keys 16w .. 16w+15 (lanes l and
+  // l+16 share key 16w + l%16, each summing half of the dimensions), keeps its
+  // keys' maximum and sum, and accumulates their weighted values; the four
+  // partial results are then merged through shared memory.  (Most chunks are
+  // kept by one head of the kv head, so spreading a head's keys over the
+  // warps, rather than one head per warp, keeps all four warps busy.)
+  const int key = warp * 16 + (lane & 15), half = lane >> 4;
+  const bool vk = j0 + key < j1;
+  float* my_red = s_red + warp * U::RED;
+  for (int g = 0; g < G; ++g) {
     const int slot = s_slot[g];
-    if (slot < 0) continue;   // warp-uniform
-    // scores of the lane's two keys
-    float sa = 0.f, sb = 0.f;
+    if (slot < 0) continue;   // the same for the whole CTA
     const float* qg = sq + g * D;
-#pragma unroll 4
-    for (int blk = 0; blk < U::NB; ++blk) {
-      float xa[EB], xb[EB];
-      lds16<T>(sk_a + uint32_t(ra * U::RB + ((blk ^ (ra & 7)) << 4)), xa);
-      lds16<T>(sk_a + uint32_t(rb * U::RB + ((blk ^ (rb & 7)) << 4)), xb);
+    float sd = 0.f;
 #pragma unroll
-      for (int e = 0; e < EB; ++e) {
-        sa = fmaf(qg[blk * EB + e], xa[e], sa);
-        sb = fmaf(qg[blk * EB + e], xb[e], sb);
-      }
+    for (int bb = 0; bb < U::NB / 2; ++bb) {
+      const int blk = half * (U::NB / 2) + bb;
+      float x[EB];
+      lds16<T>(sk_a + uint32_t(key * U::RB + ((blk ^ (key & 7)) << 4)), x);
+#pragma unroll
+      for (int e = 0; e < EB; ++e) sd = fmaf(qg[blk * EB + e], x[e], sd);
     }
-    // softmax over the chunk's keys (keys after the query excluded)
-    const float za = va ? sa * tau : -INFINITY, zb = vb ? sb * tau : -INFINITY;
-    float m = fmaxf(za, zb);
+    sd += __shfl_xor_sync(0xffffffffu, sd, 16);
+    const float z = vk ? sd * tau : -INFINITY;
+    float m = z;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float pa = va ? expf(za - m) : 0.f, pb = vb ? expf(zb - m) : 0.f;
-    float l = pa + pb;
+    for (int off = 8; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float pk = (vk && m > -INFINITY) ? expf(z - m) : 0.f;
+    float l = pk;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    // P V: lane owns dims lane * EL .. + EL - 1
+    for (int off = 8; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    // the warp's 16 keys' weighted values: lane owns dims lane * EL .. + EL - 1
     float o[EL];
 #pragma unroll
     for (int e = 0; e < EL; ++e) o[e] = 0.f;
-    const int nk = int(j1 - j0);
-#pragma unroll 8
-    for (int jj = 0; jj < nk; ++jj) {
-      const T* vrow = reinterpret_cast<const T*>(sv + jj * U::RB) + lane * EL;
-      const float pj = __shfl_sync(0xffffffffu, jj < 32 ? pa : pb, jj & 31);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const T* vrow = reinterpret_cast<const T*>(sv + (warp * 16 + jj) * U::RB) + lane * EL;
+      const float pj = __shfl_sync(0xffffffffu, pk, jj);
 #pragma unroll
       for (int e = 0; e < EL; ++e) {
-        float x;
-        if constexpr (sizeof(T) == 2) x = __bfloat162float(vrow[e]);
-        else x = vrow[e];
-        o[e] = fmaf(pj, x, o[e]);
+        float xv;
+        if constexpr (sizeof(T) == 2) xv = __bfloat162float(vrow[e]);
+        else xv = vrow[e];
+        o[e] = fmaf(pj, xv, o[e]);
       }
     }
-    const int64_t row = row0 + g;
-    float* po = part_o + (row * PS + slot) * D + lane * EL;
-    const float inv = 1.f / l;
 #pragma unroll
-    for (int e = 0; e < EL; ++e) po[e] = o[e] * inv;
-    if (lane == 0) part_u[row * PS + slot] = slot >= K ? m + logf(l) : sel_scores[row * K + slot];
+    for (int e = 0; e < EL; ++e) my_red[lane * EL + e] = o[e];
+    if (lane == 0) {
+      my_red[D] = m;
+      my_red[D + 1] = l;
+    }
+    __syncthreads();
+    // merge the four warps: M = max m_w, L = sum l_w e^(m_w - M), O = sum o_w e^(m_w - M) / L
+    float mw[4], M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      mw[w] = s_red[w * U::RED + D];
+      M = fmaxf(M, mw[w]);
+    }
+    float L = 0.f, f[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      f[w] = mw[w] > -INFINITY ? expf(mw[w] - M) : 0.f;
+      L = fmaf(s_red[w * U::RED + D + 1], f[w], L);
+    }
+    const int64_t row = row0 + g;
+    if (tid < D) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) acc = fmaf(s_red[w * U::RED + tid], f[w], acc);
+      part_o[(row * PS + slot) * D + tid] = acc / L;
+    }
+    if (tid == 0) part_u[row * PS + slot] = slot >= K ? M + logf(L) : sel_scores[row * K + slot];
+    __syncthreads();   // s_red is reused by the next head
   }
 }
 
