@@ -394,32 +394,38 @@ decode_topk_reg_kernel(const float* __restrict__ ws_scores, const int32_t* __res
 // D3, grouped by kv head: the G query heads of a kv head select overlapping
 // chunk sets, so each distinct chunk is read once and attended by all heads
 // that kept it.  One CTA per candidate slot (g, k) of the (b, kv head)'s
-// G x K selections, plus one per chunk of the local window.  A slot whose
-// chunk already appears for an earlier head is skipped; otherwise the warp
-// finds the heads that kept the chunk (binary search in their ascending id
-// lists, one lane per head), brings the chunk's 64 key and value rows into
-// shared memory with all copies in flight at once (cp.async, 16 bytes per
-// copy; keys with the 16-byte blocks of row r rotated by r mod 8 so that the
-// key-per-lane reads hit distinct banks), then, one head that kept it at a
-// time, the four warps split the 64 keys: each scores its 16 keys (two lanes
-// per key, half of the dimensions each), takes their maximum and sum, and
-// accumulates their weighted values (lanes own dims, weights broadcast by
-// shuffle); the four partial results merge through shared memory.  A chunk
-// is usually kept by one head only, so this keeps all four warps busy.
-// Each head's partial goes to its own slot; invalid slots get score -inf.
+// G x K selections, plus one per chunk of the local window.  Thread 0 reads
+// the slot's chunk id and starts the copies of its 64 key rows into shared
+// memory at once (cp.async, 16 bytes per copy, all in flight; the 16-byte
+// blocks of row r rotated by r mod 8 so that the key-per-lane reads hit
+// distinct banks), after an L2 prefetch of the key and value rows.  While
+// they land, warp 0 finds the heads that kept the chunk (binary search in
+// their ascending id lists, one lane per head); a slot whose chunk an earlier
+// head also kept is skipped (its copies are drained first).  Then, for up to
+// four kept heads at a time, the four warps split the 64 keys: each scores
+// its 16 keys (two lanes per key, half of the dimensions each) and keeps
+// their weights, maximum and sum; the value rows replace the key rows in the
+// same buffer (from L2 by then), each warp accumulates its keys' weighted
+// values (lanes own dims), and the four partial results merge through shared
+// memory.  One 64-row buffer instead of two keeps eight CTAs per SM instead
+// of six.  A chunk is usually kept by one head only, so splitting its keys
+// over the warps keeps all four busy.  Each head's partial goes to its own
+// slot; invalid slots get score -inf.
 template <typename T, int D>
 struct DecUnion {
   static constexpr int RB = D * int(sizeof(T));   // bytes per key / value row
   static constexpr int NB = RB / 16;             // 16-byte blocks per row
   static constexpr uint32_t TILE = uint32_t(kChunk) * RB;
-  // keys, values, queries, kept ids, then per-head slots and a flag (all dynamic:
+  // the key-then-value rows, queries, kept ids, per-head slots, a flag and the
+  // copy offset, the kept heads' selection scores, then per warp its keys'
+  // maximum, sum and partial output row (D + 4 floats), and per head of a
+  // batch each thread's key weight and each warp's (max, sum) (all dynamic:
   // the kernel may be given the largest dynamic size, which leaves no room
   // for static shared memory)
-  // per warp: its keys' maximum, sum and partial output row (D + 4 floats)
   static constexpr int RED = D + 4;
   static size_t smem(int G, int K) {
-    return 2 * size_t(TILE) + sizeof(float) * size_t(G) * D + sizeof(int32_t) * size_t(G) * K +
-           sizeof(int32_t) * 36 + 16 + sizeof(float) * 4 * RED + 16;
+    return size_t(TILE) + sizeof(float) * size_t(G) * D + sizeof(int32_t) * size_t(G) * K + sizeof(int32_t) * 36 +
+           sizeof(float) * 32 + 16 + sizeof(float) * 4 * RED + sizeof(float) * (4 * 128 + 4 * 4 * 2) + 16;
   }
 };
 
@@ -449,7 +455,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, sizeof(T) == 2 ? 8 : 6)
 decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                             const int32_t* __restrict__ seqlens, int64_t cap, int Hq, int G, int Hkv, int K,
                             float tau, const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
@@ -458,15 +464,19 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   constexpr int EL = D / 32;                 // output dims per lane
   constexpr int EB = 16 / int(sizeof(T));    // elements per 16-byte block
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint8_t* sk = dsm;                                            // [64][D] keys, blocks rotated
-  uint8_t* sv = dsm + U::TILE;                                  // [64][D] values
-  float* sq = reinterpret_cast<float*>(dsm + 2 * U::TILE);      // [G][D] queries
+  // one [64][D] buffer: the chunk's keys (16-byte blocks rotated), then its values
+  uint8_t* sk = dsm;
+  float* sq = reinterpret_cast<float*>(dsm + U::TILE);          // [G][D] queries
   int32_t* sid = reinterpret_cast<int32_t*>(sq + G * D);        // [G][K] kept ids, ascending
   int* s_slot = sid + G * K;   // [32] per head: the chunk's slot in its list, -1 if not kept
   int& s_go = s_slot[32];
-  int* s_off = s_slot + 34;   // [2] element offset of the chunk's rows, low and high words
+  int* s_off = s_slot + 34;   // [2] element offset of the chunk's rows, low and high words; -1: no copies
+  float* s_sel = reinterpret_cast<float*>(s_slot + 36);   // [32] per kept head: its selection score
   // [4][RED] per-warp softmax statistics and partial outputs, 16-byte aligned
-  float* s_red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_slot + 36) + 15) & ~uintptr_t(15));
+  float* s_red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_sel + 32) + 15) & ~uintptr_t(15));
+  // per head of a batch: each thread's key weight [4][128], then each warp's (max, sum) [4][4][2]
+  float* s_pk = s_red + 4 * U::RED;
+  float* s_ml = s_pk + 4 * 128;
   pdl_wait();      // the top-K lists
   pdl_trigger();
   const int bh = blockIdx.y, b = bh / Hkv, h = bh % Hkv;
@@ -475,44 +485,65 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
   const int PS = K + wm1 + 1;    // partial slots per row
   // candidate slot g * K + k, or G * K + w for window chunk own - w
   const int pidx = blockIdx.x;
+  const bool window = pidx >= G * K;
   const int64_t own = decode_own_chunk(seqlens, b, cap);
-  if (own < 0 || (pidx >= G * K && own < pidx - G * K)) {
-    if (tid == 0 && pidx < G * K) part_u[(row0 + pidx / K) * PS + pidx % K] = -INFINITY;
-    if (tid < G && pidx >= G * K) part_u[(row0 + tid) * PS + K + (pidx - G * K)] = -INFINITY;
+  if (own < 0 || (window && own < pidx - G * K)) {
+    if (tid == 0 && !window) part_u[(row0 + pidx / K) * PS + pidx % K] = -INFINITY;
+    if (tid < G && window) part_u[(row0 + tid) * PS + K + (pidx - G * K)] = -INFINITY;
     return;
   }
   const int64_t n_cand = own - wm1 > 0 ? own - wm1 : 0;
+  int64_t j0, j1;
   if (tid == 0) {
-    // send the chunk's key and value rows toward L2 now, while the slot
-    // bookkeeping below runs (a chunk another head's CTA takes is on its way
-    // for that CTA too); nothing is prefetched for an invalid chunk or page
+    // the chunk and where its rows live (contiguous cache or chunk page; a
+    // page outside the pool is recorded); the copies start right after the
+    // barrier below, before the slot bookkeeping, and are drained if the
+    // chunk turns out to belong to an earlier head
     int64_t c = -1;
-    if (pidx >= G * K) {
+    if (window) {
       c = own - (pidx - G * K);
     } else {
       const int32_t ci = sel_ids[row0 * K + pidx];
       if (ci >= 0 && ci < n_cand) c = ci;
     }
-    int64_t off = -1;
-    if (c >= 0 && pk.table == nullptr) {
-      off = ((int64_t(b) * Hkv + h) * cap + c * kChunk) * D;
-    } else if (c >= 0) {
-      const int64_t page = __ldg(pk.table + int64_t(b) * (cap / kChunk) + c);
-      if (page >= 0 && page < pk.n_pages) off = (page * Hkv + h) * kChunk * D;
-    }
+    const int64_t off = c >= 0 ? kv_chunk_offset(pk, b, h, c, Hkv, cap, cap / kChunk, D) : -1;
     if (off >= 0) {
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kc + off), "r"(U::TILE) : "memory");
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vc + off), "r"(U::TILE) : "memory");
     }
+    s_off[0] = int(uint32_t(uint64_t(off)));
+    s_off[1] = int(uint32_t(uint64_t(off) >> 32));
   }
-  for (int idx = tid; idx < G * K; idx += 128) sid[idx] = sel_ids[row0 * K + idx];
+  if (!window)
+    for (int idx = tid; idx < G * K; idx += 128) sid[idx] = sel_ids[row0 * K + idx];
+  for (int idx = tid; idx < G * D; idx += 128) {
+    const T x = q[row0 * D + idx];
+    if constexpr (sizeof(T) == 2) sq[idx] = __bfloat162float(x);
+    else sq[idx] = x;
+  }
   __syncthreads();
-  int64_t j0, j1;
-  if (pidx >= G * K) {
+  const int64_t koff = int64_t((uint64_t(uint32_t(s_off[1])) << 32) | uint64_t(uint32_t(s_off[0])));
+  // the chunk's 64 key and value rows, all copies in flight at once (the own
+  // chunk lies inside the cache, whose capacity is a multiple of 64; keys
+  // after the query are masked below)
+  const uint8_t* kg = reinterpret_cast<const uint8_t*>(kc + (koff > 0 ? koff : 0));
+  const uint8_t* vg = reinterpret_cast<const uint8_t*>(vc + (koff > 0 ? koff : 0));
+  const uint32_t sk_a = uint32_t(__cvta_generic_to_shared(sk));
+  // the chunk's 64 key rows (blocks rotated) or value rows into the buffer,
+  // all copies in flight at once
+  auto load_rows = [&](const uint8_t* src, bool keys) {
+#pragma unroll 4
+    for (int t = tid; t < kChunk * U::NB; t += 128) {
+      const int r = t / U::NB, blk = t % U::NB;
+      cp_async16(sk_a + (keys ? uint32_t(r * U::RB + ((blk ^ (r & 7)) << 4)) : uint32_t(t) * 16), src + size_t(t) * 16);
+    }
+  };
+  if (koff >= 0) load_rows(kg, true);
+  if (window) {
     const int w = pidx - G * K;
     j0 = (own - w) * kChunk;
     j1 = w == 0 ? int64_t(__ldg(seqlens + b)) : j0 + kChunk;
-    if (tid < G) s_slot[tid] = K + w;
+    if (tid < G) s_slot[tid] = koff >= 0 ? K + w : -1;
     if (tid == 0) s_go = 1;
   } else {
     const int g = pidx / K, k = pidx % K;
@@ -534,135 +565,151 @@ decode_partial_union_kernel(const T* __restrict__ q, const T* __restrict__ kc, c
         }
       }
       const uint32_t mask = __ballot_sync(0xffffffffu, my_slot >= 0);
+      // an earlier head's CTA takes a chunk that head also kept
+      const bool go = !bad && !(mask & ((1u << g) - 1u));
+      if (go && my_slot >= 0) {
+        s_sel[lane] = sel_scores[(row0 + lane) * K + my_slot];
+        // a page outside the pool: the chunk counts as not kept
+        if (koff < 0) part_u[(row0 + lane) * PS + my_slot] = -INFINITY;
+      }
       if (lane < G) s_slot[lane] = my_slot;
       if (lane == 0) {
         if (bad) {
           part_u[(row0 + g) * PS + k] = -INFINITY;
           if (c >= n_cand) record_error(HILS_ERR_DEVICE_BOUNDS);
         }
-        // an earlier head's CTA takes a chunk that head also kept
-        s_go = !bad && !(mask & ((1u << g) - 1u));
+        s_go = go;
       }
     }
   }
   __syncthreads();
-  if (!s_go) return;
-  // where the chunk's rows live (contiguous cache or chunk page); a page
-  // outside the pool is recorded and the chunk counts as not kept
-  if (tid == 0) {
-    const int64_t off = kv_chunk_offset(pk, b, h, j0 / kChunk, Hkv, cap, cap / kChunk, D);
-    s_off[0] = int(uint32_t(uint64_t(off)));
-    s_off[1] = int(uint32_t(uint64_t(off) >> 32));
-    if (off < 0) {
-      for (int g = 0; g < G; ++g)
-        if (s_slot[g] >= 0) part_u[(row0 + g) * PS + s_slot[g]] = -INFINITY;
-    }
-  }
-  __syncthreads();
-  const int64_t koff = int64_t((uint64_t(uint32_t(s_off[1])) << 32) | uint64_t(uint32_t(s_off[0])));
-  if (koff < 0) return;
-  // the chunk's 64 key and value rows, all copies in flight at once (the own
-  // chunk lies inside the cache, whose capacity is a multiple of 64; keys
-  // after the query are masked below)
-  const uint8_t* kg = reinterpret_cast<const uint8_t*>(kc + koff);
-  const uint8_t* vg = reinterpret_cast<const uint8_t*>(vc + koff);
-  const uint32_t sk_a = uint32_t(__cvta_generic_to_shared(sk)), sv_a = uint32_t(__cvta_generic_to_shared(sv));
-#pragma unroll 4
-  for (int t = tid; t < kChunk * U::NB; t += 128) {
-    const int r = t / U::NB, blk = t % U::NB;
-    cp_async16(sk_a + uint32_t(r * U::RB + ((blk ^ (r & 7)) << 4)), kg + size_t(t) * 16);
-    cp_async16(sv_a + uint32_t(t) * 16, vg + size_t(t) * 16);
-  }
-  for (int idx = tid; idx < G * D; idx += 128) {
-    const T x = q[row0 * D + idx];
-    if constexpr (sizeof(T) == 2) sq[idx] = __bfloat162float(x);
-    else sq[idx] = x;
-  }
+  if (window && koff < 0 && tid < G) part_u[(row0 + tid) * PS + K + (pidx - G * K)] = -INFINITY;
+  // a skipped chunk's copies (if any) land before the CTA's shared memory is released
   cp_async_wait_all();
+  if (!s_go || koff < 0) return;
   __syncthreads();
-  // The heads that kept the chunk are taken one at a time by all four warps:
-  // warp w scores and weighs the chunk's keys 16w .. 16w+15 (lanes l and
-  // l+16 share key 16w + l%16, each summing half of the dimensions), keeps its
-  // keys' maximum and sum, and accumulates their weighted values; the four
-  // partial results are then merged through shared memory.  (Most chunks are
-  // kept by one head of the kv head, so spreading a head's keys over the
-  // warps, rather than one head per warp, keeps all four warps busy.)
+  // The heads that kept the chunk are taken in batches of up to four.  The
+  // buffer first holds the keys: all four warps score the batch's heads,
+  // warp w the keys 16w .. 16w+15 (lanes l and l+16 share key 16w + l%16,
+  // each summing half of the dimensions), and keep each head's weights, key
+  // maximum and sum.  Then the values replace the keys (they are in L2 by
+  // now), each warp accumulates its keys' weighted values per head, and the
+  // four warps' partial results merge through shared memory.  A chunk is
+  // kept by one head of the kv head in most cases: one batch, each row read
+  // once; a later batch reads the keys again.
   const int key = warp * 16 + (lane & 15), half = lane >> 4;
   const bool vk = j0 + key < j1;
   float* my_red = s_red + warp * U::RED;
-  for (int g = 0; g < G; ++g) {
-    const int slot = s_slot[g];
-    if (slot < 0) continue;   // the same for the whole CTA
-    const float* qg = sq + g * D;
-    float sd = 0.f;
-#pragma unroll
-    for (int bb = 0; bb < U::NB / 2; ++bb) {
-      const int blk = half * (U::NB / 2) + bb;
-      float x[EB];
-      lds16<T>(sk_a + uint32_t(key * U::RB + ((blk ^ (key & 7)) << 4)), x);
-#pragma unroll
-      for (int e = 0; e < EB; ++e) sd = fmaf(qg[blk * EB + e], x[e], sd);
+  int next = 0;            // the next head to look at
+  bool keys_in = true;     // the buffer holds the keys
+  while (true) {
+    uint32_t hb = 0;       // the batch, a head per byte (the same for the whole CTA)
+    int nb = 0;
+    while (next < G && nb < 4) {
+      if (s_slot[next] >= 0) hb |= uint32_t(next) << (8 * nb++);
+      ++next;
     }
-    sd += __shfl_xor_sync(0xffffffffu, sd, 16);
-    const float z = vk ? sd * tau : -INFINITY;
-    float m = z;
+    if (nb == 0) break;
+    if (!keys_in) {
+      load_rows(kg, true);
+      cp_async_wait_all();
+      __syncthreads();
+    }
+#pragma unroll 1
+    for (int i = 0; i < nb; ++i) {
+      const float* qg = sq + int((hb >> (8 * i)) & 255u) * D;
+      float sd = 0.f;
 #pragma unroll
-    for (int off = 8; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float pk = (vk && m > -INFINITY) ? expf(z - m) : 0.f;
-    float l = pk;
+      for (int bb = 0; bb < U::NB / 2; ++bb) {
+        const int blk = half * (U::NB / 2) + bb;
+        float x[EB];
+        lds16<T>(sk_a + uint32_t(key * U::RB + ((blk ^ (key & 7)) << 4)), x);
 #pragma unroll
-    for (int off = 8; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    // the warp's 16 keys' weighted values: lane owns dims lane * EL .. + EL - 1
-    float o[EL];
+        for (int e = 0; e < EB; ++e) sd = fmaf(qg[blk * EB + e], x[e], sd);
+      }
+      sd += __shfl_xor_sync(0xffffffffu, sd, 16);
+      const float z = vk ? sd * tau : -INFINITY;
+      float m = z;
 #pragma unroll
-    for (int e = 0; e < EL; ++e) o[e] = 0.f;
+      for (int off = 8; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float p = (vk && m > -INFINITY) ? expf(z - m) : 0.f;
+      float l = p;
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const T* vrow = reinterpret_cast<const T*>(sv + (warp * 16 + jj) * U::RB) + lane * EL;
-      const float pj = __shfl_sync(0xffffffffu, pk, jj);
-#pragma unroll
-      for (int e = 0; e < EL; ++e) {
-        float xv;
-        if constexpr (sizeof(T) == 2) xv = __bfloat162float(vrow[e]);
-        else xv = vrow[e];
-        o[e] = fmaf(pj, xv, o[e]);
+      for (int off = 8; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      s_pk[i * 128 + tid] = p;
+      if (lane == 0) {
+        s_ml[(i * 4 + warp) * 2] = m;
+        s_ml[(i * 4 + warp) * 2 + 1] = l;
       }
     }
-#pragma unroll
-    for (int e = 0; e < EL; ++e) my_red[lane * EL + e] = o[e];
-    if (lane == 0) {
-      my_red[D] = m;
-      my_red[D + 1] = l;
-    }
+    __syncthreads();   // every warp is done with the keys
+    load_rows(vg, false);
+    cp_async_wait_all();
     __syncthreads();
-    // merge the four warps: M = max m_w, L = sum l_w e^(m_w - M), O = sum o_w e^(m_w - M) / L
-    float mw[4], M = -INFINITY;
+    keys_in = false;
+#pragma unroll 1
+    for (int i = 0; i < nb; ++i) {
+      const int g = int((hb >> (8 * i)) & 255u), slot = s_slot[g];
+      // the warp's 16 keys' weighted values: lane owns dims lane * EL .. + EL - 1
+      float o[EL];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      mw[w] = s_red[w * U::RED + D];
-      M = fmaxf(M, mw[w]);
-    }
-    float L = 0.f, f[4];
+      for (int e = 0; e < EL; ++e) o[e] = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      f[w] = mw[w] > -INFINITY ? expf(mw[w] - M) : 0.f;
-      L = fmaf(s_red[w * U::RED + D + 1], f[w], L);
-    }
-    const int64_t row = row0 + g;
-    if (tid < D) {
-      float acc = 0.f;
+      for (int jj = 0; jj < 16; ++jj) {
+        const T* vrow = reinterpret_cast<const T*>(sk + (warp * 16 + jj) * U::RB) + lane * EL;
+        const float pj = s_pk[i * 128 + warp * 32 + jj];   // key 16w + jj, as lane jj holds it
 #pragma unroll
-      for (int w = 0; w < 4; ++w) acc = fmaf(s_red[w * U::RED + tid], f[w], acc);
-      part_o[(row * PS + slot) * D + tid] = acc / L;
+        for (int e = 0; e < EL; ++e) {
+          float xv;
+          if constexpr (sizeof(T) == 2) xv = __bfloat162float(vrow[e]);
+          else xv = vrow[e];
+          o[e] = fmaf(pj, xv, o[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EL; ++e) my_red[lane * EL + e] = o[e];
+      if (lane == 0) {
+        my_red[D] = s_ml[(i * 4 + warp) * 2];
+        my_red[D + 1] = s_ml[(i * 4 + warp) * 2 + 1];
+      }
+      __syncthreads();
+      // merge the four warps: M = max m_w, L = sum l_w e^(m_w - M), O = sum o_w e^(m_w - M) / L
+      float mw[4], M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        mw[w] = s_red[w * U::RED + D];
+        M = fmaxf(M, mw[w]);
+      }
+      float L = 0.f, f[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        f[w] = mw[w] > -INFINITY ? expf(mw[w] - M) : 0.f;
+        L = fmaf(s_red[w * U::RED + D + 1], f[w], L);
+      }
+      const int64_t row = row0 + g;
+      if (tid < D) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc = fmaf(s_red[w * U::RED + tid], f[w], acc);
+        part_o[(row * PS + slot) * D + tid] = acc / L;
+      }
+      if (tid == 0) part_u[row * PS + slot] = slot >= K ? M + logf(L) : s_sel[g];
+      __syncthreads();   // s_red is reused by the next head
     }
-    if (tid == 0) part_u[row * PS + slot] = slot >= K ? M + logf(L) : sel_scores[row * K + slot];
-    __syncthreads();   // s_red is reused by the next head
   }
 }
 
-// D4: one CTA of D threads per row, thread t owns output dim t; the slots'
-// partial rows are read 8 at a time with all loads in flight (the per-slot
-// work is one fused multiply-add, so the kernel is load-latency bound).
+// D4: one CTA of D threads per row, thread t owns output dim t.  Every
+// thread reads the row's slot scores itself (the same addresses for the
+// whole CTA, so no shared memory and no block barrier) together with its
+// dim of the slots' partial rows, kCombBlock slots per round with all
+// loads in flight, and folds each round into a running softmax (maximum,
+// sum of weights, weighted sum).  A slot with score -inf was not written
+// with a partial row: its load is made but its value is discarded by a
+// select, never multiplied.  The kernel is load-latency bound: one round
+// trip per kCombBlock slots.
+constexpr int kCombBlock = 24;
+
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
 decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict__ part_o,
@@ -670,8 +717,6 @@ decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict_
                       const int32_t* __restrict__ sel_ids, const float* __restrict__ sel_scores,
                       T* __restrict__ o, int32_t* __restrict__ ids_out, float* __restrict__ scores_out,
                       int64_t n_rows, int wm1) {
-  __shared__ float s_w[kMaxTopK + 17];   // fusion weight of each slot
-  __shared__ float s_z;
   pdl_wait();      // the partial outputs
   const int t = threadIdx.x;
   const int64_t row = blockIdx.x;
@@ -679,36 +724,33 @@ decode_combine_kernel(const float* __restrict__ part_u, const float* __restrict_
   const bool valid = decode_own_chunk(seqlens, b, cap) >= 0;
   const int PS = K + wm1 + 1;
   const float* pu = part_u + row * PS;
-  if (t < 32) {
-    float M = -INFINITY;
-    for (int s = t; s < PS; s += 32) M = fmaxf(M, pu[s]);
-#pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float Z = 0.f;
-    for (int s = t; s < PS; s += 32) {
-      const float u = pu[s];
-      const float w = (valid && u != -INFINITY) ? expf(u - M) : 0.f;
-      s_w[s] = w;
-      Z += w;
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
-    if (t == 0) s_z = Z;
-  }
-  __syncthreads();
   const float* po = part_o + row * PS * D + t;
-  float acc = 0.f;
-  int s = 0;
-  for (; s + 8 <= PS; s += 8) {
-    float x[8];
+  float M = -INFINITY, Z = 0.f, acc = 0.f;
+  for (int s0 = 0; s0 < PS; s0 += kCombBlock) {
+    float u[kCombBlock], x[kCombBlock];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = s_w[s + e] != 0.f ? po[int64_t(s + e) * D] : 0.f;
+    for (int e = 0; e < kCombBlock; ++e) {
+      const bool in = s0 + e < PS;
+      u[e] = in ? __ldg(pu + s0 + e) : -INFINITY;
+      x[e] = in ? po[int64_t(s0 + e) * D] : 0.f;
+    }
+    float m = M;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc = fmaf(s_w[s + e], x[e], acc);
+    for (int e = 0; e < kCombBlock; ++e) m = fmaxf(m, u[e]);
+    if (!valid || m == -INFINITY) continue;
+    // rescale what the earlier rounds summed to the new maximum
+    const float r = M == -INFINITY ? 0.f : expf(M - m);
+    Z *= r;
+    acc *= r;
+#pragma unroll
+    for (int e = 0; e < kCombBlock; ++e) {
+      const bool live = u[e] != -INFINITY;
+      const float w = live ? expf(u[e] - m) : 0.f;
+      Z += w;
+      acc = fmaf(w, live ? x[e] : 0.f, acc);
+    }
+    M = m;
   }
-  for (; s < PS; ++s)
-    if (s_w[s] != 0.f) acc = fmaf(s_w[s], po[int64_t(s) * D], acc);
-  const float Z = s_z;
   const float y = Z > 0.f ? acc / Z : 0.f;
   if constexpr (sizeof(T) == 2) o[row * D + t] = __float2bfloat16_rn(y);
   else o[row * D + t] = y;

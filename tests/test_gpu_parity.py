@@ -141,6 +141,27 @@ def test_decode_ragged_seqlens(dtype):
     run_decode_check(w, inp, q, k, v, summ, seqlens, oracle, kp, bp, inp.q_f32)
 
 
+DECODE_GROUPS = [
+    # query heads per kv head beyond one group of eight (the bf16 partial
+    # kernel takes eight heads per tensor-core tile), an odd group, d 128
+    custom("decode-g12-d128", B=2, Hq=12, Hkv=1, d=128, N=4096, K=8, seed=42, dtype="bf16", kind="decode"),
+    custom("decode-g3-d64", B=3, Hq=6, Hkv=2, d=64, N=4096, K=16, seed=43, dtype="bf16", kind="decode"),
+    custom("decode-g32-d64", B=1, Hq=32, Hkv=1, d=64, N=2048, K=4, seed=44, dtype="bf16", kind="decode"),
+]
+
+
+@pytest.mark.parametrize("w", DECODE_GROUPS, ids=[w.name for w in DECODE_GROUPS])
+def test_decode_head_groups(w):
+    inp = generate(w)
+    q, k, v, lq = (to_dev(inp, n) for n in ("q", "k", "v", "lq"))
+    summ = hils.landmark_summary(k, lq, w.K)
+    oracle = Oracle.for_workload(w)
+    kp, bp = oracle.summary(inp.k_f32, inp.lq_f32)
+    # a full cache, a ragged one and one whose own chunk holds a single key
+    seqlens = np.array([w.N, w.N - 29, 64 * 7 + 1][:w.B], np.int32)
+    run_decode_check(w, inp, q, k, v, summ, seqlens, oracle, kp, bp, inp.q_f32)
+
+
 def test_prefill_and_decode_512k():
     """512K workload: sampled-row prefill parity, then the decode step at full
     length, which must agree with prefill row N-1."""
