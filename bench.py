@@ -736,15 +736,23 @@ def run_backward(args, w, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     max_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
     ach = flops / (ms_step / 1e3) / 1e12
-    # every backward kernel runs on CUDA cores in fp32 (bf16 inputs are widened)
-    bound = "alu"
-    peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
-    psrc = f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {max_mhz:.0f} MHz"
+    if w.dtype == "bf16":
+        # bf16: the selected chunks' products (most of the flops) run on the
+        # tensor cores, the window branch and the summaries on CUDA cores
+        peaks = load_peaks()
+        bound = "tensor"
+        peak = peaks["bf16_tflops"]
+        psrc = f"{peaks['source']} bf16 dense burst"
+    else:
+        # fp32: every backward kernel runs on CUDA cores
+        bound = "alu"
+        peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+        psrc = f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {max_mhz:.0f} MHz"
     line = {
         "metric": "HiLS backward tokens/s (gradients of q, k, v, lq for a fixed selection)",
         "value": job_throughput(world, B * N, ms_step), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 (bf16 inputs)" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16 (fp32 sums)" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": workload_config(w, world),
         "roofline": {"kernel": "backward (whole call)", "bound": bound, "achieved": ach, "peak": peak,
                      "unit": "TFLOP/s", "frac": ach / peak, "traffic": None, "peak_source": psrc},

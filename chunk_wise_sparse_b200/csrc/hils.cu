@@ -19,6 +19,7 @@
 #include "qcal.cuh"
 #include "backward.cuh"
 #include "backward_tc.cuh"
+#include "backward_mma.cuh"
 
 using namespace hils;
 
@@ -471,6 +472,16 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
     if (set_smem_max<tfn>() != cudaSuccess) return HILS_ERR_CUDA;
     tfn<<<unsigned(sm_count() * (D == 64 ? 2 : 1)), CT::THREADS, CT::SMEM, st>>>(
         mq, mg, mk, mv, kprime, dvec, tiles, items, e_pair, P.c, dq, dk, dv, dkp, dbp);
+  } else if (std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
+    // bf16 with the attention query as the scoring query: the selected
+    // chunks' five products on tensor cores (mma.sync)
+    using MT = BwdMma<D>;
+    constexpr auto mfn = bwd_chunk_mma_kernel<D>;
+    if (set_smem_max<mfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    mfn<<<unsigned(sm_count() * MT::CTAS_PER_SM), MT::THREADS, MT::SMEM, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(d_o), kprime, dvec, tiles, items,
+        e_pair, P.c, dq, dk, dv, dkp, dbp);
   } else {
     const size_t smem_c = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(2 * D + 4) * 4;
     constexpr auto cfn2 = bwd_chunk_kernel<T, D>;

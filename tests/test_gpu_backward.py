@@ -89,6 +89,8 @@ CASES = [
     custom("bwd-bf16-d64-g4", B=1, Hq=8, Hkv=2, d=64, N=1024, K=8, seed=203, dtype="bf16"),
     custom("bwd-bf16-d128-w256", B=1, Hq=2, Hkv=1, d=128, N=640, K=5, seed=204, dtype="bf16", window=256),
     custom("bwd-fp32-d64-g3", B=1, Hq=6, Hkv=2, d=64, N=384, K=2, seed=205, dtype="fp32"),
+    # bf16 without a window, d 128, two batch elements: full and ragged tiles of the tensor-core kernel
+    custom("bwd-bf16-d128-g2", B=2, Hq=4, Hkv=2, d=128, N=1024, K=6, seed=209, dtype="bf16"),
 ]
 
 
