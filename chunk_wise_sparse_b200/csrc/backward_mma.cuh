@@ -337,4 +337,176 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   }
 }
 
+// The window branch on tensor cores: one CTA per (chunk o of positions,
+// (b, hq)), the 64 rows at positions 64 o .. 64 o + 63 against the key
+// chunks o - wm1 .. o (the last under the causal mask), with weights
+// P = exp(tau s - M'):
+//   dz_j = tau P_j (<g, v_j> - Dg),  dq = sum_j dz_j k_j (written: this
+//   kernel runs first), dk_j += sum_i dz_j q_i, dv_j += sum_i P_j g_i.
+// Warps 0-3 take 16 rows each for S, G, the weights and dQ (kept in
+// registers across the window's chunks); all eight warps take dK or dV of
+// 16 keys of each chunk, as in bwd_chunk_mma_kernel.
+template <int D>
+struct BwdWinMma {
+  static constexpr int RB = D * 2;
+  static constexpr int NB = RB / 16;
+  static constexpr int THREADS = 256;
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = OFF_K + kChunk * RB;
+  static constexpr uint32_t OFF_Q = OFF_V + kChunk * RB;
+  static constexpr uint32_t OFF_G = OFF_Q + kChunk * RB;
+  static constexpr uint32_t OFF_DZ = OFF_G + kChunk * RB;   // [64][64] bf16
+  static constexpr uint32_t OFF_PW = OFF_DZ + kChunk * 128;
+  static constexpr uint32_t SMEM = OFF_PW + kChunk * 128;
+  static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
+};
+
+template <int D>
+__global__ void __launch_bounds__(BwdWinMma<D>::THREADS, BwdWinMma<D>::CTAS_PER_SM)
+bwd_window_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                      const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ d_o,
+                      const float* __restrict__ rowstat, const float* __restrict__ dvec, int64_t n_tok, int Hq,
+                      int G, int Hkv, int wm1, float tau, float* __restrict__ dq, float* __restrict__ dk,
+                      float* __restrict__ dv) {
+  using C = BwdWinMma<D>;
+  extern __shared__ __align__(16) uint8_t bsm[];
+  const uint32_t sbase = uint32_t(__cvta_generic_to_shared(bsm));
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sQ = sbase + C::OFF_Q, sG = sbase + C::OFF_G;
+  const uint32_t sDZ = sbase + C::OFF_DZ, sPW = sbase + C::OFF_PW;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int mi = lane >> 3, ri = lane & 7;
+  const int64_t own = blockIdx.x;
+  const int bhq = int(blockIdx.y), b = bhq / Hq, hq = bhq % Hq, h = hq / G;
+  const int64_t p0 = own * kChunk;
+  const int64_t row0 = int64_t(bhq) * n_tok + p0;
+  const int64_t kv0 = (int64_t(b) * Hkv + h) * n_tok;
+  // the 64 rows' queries and output gradients (contiguous rows)
+  for (int u = tid; u < 2 * kChunk * C::NB; u += C::THREADS) {
+    const int which = u / (kChunk * C::NB), rem = u % (kChunk * C::NB);
+    const int r = rem / C::NB, blk = rem % C::NB;
+    bm_cp16((which ? sG : sQ) + bm_at(r, blk, C::RB), (which ? d_o : q) + (row0 + r) * D + blk * 8);
+  }
+  const int rb = warp * 16;
+  const int r0 = rb + gq, r1 = rb + gq + 8;   // this lane's rows (warps 0-3)
+  float mp0 = 0.f, mp1 = 0.f, dg0 = 0.f, dg1 = 0.f;
+  if (warp < 4) {
+    mp0 = rowstat[row0 + r0];
+    mp1 = rowstat[row0 + r1];
+    dg0 = dvec[row0 + r0];
+    dg1 = dvec[row0 + r1];
+  }
+  float qacc[D / 8][4];
+#pragma unroll
+  for (int nd = 0; nd < D / 8; ++nd) qacc[nd][0] = qacc[nd][1] = qacc[nd][2] = qacc[nd][3] = 0.f;
+  const int64_t c_lo = own - wm1 > 0 ? own - wm1 : 0;
+  for (int64_t cj = c_lo; cj <= own; ++cj) {
+    __syncthreads();   // the previous chunk's K, V, dZ, aP are no longer read
+    for (int u = tid; u < 2 * kChunk * C::NB; u += C::THREADS) {
+      const int which = u / (kChunk * C::NB), rem = u % (kChunk * C::NB);
+      const int r = rem / C::NB, blk = rem % C::NB;
+      bm_cp16((which ? sV : sK) + bm_at(r, blk, C::RB), (which ? v : k) + (kv0 + cj * kChunk + r) * D + blk * 8);
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (warp < 4) {
+      float sacc[8][4], gacc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = gacc[nt][e] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t aq[4], ag[4];
+        const int ar = rb + ri + ((mi & 1) << 3), ablk = 2 * kk + (mi >> 1);
+        bm_ldsm4(sQ + bm_at(ar, ablk, C::RB), aq);
+        bm_ldsm4(sG + bm_at(ar, ablk, C::RB), ag);
+#pragma unroll
+        for (int nt = 0; nt < 8; nt += 2) {
+          uint32_t bk[4], bv[4];
+          const int key = 8 * nt + ri + ((mi >> 1) << 3), bblk = 2 * kk + (mi & 1);
+          bm_ldsm4(sK + bm_at(key, bblk, C::RB), bk);
+          bm_ldsm4(sV + bm_at(key, bblk, C::RB), bv);
+          bm_mma(sacc[nt], aq, bk[0], bk[1]);
+          bm_mma(sacc[nt + 1], aq, bk[2], bk[3]);
+          bm_mma(gacc[nt], ag, bv[0], bv[1]);
+          bm_mma(gacc[nt + 1], ag, bv[2], bv[3]);
+        }
+      }
+      // P (causal in the own chunk), dZ into sacc, P into gacc; both to shared memory
+      const int64_t kbase = cj * kChunk;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t key = kbase + 8 * nt + 2 * tq + (e & 1);
+          const int64_t pos = p0 + (e < 2 ? r0 : r1);
+          const float mp = e < 2 ? mp0 : mp1, dg = e < 2 ? dg0 : dg1;
+          const float P = key <= pos ? expf(tau * sacc[nt][e] - mp) : 0.f;
+          sacc[nt][e] = tau * P * (gacc[nt][e] - dg);
+          gacc[nt][e] = P;
+        }
+        const uint32_t o0 = bm_at(r0, nt, 128) + 4 * tq, o1 = bm_at(r1, nt, 128) + 4 * tq;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sDZ + o0), "r"(bm_pack(sacc[nt][0], sacc[nt][1])) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sDZ + o1), "r"(bm_pack(sacc[nt][2], sacc[nt][3])) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sPW + o0), "r"(bm_pack(gacc[nt][0], gacc[nt][1])) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sPW + o1), "r"(bm_pack(gacc[nt][2], gacc[nt][3])) : "memory");
+      }
+      // dQ += dZ K
+#pragma unroll
+      for (int nd = 0; nd < D / 8; nd += 2) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a[4] = {bm_pack(sacc[2 * kk][0], sacc[2 * kk][1]), bm_pack(sacc[2 * kk][2], sacc[2 * kk][3]),
+                                 bm_pack(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]),
+                                 bm_pack(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3])};
+          uint32_t bq[4];
+          const int key = 16 * kk + ri + ((mi & 1) << 3), bblk = nd + (mi >> 1);
+          bm_ldsm4_t(sK + bm_at(key, bblk, C::RB), bq);
+          bm_mma(qacc[nd], a, bq[0], bq[1]);
+          bm_mma(qacc[nd + 1], a, bq[2], bq[3]);
+        }
+      }
+    }
+    __syncthreads();
+    // dK = dZ^T Q (warps 0-3), dV = P^T dO (warps 4-7) for this chunk's keys 16 (w % 4) .. +15
+    {
+      const uint32_t sA = warp < 4 ? sDZ : sPW, sB = warp < 4 ? sQ : sG;
+      float* gout = warp < 4 ? dk : dv;
+      const int mt = warp & 3;
+      float acc[D / 8][4];
+#pragma unroll
+      for (int nd = 0; nd < D / 8; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < kChunk / 16; ++kk) {
+        uint32_t a[4];
+        const int ar = 16 * kk + ri + ((mi >> 1) << 3), ablk = 2 * mt + (mi & 1);
+        bm_ldsm4_t(sA + bm_at(ar, ablk, 128), a);
+#pragma unroll
+        for (int nd = 0; nd < D / 8; nd += 2) {
+          uint32_t bb[4];
+          const int br = 16 * kk + ri + ((mi & 1) << 3), bblk = nd + (mi >> 1);
+          bm_ldsm4_t(sB + bm_at(br, bblk, C::RB), bb);
+          bm_mma(acc[nd], a, bb[0], bb[1]);
+          bm_mma(acc[nd + 1], a, bb[2], bb[3]);
+        }
+      }
+      const int64_t k0 = kv0 + cj * kChunk + 16 * mt + gq;
+#pragma unroll
+      for (int nd = 0; nd < D / 8; ++nd)
+        bm_red4(gout + k0 * D, gout + (k0 + 8) * D, 8 * nd + 2 * tq, tq, acc[nd][0], acc[nd][1], acc[nd][2],
+                acc[nd][3], true, true);
+    }
+  }
+  // the window kernel runs first: dq is written here, the selected chunks add to it
+  if (warp < 4) {
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+      const int t0 = 8 * nd + 2 * tq;
+      *reinterpret_cast<float2*>(dq + (row0 + r0) * D + t0) = make_float2(qacc[nd][0], qacc[nd][1]);
+      *reinterpret_cast<float2*>(dq + (row0 + r1) * D + t0) = make_float2(qacc[nd][2], qacc[nd][3]);
+    }
+  }
+}
+
 }  // namespace hils

@@ -450,11 +450,22 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
     cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
                                                                        P.c, P.n_slots);
   const float tau = 1.f / sqrtf(float(D));
-  const size_t smem_w = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(BT::SUB) * D * 4;
-  constexpr auto wfn = bwd_window_kernel<T, D>;
-  if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
-  wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
-      tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
+  if (std::is_same<T, __nv_bfloat16>::value) {
+    // bf16: the window branch's products on tensor cores
+    using WT = BwdWinMma<D>;
+    constexpr auto wfn = bwd_window_mma_kernel<D>;
+    if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), WT::THREADS, WT::SMEM, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(d_o), rowstat, dvec, N,
+        d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
+  } else {
+    const size_t smem_w = BT::KV_BYTES + BT::ROW_BYTES + BT::P_BYTES + size_t(BT::SUB) * D * 4;
+    constexpr auto wfn = bwd_window_kernel<T, D>;
+    if (set_smem_max<wfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
+        tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
+  }
   // The tensor-core kernel (bwd_chunk_tc_kernel) is kept but not launched
   // until a hang seen with it is explained.
   constexpr bool kUseTensorCoreBackward = false;

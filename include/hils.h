@@ -350,9 +350,10 @@ size_t hils_attn_backward_workspace_bytes(const hils_dims* dims);
  *                the chunk scores when dq_score is NULL
  *   dq_score     [B,Hq,N,d] fp32 out (nullable): the scoring query's gradient
  *   dk, dv       [B,Hkv,N,d] fp32 out;  dlq [B,Hkv,nc,d] fp32 out
- * Outputs are overwritten.  fp32 arithmetic on CUDA cores, except for bf16
- * with q_score == NULL: there the selected chunks' products run on tensor
- * cores with bf16 operands (dZ and a p rounded to bf16) and fp32 sums.
+ * Outputs are overwritten.  fp32 arithmetic on CUDA cores, except for bf16:
+ * there the window branch's products, and with q_score == NULL also the
+ * selected chunks', run on tensor cores with bf16 operands (dZ and the
+ * weights rounded to bf16) and fp32 sums.
  * Gradients are summed with fp32 atomics (the order of the sums is not
  * fixed).  Any G;
  * B * Hq <= 65535.  Ids outside a row's candidates are recorded as
