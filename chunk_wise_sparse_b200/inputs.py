@@ -94,6 +94,10 @@ WORKLOADS = {
                                               "bf16", 0, "none", "decode", 0, window=512),
     "prefill-128k-gqa4-d128": Workload("prefill-128k-gqa4-d128", 1, 32, 8, 128, 131072, 64, 32, 3,
                                        "bf16", 64, "random", "prefill", 4096),
+    # the 128K GQA workload's shape at 32K tokens: a profiling case for the d = 128 kernels that keeps the
+    # device footprint near 1.5 GB while Q (268 MB) still exceeds L2
+    "prefill-32k-gqa4-d128": Workload("prefill-32k-gqa4-d128", 1, 32, 8, 128, 32768, 64, 32, 3,
+                                      "bf16", 16, "random", "prefill", 4096),
     "prefill-512k-h16-d64": Workload("prefill-512k-h16-d64", 1, 16, 16, 64, 524288, 64, 16, 4,
                                      "bf16", 128, "random", "prefill+decode", 4096),
     # the 512K workload with rank-16 Q-Cal: chunk scores from q^ = q + W_up W_down q
