@@ -91,6 +91,9 @@ CASES = [
     custom("bwd-fp32-d64-g3", B=1, Hq=6, Hkv=2, d=64, N=384, K=2, seed=205, dtype="fp32"),
     # bf16 without a window, d 128, two batch elements: full and ragged tiles of the tensor-core kernel
     custom("bwd-bf16-d128-g2", B=2, Hq=4, Hkv=2, d=128, N=1024, K=6, seed=209, dtype="bf16"),
+    # one query head per kv head with a window (tiles of every pair count), and eight heads per kv head
+    custom("bwd-bf16-d64-g1-w128", B=2, Hq=2, Hkv=2, d=64, N=768, K=3, seed=210, dtype="bf16", window=128),
+    custom("bwd-bf16-d128-g8", B=1, Hq=8, Hkv=1, d=128, N=512, K=4, seed=211, dtype="bf16"),
 ]
 
 
