@@ -19,7 +19,8 @@
 //                               summed over the tile's rows)
 // dZ and aP enter the MMAs rounded to bf16 (the inputs are bf16); every sum
 // is fp32.  Rows of a tile are gathered into shared memory by 16-byte
-// cp.async copies; every row-major bf16 tile keeps its 16-byte blocks of row r
+// cp.async copies (the next tile's keys, values and row list while the
+// current tile's dK, dV products run); every row-major bf16 tile keeps its 16-byte blocks of row r
 // at block ^ (r mod 8), so that the eight rows an ldmatrix reads hit
 // distinct banks.  No TMEM and no mbarrier: the only waits are block
 // barriers that every thread reaches.
@@ -83,7 +84,8 @@ struct BwdMma {
   static constexpr uint32_t OFF_DU = OFF_PW + M * 128;     // [M] fp32
   static constexpr uint32_t OFF_KP = OFF_DU + M * 4;       // [D] fp32, the chunk's k'
   static constexpr uint32_t OFF_DKP = OFF_KP + D * 4;      // [D] fp32: tau sum du q over the tile, then sum du
-  static constexpr uint32_t SMEM = OFF_DKP + D * 4 + 16;
+  static constexpr uint32_t OFF_ROWS = OFF_DKP + D * 4 + 16;  // [M] int32: the tile's pair rows
+  static constexpr uint32_t SMEM = OFF_ROWS + M * 4;
   static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
 };
 
@@ -109,40 +111,47 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   float* s_du = reinterpret_cast<float*>(bsm + C::OFF_DU);
   float* s_kp = reinterpret_cast<float*>(bsm + C::OFF_KP);
   float* s_dkp = reinterpret_cast<float*>(bsm + C::OFF_DKP);   // [D], then [D] the tile's sum of du
+  int32_t* s_rows = reinterpret_cast<int32_t*>(bsm + C::OFF_ROWS);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;   // fragment row group and column pair
   const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: the matrix and row this lane addresses
   const float tau = c.tau;
   const int n_all = tile_start[c.n_keys];
+  // a tile's keys, values and k' and its pair rows, staged ahead: the first
+  // tile's before the loop, the next tile's while the current one's dK, dV
+  // products run (they read neither K, V, k' nor the row list)
+  auto stage = [&](int t) {
+    const int4 st = items[t];
+    const int64_t kvr = st.y;
+    for (int u = tid; u < 2 * kChunk * C::NB; u += C::THREADS) {
+      const int which = u / (kChunk * C::NB), rem = u % (kChunk * C::NB);
+      const int r = rem / C::NB, blk = rem % C::NB;
+      bm_cp16((which ? sV : sK) + bm_at(r, blk, C::RB), (which ? v : k) + (kvr + r) * D + blk * 8);
+    }
+    for (int r = tid; r < st.z; r += C::THREADS) s_rows[r] = e_pair[st.x + r].x;
+    const int64_t sbh = kvr / c.n_tok, sch = (kvr % c.n_tok) / kChunk;
+    for (int d2 = tid; d2 < D; d2 += C::THREADS) s_kp[d2] = kprime[(sbh * c.nc + sch) * D + d2];
+  };
+  if (int(blockIdx.x) < n_all) stage(blockIdx.x);
   for (int tile = blockIdx.x; tile < n_all; tile += gridDim.x) {
     const int4 it = items[tile];   // first entry, K/V row, pair count
     const int64_t first = it.x, kvrow = it.y;
     const int n = it.z;
     const int64_t bh = kvrow / c.n_tok, chunk = (kvrow % c.n_tok) / kChunk;
     const int n16 = (n + 15) & ~15;   // rows the products read (the rest of the last 16 zeroed)
-    __syncthreads();   // the previous tile's shared memory is no longer read
-    // ---- the chunk's keys and values, the pairs' query and output-gradient rows
-    for (int u = tid; u < 2 * kChunk * C::NB; u += C::THREADS) {
-      const int which = u / (kChunk * C::NB), rem = u % (kChunk * C::NB);
-      const int r = rem / C::NB, blk = rem % C::NB;
-      const __nv_bfloat16* src = (which ? v : k) + (kvrow + r) * D + blk * 8;
-      bm_cp16((which ? sV : sK) + bm_at(r, blk, C::RB), src);
-    }
+    __syncthreads();   // the previous tile's shared memory is no longer read; this tile's rows are staged
+    // ---- the pairs' query and output-gradient rows (the keys and values are on their way)
     for (int u = tid; u < 2 * n16 * C::NB; u += C::THREADS) {
       const int which = u / (n16 * C::NB), rem = u % (n16 * C::NB);
       const int r = rem / C::NB, blk = rem % C::NB;
       const uint32_t dst = (which ? sG : sQ) + bm_at(r, blk, C::RB);
       if (r < n) {
-        const int64_t row = e_pair[first + r].x;
-        bm_cp16(dst, (which ? d_o : q) + row * D + blk * 8);
+        bm_cp16(dst, (which ? d_o : q) + int64_t(s_rows[r]) * D + blk * 8);
       } else {
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
       }
     }
-    for (int t = tid; t < D; t += C::THREADS) {
-      s_kp[t] = kprime[(bh * c.nc + chunk) * D + t];
-      s_dkp[t] = 0.f;
-    }
+    for (int t = tid; t < D; t += C::THREADS) s_dkp[t] = 0.f;
     if (tid == 0) s_dkp[D] = 0.f;
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     __syncthreads();
@@ -301,6 +310,8 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
     }
     __syncthreads();
+    // the next tile's keys, values, k' and rows start while dK, dV run
+    if (tile + int(gridDim.x) < n_all) stage(tile + int(gridDim.x));
     // ---- dK = dZ^T Q (warps 0-3) and dV = (aP)^T dO (warps 4-7), keys 16 (w % 4) .. +15
     {
       const uint32_t sA = warp < 4 ? sDZ : sPW, sB = warp < 4 ? sQ : sG;
