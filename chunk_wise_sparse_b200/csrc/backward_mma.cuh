@@ -85,7 +85,13 @@ struct BwdMma {
   static constexpr uint32_t OFF_KP = OFF_DU + M * 4;       // [D] fp32, the chunk's k'
   static constexpr uint32_t OFF_DKP = OFF_KP + D * 4;      // [D] fp32: tau sum du q over the tile, then sum du
   static constexpr uint32_t OFF_ROWS = OFF_DKP + D * 4 + 16;  // [M] int32: the tile's pair rows
-  static constexpr uint32_t SMEM = OFF_ROWS + M * 4;
+  // d = 128 (one CTA per SM, shared memory to spare): a second query and
+  // output-gradient row buffer, so that the next tile's rows are gathered
+  // while the current tile's dK, dV products still read the first
+  static constexpr bool DB = D == 128;
+  static constexpr uint32_t OFF_Q2 = (OFF_ROWS + M * 4 + 127u) & ~127u;
+  static constexpr uint32_t OFF_G2 = OFF_Q2 + M * RB;
+  static constexpr uint32_t SMEM = DB ? OFF_G2 + M * RB : OFF_ROWS + M * 4;
   static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
 };
 
@@ -132,23 +138,47 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const int64_t sbh = kvr / c.n_tok, sch = (kvr % c.n_tok) / kChunk;
     for (int d2 = tid; d2 < D; d2 += C::THREADS) s_kp[d2] = kprime[(sbh * c.nc + sch) * D + d2];
   };
-  if (int(blockIdx.x) < n_all) stage(blockIdx.x);
-  for (int tile = blockIdx.x; tile < n_all; tile += gridDim.x) {
+  // DB: the pairs' query and output-gradient rows of tile t into the buffer
+  // pair (qb, gb), row ids read from the index (rows past the pairs zeroed)
+  auto gather = [&](int t, uint32_t qb, uint32_t gb) {
+    const int4 gt = items[t];
+    const int gn = gt.z, gn16 = (gn + 15) & ~15;
+    for (int u = tid; u < 2 * gn16 * C::NB; u += C::THREADS) {
+      const int which = u / (gn16 * C::NB), rem = u % (gn16 * C::NB);
+      const int r = rem / C::NB, blk = rem % C::NB;
+      const uint32_t dst = (which ? gb : qb) + bm_at(r, blk, C::RB);
+      if (r < gn) {
+        bm_cp16(dst, (which ? d_o : q) + int64_t(e_pair[gt.x + r].x) * D + blk * 8);
+      } else {
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+      }
+    }
+  };
+  const uint32_t sQ2 = sbase + C::OFF_Q2, sG2 = sbase + C::OFF_G2;
+  if (int(blockIdx.x) < n_all) {
+    stage(blockIdx.x);
+    if constexpr (C::DB) gather(blockIdx.x, sQ, sG);
+  }
+  int pb = 0;   // DB: the buffer pair of the current tile
+  for (int tile = blockIdx.x; tile < n_all; tile += gridDim.x, pb ^= 1) {
     const int4 it = items[tile];   // first entry, K/V row, pair count
     const int64_t first = it.x, kvrow = it.y;
     const int n = it.z;
     const int64_t bh = kvrow / c.n_tok, chunk = (kvrow % c.n_tok) / kChunk;
     const int n16 = (n + 15) & ~15;   // rows the products read (the rest of the last 16 zeroed)
+    const uint32_t cQ = (C::DB && pb) ? sQ2 : sQ, cG = (C::DB && pb) ? sG2 : sG;   // this tile's rows
     __syncthreads();   // the previous tile's shared memory is no longer read; this tile's rows are staged
-    // ---- the pairs' query and output-gradient rows (the keys and values are on their way)
-    for (int u = tid; u < 2 * n16 * C::NB; u += C::THREADS) {
-      const int which = u / (n16 * C::NB), rem = u % (n16 * C::NB);
-      const int r = rem / C::NB, blk = rem % C::NB;
-      const uint32_t dst = (which ? sG : sQ) + bm_at(r, blk, C::RB);
-      if (r < n) {
-        bm_cp16(dst, (which ? d_o : q) + int64_t(s_rows[r]) * D + blk * 8);
-      } else {
-        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+    if constexpr (!C::DB) {
+      // ---- the pairs' query and output-gradient rows (the keys and values are on their way)
+      for (int u = tid; u < 2 * n16 * C::NB; u += C::THREADS) {
+        const int which = u / (n16 * C::NB), rem = u % (n16 * C::NB);
+        const int r = rem / C::NB, blk = rem % C::NB;
+        const uint32_t dst = (which ? sG : sQ) + bm_at(r, blk, C::RB);
+        if (r < n) {
+          bm_cp16(dst, (which ? d_o : q) + int64_t(s_rows[r]) * D + blk * 8);
+        } else {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+        }
       }
     }
     for (int t = tid; t < D; t += C::THREADS) s_dkp[t] = 0.f;
@@ -167,8 +197,8 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t aq[4], ag[4];
         const int ar = rb + ri + ((mi & 1) << 3), ablk = 2 * kk + (mi >> 1);
-        bm_ldsm4(sQ + bm_at(ar, ablk, C::RB), aq);
-        bm_ldsm4(sG + bm_at(ar, ablk, C::RB), ag);
+        bm_ldsm4(cQ + bm_at(ar, ablk, C::RB), aq);
+        bm_ldsm4(cG + bm_at(ar, ablk, C::RB), ag);
 #pragma unroll
         for (int nt = 0; nt < 8; nt += 2) {
           // keys 8nt .. 8nt+15 as the B operand (k = dims): b0, b1 of n-tiles nt and nt+1
@@ -278,7 +308,7 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 #pragma unroll 4
           for (int r = 0; r < 16; ++r) {
             unsigned short hb;
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hb) : "r"(sQ + bm_at(rb + r, t >> 3, C::RB) + uint32_t((t & 7) * 2)));
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hb) : "r"(cQ + bm_at(rb + r, t >> 3, C::RB) + uint32_t((t & 7) * 2)));
             acc_t = fmaf(s_du[rb + r], __uint_as_float(uint32_t(hb) << 16), acc_t);
           }
           atomicAdd(s_dkp + t, tau * acc_t);
@@ -310,11 +340,15 @@ bwd_chunk_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
     }
     __syncthreads();
-    // the next tile's keys, values, k' and rows start while dK, dV run
-    if (tile + int(gridDim.x) < n_all) stage(tile + int(gridDim.x));
+    // the next tile's keys, values, k' and rows (DB: and its query and
+    // output-gradient rows, into the other buffer pair) start while dK, dV run
+    if (tile + int(gridDim.x) < n_all) {
+      stage(tile + int(gridDim.x));
+      if constexpr (C::DB) gather(tile + int(gridDim.x), pb ? sQ : sQ2, pb ? sG : sG2);
+    }
     // ---- dK = dZ^T Q (warps 0-3) and dV = (aP)^T dO (warps 4-7), keys 16 (w % 4) .. +15
     {
-      const uint32_t sA = warp < 4 ? sDZ : sPW, sB = warp < 4 ? sQ : sG;
+      const uint32_t sA = warp < 4 ? sDZ : sPW, sB = warp < 4 ? cQ : cG;
       float* gout = warp < 4 ? dk : dv;
       const int mt = warp & 3;
       float acc[D / 8][4];
