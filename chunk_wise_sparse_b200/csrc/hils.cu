@@ -18,7 +18,6 @@
 #include "prefill_local.cuh"
 #include "qcal.cuh"
 #include "backward.cuh"
-#include "backward_tc.cuh"
 #include "backward_mma.cuh"
 
 using namespace hils;
@@ -466,24 +465,7 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
     wfn<<<dim3(unsigned(P.c.nc), unsigned(d->batch * d->heads_q)), BT::THREADS, smem_w, st>>>(
         tq, tk, tv, tdo, rowstat, dvec, N, d->heads_q, G, d->heads_kv, P.c.wm1, tau, dq, dk, dv);
   }
-  // The tensor-core kernel (bwd_chunk_tc_kernel) is kept but not launched
-  // until a hang seen with it is explained.
-  constexpr bool kUseTensorCoreBackward = false;
-  if (kUseTensorCoreBackward && std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
-    // bf16 with the attention query as the scoring query: selected chunks on tensor cores
-    using CT = BwdTc<D>;
-    CUtensorMap mq, mg, mk, mv;
-    const uint64_t kv_rows = uint64_t(d->batch) * d->heads_kv * N;
-    if (!make_map_2d(&mq, q, D, uint64_t(P.rows), D * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&mg, d_o, D, uint64_t(P.rows), D * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&mk, k, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&mv, v, D, kv_rows, D * 2, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
-      return HILS_ERR_CUDA;
-    constexpr auto tfn = bwd_chunk_tc_kernel<D>;
-    if (set_smem_max<tfn>() != cudaSuccess) return HILS_ERR_CUDA;
-    tfn<<<unsigned(sm_count() * (D == 64 ? 2 : 1)), CT::THREADS, CT::SMEM, st>>>(
-        mq, mg, mk, mv, kprime, dvec, tiles, items, e_pair, P.c, dq, dk, dv, dkp, dbp);
-  } else if (std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
+  if (std::is_same<T, __nv_bfloat16>::value && q_score == nullptr && dq_score == nullptr) {
     // bf16 with the attention query as the scoring query: the selected
     // chunks' five products on tensor cores (mma.sync)
     using MT = BwdMma<D>;
