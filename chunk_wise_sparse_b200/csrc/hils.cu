@@ -191,7 +191,7 @@ struct CcPlan {
   CcDims c;
   int64_t rows, n_slots, max_items, n_scan_blocks;
   int P, own_tiles;
-  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair,
+  size_t off_oacc, off_rowstat, off_counts, off_ranks, off_cbase, off_offsets, off_tiles, off_items, off_sums, off_epair,
       off_rescore, total;
 };
 
@@ -225,6 +225,45 @@ CcDims make_cc_dims(const hils_dims* d) {
   return c;
 }
 
+// The count takes one shared-memory histogram per kCountRows rows when those
+// rows stay in one window and the chunk histogram fits; its per-(CTA, chunk)
+// bases then need a table of rows / kCountRows x nc entries.
+bool cc_two_level_count(const CcDims& c) {
+  return c.n_tok % kCountRows == 0 && (int64_t(1) << c.win_shift) % kCountRows == 0 &&
+         sizeof(int32_t) * size_t(c.nc) <= 96 * 1024;
+}
+size_t cc_cbase_entries(const CcDims& c, int64_t rows) {
+  return cc_two_level_count(c) ? size_t(rows / kCountRows) * size_t(c.nc) : 0;
+}
+
+// The chunk-centric index of a selection (counts zeroed by the caller): pair
+// counts and ranks, the scan into per-key offsets and tiles, and the fill of
+// the (row, s^ - M') records.  Five launches.
+int launch_cc_index(const CcDims& c, int64_t rows, int64_t n_slots, int64_t n_scan_blocks, const int32_t* ids,
+                    const float* scores, const float* rowstat, int32_t* counts, int32_t* ranks, int32_t* cbase,
+                    int64_t* offsets, int32_t* tiles, int4* items, int64_t* sums, int2* e_pair, cudaStream_t st) {
+  if (cc_two_level_count(c)) {
+    const size_t hist_bytes = sizeof(int32_t) * size_t(c.nc);
+    constexpr auto cfn = cc_count_kernel;
+    if (hist_bytes > 48 * 1024 && set_smem_max<cfn>() != cudaSuccess) return HILS_ERR_CUDA;
+    cfn<<<unsigned(rows / kCountRows), kCountThreads, hist_bytes, st>>>(ids, counts, ranks, cbase, c);
+  } else {
+    cbase = nullptr;
+    cc_count_direct_kernel<<<unsigned((n_slots + 255) / 256), 256, 0, st>>>(ids, counts, ranks, c, n_slots);
+  }
+  const unsigned nsb = unsigned(n_scan_blocks);
+  cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, c.n_keys, sums);
+  cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, n_scan_blocks, c.n_keys, offsets, tiles);
+  cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, c, sums, offsets, tiles, items);
+  if (c.K % 4 == 0)
+    cc_fill4_kernel<<<unsigned((n_slots / 4 + 255) / 256), 256, 0, st>>>(ids, ranks, cbase, scores, rowstat, offsets,
+                                                                          e_pair, c, n_slots / 4);
+  else
+    cc_fill_kernel<<<unsigned((n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, cbase, scores, rowstat, offsets,
+                                                                     e_pair, c, n_slots);
+  return HILS_OK;
+}
+
 CcPlan cc_plan(const hils_dims* d) {
   CcPlan P;
   const int64_t N = d->seqlen, D = d->head_dim, G = d->heads_q / d->heads_kv;
@@ -240,6 +279,7 @@ CcPlan cc_plan(const hils_dims* d) {
   P.off_rowstat = take(sizeof(float) * P.rows);
   P.off_counts = take(sizeof(int32_t) * P.c.n_keys);
   P.off_ranks = take(sizeof(int32_t) * P.n_slots);
+  P.off_cbase = take(sizeof(int32_t) * cc_cbase_entries(P.c, P.rows));
   P.off_offsets = take(sizeof(int64_t) * (P.c.n_keys + 1));
   P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
   P.max_items = P.n_slots / kCcTileRows + P.c.n_keys + 1;
@@ -276,6 +316,7 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
   float* rowstat = reinterpret_cast<float*>(base + P.off_rowstat);
   int32_t* counts = reinterpret_cast<int32_t*>(base + P.off_counts);
   int32_t* ranks = reinterpret_cast<int32_t*>(base + P.off_ranks);
+  int32_t* cbase = reinterpret_cast<int32_t*>(base + P.off_cbase);
   int64_t* offsets = reinterpret_cast<int64_t*>(base + P.off_offsets);
   int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
   int4* items = reinterpret_cast<int4*>(base + P.off_items);
@@ -326,25 +367,9 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
     if (set_smem_max<loc_fn>() != cudaSuccess) return HILS_ERR_CUDA;
     loc_fn<<<own_grid, CL::THREADS, CL::SMEM, st>>>(tq_tile, tk, tv, op);
   }
-  // two-level count when a CTA's rows stay in one window and the chunk histogram fits
-  const size_t hist_bytes = sizeof(int32_t) * size_t(P.c.nc);
-  if (d->seqlen % kCountRows == 0 && (int64_t(1) << P.c.win_shift) % kCountRows == 0 && hist_bytes <= 96 * 1024) {
-    constexpr auto cfn = cc_count_kernel;
-    if (hist_bytes > 48 * 1024 && set_smem_max<cfn>() != cudaSuccess) return HILS_ERR_CUDA;
-    cfn<<<unsigned(P.rows / kCountRows), kCountThreads, hist_bytes, st>>>(ids, counts, ranks, P.c);
-  } else {
-    cc_count_direct_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, counts, ranks, P.c, P.n_slots);
-  }
-  const unsigned nsb = unsigned(P.n_scan_blocks);
-  cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
-  cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
-  cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  if (d->topk % 4 == 0)
-    cc_fill4_kernel<<<unsigned((P.n_slots / 4 + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets,
-                                                                            e_pair, P.c, P.n_slots / 4);
-  else
-    cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
-                                                                       P.c, P.n_slots);
+  const int ix = launch_cc_index(P.c, P.rows, P.n_slots, P.n_scan_blocks, ids, scores, rowstat, counts, ranks, cbase,
+                                 offsets, tiles, items, sums, e_pair, st);
+  if (ix != HILS_OK) return ix;
   constexpr auto fn = cc_attend_kernel<D>;
   if (set_smem_max<fn>() != cudaSuccess) return HILS_ERR_CUDA;
   CcTcParams prm;
@@ -363,8 +388,8 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
 struct BwdPlan {
   CcDims c;
   int64_t rows, n_slots, max_items, n_scan_blocks, n_units;
-  size_t off_rowstat, off_dvec, off_counts, off_ranks, off_offsets, off_tiles, off_items, off_sums, off_epair,
-      off_dkp, off_dbp, total;
+  size_t off_rowstat, off_dvec, off_counts, off_ranks, off_cbase, off_offsets, off_tiles, off_items, off_sums,
+      off_epair, off_dkp, off_dbp, total;
 };
 
 BwdPlan bwd_plan(const hils_dims* d) {
@@ -382,6 +407,7 @@ BwdPlan bwd_plan(const hils_dims* d) {
   P.off_dvec = take(sizeof(float) * P.rows);
   P.off_counts = take(sizeof(int32_t) * P.c.n_keys);
   P.off_ranks = take(sizeof(int32_t) * P.n_slots);
+  P.off_cbase = take(sizeof(int32_t) * cc_cbase_entries(P.c, P.rows));
   P.off_offsets = take(sizeof(int64_t) * (P.c.n_keys + 1));
   P.off_tiles = take(sizeof(int32_t) * (P.c.n_keys + 1));
   P.off_items = take(sizeof(int4) * P.max_items);
@@ -405,6 +431,7 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   float* dvec = reinterpret_cast<float*>(base + P.off_dvec);
   int32_t* counts = reinterpret_cast<int32_t*>(base + P.off_counts);
   int32_t* ranks = reinterpret_cast<int32_t*>(base + P.off_ranks);
+  int32_t* cbase = reinterpret_cast<int32_t*>(base + P.off_cbase);
   int64_t* offsets = reinterpret_cast<int64_t*>(base + P.off_offsets);
   int32_t* tiles = reinterpret_cast<int32_t*>(base + P.off_tiles);
   int4* items = reinterpret_cast<int4*>(base + P.off_items);
@@ -430,24 +457,9 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   bwd_prep_kernel<T, D><<<unsigned((P.rows * 32 + 127) / 128), 128, 0, st>>>(
       ids, scores, lse_w, static_cast<const T*>(o), tdo, N, d->topk, P.c.wm1, P.rows, rowstat, dvec);
   // the forward's index: per (kv head, window, chunk) its (row, slot) pairs and s^ - M'
-  const size_t hist_bytes = sizeof(int32_t) * size_t(P.c.nc);
-  if (N % kCountRows == 0 && (int64_t(1) << P.c.win_shift) % kCountRows == 0 && hist_bytes <= 96 * 1024) {
-    constexpr auto cfn = cc_count_kernel;
-    if (hist_bytes > 48 * 1024 && set_smem_max<cfn>() != cudaSuccess) return HILS_ERR_CUDA;
-    cfn<<<unsigned(P.rows / kCountRows), kCountThreads, hist_bytes, st>>>(ids, counts, ranks, P.c);
-  } else {
-    cc_count_direct_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, counts, ranks, P.c, P.n_slots);
-  }
-  const unsigned nsb = unsigned(P.n_scan_blocks);
-  cc_scan_sums_kernel<<<nsb, 256, 0, st>>>(counts, P.c.n_keys, sums);
-  cc_scan_blocks_kernel<<<1, 1024, 0, st>>>(sums, P.n_scan_blocks, P.c.n_keys, offsets, tiles);
-  cc_scan_apply_kernel<<<nsb, 256, 0, st>>>(counts, P.c, sums, offsets, tiles, items);
-  if (d->topk % 4 == 0)
-    cc_fill4_kernel<<<unsigned((P.n_slots / 4 + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets,
-                                                                            e_pair, P.c, P.n_slots / 4);
-  else
-    cc_fill_kernel<<<unsigned((P.n_slots + 255) / 256), 256, 0, st>>>(ids, ranks, scores, rowstat, offsets, e_pair,
-                                                                       P.c, P.n_slots);
+  const int ix = launch_cc_index(P.c, P.rows, P.n_slots, P.n_scan_blocks, ids, scores, rowstat, counts, ranks, cbase,
+                                 offsets, tiles, items, sums, e_pair, st);
+  if (ix != HILS_OK) return ix;
   const float tau = 1.f / sqrtf(float(D));
   if (std::is_same<T, __nv_bfloat16>::value) {
     // bf16: the window branch's products on tensor cores

@@ -376,17 +376,20 @@ cc_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 // ---------------------------------------------------------------- pair counts
 // Each CTA takes kCountRows consecutive rows of one query head (inside one
-// window), counts their kept pairs per chunk in a shared-memory histogram,
-// then adds each touched chunk's count to the global per-key count with one
-// atomic, whose old value is the base of this CTA's pairs of that chunk.  A
-// pair's rank within its key is base + its rank in the histogram.  Ids outside
-// the row's candidates are recorded as HILS_ERR_DEVICE_BOUNDS and skipped.
+// window) and counts their kept pairs per chunk in a shared-memory histogram;
+// a pair's rank among the CTA's pairs of its chunk is the histogram's old
+// value.  Then each touched chunk's count goes to the global per-key count
+// with one atomic, whose old value -- the base of this CTA's pairs of that
+// chunk -- is stored in cbase[CTA][chunk].  A pair's position within its key
+// is cbase + its rank; the fill adds the two, so the ids and ranks are read
+// once here.  Ids outside the row's candidates are recorded as
+// HILS_ERR_DEVICE_BOUNDS and skipped.
 constexpr int kCountRows = 4096;
 constexpr int kCountThreads = 1024;
 
 __global__ void __launch_bounds__(kCountThreads)
 cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, int32_t* __restrict__ ranks,
-                const CcDims c) {
+                int32_t* __restrict__ cbase, const CcDims c) {
   extern __shared__ int32_t hist[];   // [nc]
   const int64_t row0 = int64_t(blockIdx.x) * kCountRows;   // rows of one (b, hq); kCountRows | n_tok
   const int64_t bhq = row0 / c.n_tok, i0 = row0 % c.n_tok;
@@ -418,45 +421,24 @@ cc_count_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ counts, i
       }
       rk4[t] = make_int4(r[0], r[1], r[2], r[3]);
     }
-    __syncthreads();
-    for (int64_t t = threadIdx.x; t < nch; t += blockDim.x) {
-      const int32_t h = hist[t];
-      hist[t] = h > 0 ? atomicAdd(counts + key0 + t, h) : 0;
+  } else {
+    for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
+      const int32_t ci = __ldg(id0 + t);
+      if (ci < 0) continue;
+      const int64_t i = i0 + t / c.K;
+      if (ci >= n_candidates(i, c.wm1)) {
+        record_error(HILS_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      rk0[t] = atomicAdd(hist + ci, 1);
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int64_t t = threadIdx.x; t < n4; t += blockDim.x) {
-      const int4 ci = __ldg(id4 + t);
-      const int64_t nc_i = n_candidates(i0 + (4 * t) / c.K, c.wm1);
-      int4 r = rk4[t];
-      if (ci.x >= 0 && ci.x < nc_i) r.x += hist[ci.x];
-      if (ci.y >= 0 && ci.y < nc_i) r.y += hist[ci.y];
-      if (ci.z >= 0 && ci.z < nc_i) r.z += hist[ci.z];
-      if (ci.w >= 0 && ci.w < nc_i) r.w += hist[ci.w];
-      rk4[t] = r;
-    }
-    return;
-  }
-  for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
-    const int32_t ci = __ldg(id0 + t);
-    if (ci < 0) continue;
-    const int64_t i = i0 + t / c.K;
-    if (ci >= n_candidates(i, c.wm1)) {
-      record_error(HILS_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    rk0[t] = atomicAdd(hist + ci, 1);
   }
   __syncthreads();
+  // chunks no pair of this CTA touched keep stale entries: no pair reads them
+  int32_t* cb = cbase + int64_t(blockIdx.x) * c.nc;
   for (int64_t t = threadIdx.x; t < nch; t += blockDim.x) {
     const int32_t h = hist[t];
-    hist[t] = h > 0 ? atomicAdd(counts + key0 + t, h) : 0;
-  }
-  __syncthreads();
-  for (int64_t t = threadIdx.x; t < n; t += blockDim.x) {
-    const int32_t ci = __ldg(id0 + t);
-    if (ci < 0 || ci >= n_candidates(i0 + t / c.K, c.wm1)) continue;
-    rk0[t] += hist[ci];
+    if (h > 0) cb[t] = atomicAdd(counts + key0 + t, h);
   }
 }
 
@@ -598,13 +580,15 @@ cc_scan_apply_kernel(const int32_t* __restrict__ counts, const CcDims c, const i
 }
 
 // ---------------------------------------------------------------- fill the inverted index
-// ranks[slot] is the slot's position within its key's list, taken when the
-// pair was counted, so filling is a plain scatter of the pair's global row id
-// and its fusion factor s^ - M'.
+// A pair's position within its key's list is known from the count: its rank
+// among its count CTA's pairs of the chunk (ranks[slot]) plus that CTA's base
+// for the chunk (cbase; null when the count took one global atomic per pair,
+// whose old value is the position itself), so filling is a plain scatter of
+// the pair's global row id and its fusion factor s^ - M'.
 __global__ void __launch_bounds__(256)
-cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const float* __restrict__ scores,
-               const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int2* __restrict__ e_pair,
-               const CcDims c, int64_t n_slots) {
+cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const int32_t* __restrict__ cbase,
+               const float* __restrict__ scores, const float* __restrict__ rowstat,
+               const int64_t* __restrict__ offsets, int2* __restrict__ e_pair, const CcDims c, int64_t n_slots) {
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n_slots) return;
   const int32_t ci = __ldg(ids + idx);
@@ -614,7 +598,8 @@ cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ rank
   if (ci >= n_candidates(i, c.wm1)) return;   // out of range: recorded when counting
   const int64_t b = bhq / c.Hq, hq = bhq % c.Hq;
   const int64_t bh = b * c.Hkv + hq / c.G;
-  const int64_t at = offsets[cc_key(c, bh, i, ci)] + __ldg(ranks + idx);
+  int64_t at = offsets[cc_key(c, bh, i, ci)] + __ldg(ranks + idx);
+  if (cbase) at += __ldg(cbase + (row / kCountRows) * c.nc + ci);
   // one 8-byte record per pair: the row and its fusion factor
   e_pair[at] = make_int2(int32_t(row), __float_as_int(__ldg(scores + idx) - __ldg(rowstat + row)));
 }
@@ -623,9 +608,9 @@ cc_fill_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ rank
 // 16-byte loads of ids, ranks and scores, one row statistic, and the four
 // independent offset loads in flight together.
 __global__ void __launch_bounds__(256)
-cc_fill4_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const float* __restrict__ scores,
-                const float* __restrict__ rowstat, const int64_t* __restrict__ offsets, int2* __restrict__ e_pair,
-                const CcDims c, int64_t n_quads) {
+cc_fill4_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ranks, const int32_t* __restrict__ cbase,
+                const float* __restrict__ scores, const float* __restrict__ rowstat,
+                const int64_t* __restrict__ offsets, int2* __restrict__ e_pair, const CcDims c, int64_t n_quads) {
   const int64_t qd = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (qd >= n_quads) return;
   const int64_t idx = qd * 4;
@@ -641,10 +626,13 @@ cc_fill4_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ ran
   const int32_t cv[4] = {ci.x, ci.y, ci.z, ci.w};
   const int32_t rv[4] = {rk.x, rk.y, rk.z, rk.w};
   const float sv[4] = {sc.x, sc.y, sc.z, sc.w};
+  const int32_t* cb = cbase ? cbase + (row / kCountRows) * c.nc : nullptr;
   int64_t at[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e)   // out-of-range ids were recorded when counting
-    at[e] = (cv[e] >= 0 && cv[e] < n_cand) ? offsets[cc_key(c, bh, i, cv[e])] + rv[e] : -1;
+  for (int e = 0; e < 4; ++e) {   // out-of-range ids were recorded when counting
+    const bool ok = cv[e] >= 0 && cv[e] < n_cand;
+    at[e] = ok ? offsets[cc_key(c, bh, i, cv[e])] + rv[e] + (cb ? __ldg(cb + cv[e]) : 0) : -1;
+  }
 #pragma unroll
   for (int e = 0; e < 4; ++e)
     if (at[e] >= 0) e_pair[at[e]] = make_int2(int32_t(row), __float_as_int(sv[e] - ms));
