@@ -71,6 +71,32 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
+// D[tmem] (+)= A[tmem] x B[smem desc]^T, bf16 inputs, fp32 accumulate.  A sits
+// in tensor memory: row m in lane m, its K elements in consecutive columns,
+// two bf16 per 32-bit column (the lower element in the low half).
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns from registers (thread t of the
+// warp writes lane (warp%4)*32 + t), then a wait until the stores are done.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+      "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // this thread's bulk groups except the newest n have finished reading shared memory
 template <int n>
@@ -699,10 +725,11 @@ cc_final_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ o, i
 //                every lane issues the gather4 loads of its four query rows
 //                (128B swizzle);
 //   warp 1       one lane issues S = Q K^T into TMEM buffer b, and once the
-//                softmax warps have written P, O = P V into TMEM buffer b,
-//                then releases the stage;
+//                softmax warps have written P, O = P V into TMEM buffer b
+//                (A = P from tensor memory), then releases the stage;
 //   warps 2-5    one thread per row: softmax of its 64 scores into P (bf16,
-//                over the stage's Q tile); the softmax of tile j+1 runs before
+//                over the row's own S columns in tensor memory, so no shared
+//                memory store and no proxy fence); the softmax of tile j+1 runs before
 //                tile j's output rows are staged in a separate padded buffer
 //                and added to the accumulator (one bulk reduction per row at
 //                d = 64, coalesced 16-byte reductions per warp row at d = 128).
@@ -717,16 +744,16 @@ struct CcTc {
   static constexpr uint32_t KV_ATOM = kChunk * 128; // 8 KB
   static constexpr uint32_t Q_BYTES = KATOMS * Q_ATOM;
   static constexpr uint32_t K_BYTES = KATOMS * KV_ATOM;
-  static constexpr uint32_t P_BYTES = M * 128;      // 128 rows x 64 keys bf16
-  // P overwrites the stage's Q tile once S = Q K^T is done; the stage goes
-  // back to the producer as soon as P V is done.  A separate buffer holds a
+  // P (bf16, two per 32-bit column) overwrites its own S columns in tensor
+  // memory and is the A operand of P V from there; the stage goes back to
+  // the producer as soon as P V is done.  A separate buffer holds a
   // tile's fp32 output rows (4D bytes each, padded to a 4D + 16 byte stride
   // so the row-per-thread stores of 8 consecutive rows hit distinct banks)
   // until the bulk reductions have read them.
   static constexpr uint32_t O_ROW = D * 4;
   static constexpr uint32_t O_STRIDE = O_ROW + 16;
   static constexpr uint32_t STAGE = Q_BYTES + 2 * K_BYTES;
-  static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES, OFF_P = 0;
+  static constexpr uint32_t OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + K_BYTES;
   static constexpr uint32_t OFF_O = NS * STAGE;
   static constexpr uint32_t O_BYTES = (M * O_STRIDE + 1023u) & ~1023u;
   static constexpr uint32_t OFF_META = OFF_O + O_BYTES;           // per stage: rows[128] i32, fac[128] f32, n
@@ -742,10 +769,9 @@ struct CcTc {
   static_assert((512 / TMEM_COLS + 1) * (SMEM + 1024) > 233472u, "TMEM never oversubscribed");
   static constexpr uint32_t TX_BYTES = M * D * 2 + 2 * K_BYTES;
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16(M, kChunk);
-  // P (K-major) x V (MN-major: d contiguous in each key row)
+  // P (in tensor memory, K-major) x V (MN-major: d contiguous in each key row)
   static constexpr uint32_t IDESC_O = sm100::idesc_bf16(M, D) | (1u << 16);
   static constexpr int THREADS = 192;
-  static_assert(P_BYTES <= Q_BYTES, "P reuses the Q tile");
 };
 
 struct CcTcParams {
@@ -889,7 +915,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!mbar_wait(&t_empty[b], (ub & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::STAGE);
-        const uint32_t sq = st + C::OFF_Q, sk = st + C::OFF_K, sv = st + C::OFF_V, sp = st + C::OFF_P;
+        const uint32_t sq = st + C::OFF_Q, sk = st + C::OFF_K, sv = st + C::OFF_V;
         const uint32_t t_s = tmem + uint32_t(b * kChunk), t_o = tmem + uint32_t(2 * kChunk + b * D);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -902,8 +928,8 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_bf16(t_o, desc_sw128(sp + kk * 32), desc_sw128_mn(sv + kk * 2048, C::KV_ATOM), C::IDESC_O,
-                   kk > 0 ? 1u : 0u);
+          mma_bf16_tmem_a(t_o, t_s + uint32_t(kk * 8), desc_sw128_mn(sv + kk * 2048, C::KV_ATOM), C::IDESC_O,
+                          kk > 0 ? 1u : 0u);
         mma_commit(&o_full[b]);
         mma_commit(&load_empty[s]);
       }
@@ -918,8 +944,8 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int r = quarter * 32 + lane;
     const uint32_t t_lane = uint32_t(quarter * 32) << 16;
     const float k2 = c.tau * 1.4426950408889634f;   // scores in log2 units
-    // softmax of tile jj: P into the stage (over its Q tile); returns the
-    // row's global row id (-1 when the row is not live) or -2 on abort
+    // softmax of tile jj: P into its own S columns in tensor memory; returns
+    // the row's global row id (-1 when the row is not live) or -2 on abort
     auto softmax_tile = [&](int jj) -> int64_t {
       const int s = jj % C::NS, u = jj / C::NS, b = jj & 1, ub = jj >> 1;
       if (!mbar_wait(&load_full[s], u & 1, abort_flag)) return -2;
@@ -940,7 +966,7 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int t = 0; t < 32; ++t) sc[32 + t] = tmp[t];
       }
-      uint8_t* prow = smem + s * C::STAGE + C::OFF_P + r * 128;
+      uint32_t pw[32];   // the row's P, two bf16 per word (zero when the row is not live)
       if (live) {
         // short dependency chains: a tree of three-input maxima, four partial sums
         float mx[22];
@@ -960,20 +986,16 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
         const float w = expf(fac) / l;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          uint32_t wd[4];
-#pragma unroll
-          for (int v2 = 0; v2 < 4; ++v2) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(sc[8 * t + 2 * v2] * w, sc[8 * t + 2 * v2 + 1] * w);
-            wd[v2] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-          *reinterpret_cast<uint4*>(prow + ((t ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        for (int t = 0; t < 32; ++t) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(sc[2 * t] * w, sc[2 * t + 1] * w);
+          pw[t] = *reinterpret_cast<uint32_t*>(&h2);
         }
       } else {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) *reinterpret_cast<uint4*>(prow + (t << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        for (int t = 0; t < 32; ++t) pw[t] = 0u;
       }
-      fence_proxy_async_smem();
+      // the whole warp, converged: S of this tile has been read into registers
+      tmem_st32(tmem + t_lane + uint32_t(b * kChunk), pw);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
