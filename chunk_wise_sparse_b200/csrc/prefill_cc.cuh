@@ -122,6 +122,33 @@ __device__ __forceinline__ float fmax3_f32(float a, float b, float c) {
   return d;
 }
 
+// Two fp32 lanes per instruction (sm_100), each rounded as its scalar form.
+__device__ __forceinline__ void fma2_f32(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                         float c1) {
+  asm("{\n\t.reg .b64 va, vb, vc, vd;\n\t"
+      "mov.b64 va, {%2, %3};\n\tmov.b64 vb, {%4, %5};\n\tmov.b64 vc, {%6, %7};\n\t"
+      "fma.rn.f32x2 vd, va, vb, vc;\n\t"
+      "mov.b64 {%0, %1}, vd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2_f32(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 va, vb, vd;\n\t"
+      "mov.b64 va, {%2, %3};\n\tmov.b64 vb, {%4, %5};\n\t"
+      "add.rn.f32x2 vd, va, vb;\n\t"
+      "mov.b64 {%0, %1}, vd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2_f32(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 va, vb, vd;\n\t"
+      "mov.b64 va, {%2, %3};\n\tmov.b64 vb, {%4, %5};\n\t"
+      "mul.rn.f32x2 vd, va, vb;\n\t"
+      "mov.b64 {%0, %1}, vd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -977,17 +1004,25 @@ cc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int t = 0; t < 7; ++t) mx[t] = fmax3_f32(mx[3 * t], mx[3 * t + 1], mx[3 * t + 2]);
         const float m = fmaxf(fmax3_f32(fmax3_f32(mx[0], mx[1], mx[2]), fmax3_f32(mx[3], mx[4], mx[5]), mx[6]), mx[21]);
         const float mb = m * k2;
+        // scores in pairs: one packed FMA, two exponentials, one packed add
+        // into four partial sums (lane pairs (0,1) and (2,3) of each 4 keys)
         float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < 64; ++t) {
-          sc[t] = ex2_approx(fmaf(sc[t], k2, -mb));
-          lp[t & 3] += sc[t];
+        for (int t = 0; t < 32; ++t) {
+          float x0, x1;
+          fma2_f32(x0, x1, sc[2 * t], sc[2 * t + 1], k2, k2, -mb, -mb);
+          sc[2 * t] = ex2_approx(x0);
+          sc[2 * t + 1] = ex2_approx(x1);
+          const int a = 2 * (t & 1);
+          add2_f32(lp[a], lp[a + 1], lp[a], lp[a + 1], sc[2 * t], sc[2 * t + 1]);
         }
         const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
         const float w = expf(fac) / l;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(sc[2 * t] * w, sc[2 * t + 1] * w);
+          float y0, y1;
+          mul2_f32(y0, y1, sc[2 * t], sc[2 * t + 1], w, w);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
           pw[t] = *reinterpret_cast<uint32_t*>(&h2);
         }
       } else {
