@@ -146,9 +146,10 @@ int hils_select(const hils_dims* dims, const void* q, const float* kprime, const
  * Device workspace bytes hils_attn_prefill needs for these dims (0 when the
  * call needs none: the fp32 path).  For bf16 it holds an fp32 output
  * accumulator (rows x d), the fusion normaliser of every row, the inverted
- * index of (row, slot) pairs per (kv head, window, chunk) and room for the
- * recomputed chunk scores of a call without scores: about
- * rows x (4d + 4 + 16K) bytes.
+ * index of (row, slot) pairs per (kv head, window, chunk), the pair count's
+ * per-(4096 rows, chunk) bases and room for the recomputed chunk scores of a
+ * call without scores: about rows x (4d + 4 + 16K + nc/1024) bytes, nc =
+ * seqlen / 64.
  */
 size_t hils_prefill_workspace_bytes(const hils_dims* dims);
 
