@@ -332,7 +332,8 @@ int launch_prefill_cc(const hils_dims* d, const void* q, const void* k, const vo
       !make_map_2d(&tk_own, k, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tv_own, v, D, kv_rows, D * 2, 64, nk_own, CU_TENSOR_MAP_SWIZZLE_128B))
     return HILS_ERR_CUDA;
-  int n_launch = 9;
+  // own (or local window), count, three scans, fill, attend, final
+  int n_launch = 8;
   if (scores == nullptr) {
     // no scores from the selection: recompute s^ of the kept ids
     float* rescore = reinterpret_cast<float*>(base + P.off_rescore);
@@ -500,7 +501,8 @@ int launch_backward(const hils_dims* d, const void* q, const void* q_score, cons
   if (set_smem_max<sfn>() != cudaSuccess) return HILS_ERR_CUDA;
   sfn<<<unsigned((P.n_units + 3) / 4), 128, smem_s, st>>>(tk, static_cast<const T*>(lq), kprime, dkp, dbp, N, P.c.nc,
                                                           P.n_units, tau, dk, dlq);
-  return launched(10);
+  // prep, count, three scans, fill, window, chunks, summary
+  return launched(9);
 }
 
 template <typename T, int D>
